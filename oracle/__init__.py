@@ -1,0 +1,211 @@
+"""CPU oracle for the decode-regime MoE layer (test infrastructure only).
+
+Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its binding) never imports, links or calls it.
+
+The arithmetic lives in ``moe_oracle.c`` (plain C, OpenMP); this module only
+compiles it with gcc and marshals numpy arrays through ctypes.  See
+``moe_oracle.h`` for the passages each function follows.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "moe_oracle.c")
+_HDR = os.path.join(_HERE, "moe_oracle.h")
+_SO = os.path.join(_HERE, "libmoe_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+WFMT_FP8 = 0
+WFMT_MXFP4 = 1
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle into ``oracle/libmoe_oracle.so`` (gcc, OpenMP)."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_HDR))
+    if not force and os.path.exists(_SO) and os.path.getmtime(_SO) >= newest:
+        return _SO
+    tmp = _SO + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp",
+           "-ffp-contract=off", "-fno-fast-math", "-Wall", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _SO)
+    return _SO
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int),
+                ("E", ctypes.c_int), ("k", ctypes.c_int), ("wfmt", ctypes.c_int),
+                ("n_shared", ctypes.c_int)]
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    with _lock:
+        if _lib is None:
+            build()
+            L = ctypes.CDLL(_SO)
+            vp = ctypes.c_void_p
+            L.orc_e4m3_decode.restype = ctypes.c_float
+            L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+            L.orc_e4m3_encode.restype = ctypes.c_uint8
+            L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+            L.orc_e2m1_decode.restype = ctypes.c_float
+            L.orc_e2m1_decode.argtypes = [ctypes.c_uint8]
+            L.orc_e8m0_decode.restype = ctypes.c_float
+            L.orc_e8m0_decode.argtypes = [ctypes.c_uint8]
+            L.orc_bf16_decode.restype = ctypes.c_float
+            L.orc_bf16_decode.argtypes = [ctypes.c_uint16]
+            L.orc_bf16_encode.restype = ctypes.c_uint16
+            L.orc_bf16_encode.argtypes = [ctypes.c_float]
+            for name in ("orc_e4m3_decode_n", "orc_e4m3_encode_n", "orc_e2m1_decode_n"):
+                getattr(L, name).restype = None
+                getattr(L, name).argtypes = [vp, vp, ctypes.c_int64]
+            L.orc_route.restype = ctypes.c_int
+            L.orc_route.argtypes = [ctypes.c_int] * 4 + [vp] * 5
+            L.orc_quant_act.restype = None
+            L.orc_quant_act.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
+            L.orc_quant_row_f32.restype = None
+            L.orc_quant_row_f32.argtypes = [ctypes.c_int, vp, vp, vp]
+            L.orc_forward.restype = ctypes.c_int
+            L.orc_forward.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 13
+            L.orc_num_threads.restype = ctypes.c_int
+            L.orc_num_threads.argtypes = []
+            _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+def num_threads() -> int:
+    return lib().orc_num_threads()
+
+
+# ---- codecs ---------------------------------------------------------------
+def e4m3_decode(codes) -> np.ndarray:
+    c = _c(np.asarray(codes, dtype=np.uint8), np.uint8)
+    out = np.empty(c.shape, np.float32)
+    lib().orc_e4m3_decode_n(_p(c), _p(out), c.size)
+    return out
+
+
+def e4m3_encode(values) -> np.ndarray:
+    v = _c(np.asarray(values, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e4m3_encode_n(_p(v), _p(out), v.size)
+    return out
+
+
+def e2m1_decode(nibbles) -> np.ndarray:
+    c = _c(np.asarray(nibbles, dtype=np.uint8), np.uint8)
+    out = np.empty(c.shape, np.float32)
+    lib().orc_e2m1_decode_n(_p(c), _p(out), c.size)
+    return out
+
+
+def e8m0_decode(code: int) -> float:
+    return float(lib().orc_e8m0_decode(code))
+
+
+def bf16_decode(bits: int) -> float:
+    return float(lib().orc_bf16_decode(bits))
+
+
+def bf16_encode(v: float) -> int:
+    return int(lib().orc_bf16_encode(v))
+
+
+# ---- steps ----------------------------------------------------------------
+def route(ids: np.ndarray, E: int, n_shared: int = 0):
+    """Counting sort of slots by expert.  Returns (counts, offsets, perm, inv, dropped)."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    S = T * k
+    P = S + n_shared * T
+    counts = np.empty(E + n_shared, np.int32)
+    offsets = np.empty(E + n_shared + 1, np.int32)
+    perm = np.empty(max(P, 1), np.int32)
+    inv = np.empty(max(P, 1), np.int32)
+    dropped = lib().orc_route(T, k, E, n_shared, _p(ids), _p(counts), _p(offsets),
+                              _p(perm), _p(inv))
+    return counts, offsets, perm[:P], inv[:P], dropped
+
+
+def quant_act(x_bf16_bits: np.ndarray):
+    """x as uint16 bf16 bits [T,H] -> (xq uint8 [T,H], xs float32 [T,H/128])."""
+    x = _c(x_bf16_bits, np.uint16)
+    T, H = x.shape
+    xq = np.empty((T, H), np.uint8)
+    xs = np.empty((T, H // 128), np.float32)
+    lib().orc_quant_act(T, H, _p(x), _p(xq), _p(xs))
+    return xq, xs
+
+
+def quant_row_f32(v: np.ndarray):
+    v = _c(v, np.float32)
+    (K,) = v.shape
+    q = np.empty(K, np.uint8)
+    s = np.empty(K // 128, np.float32)
+    lib().orc_quant_row_f32(K, _p(v), _p(q), _p(s))
+    return q, s
+
+
+def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
+            n_shared=0, token_mask=None, debug=False):
+    """Whole layer on the CPU.
+
+    Returns a dict with ``out_f32`` [T,H], ``out_bf16`` (uint16 bits) [T,H],
+    ``dropped`` and, with ``debug``, ``xq``/``xs`` per token and ``hq``/``hs``
+    per routed position.  Rows of unselected tokens are NaN / 0.
+    """
+    x = _c(x_bf16_bits, np.uint16)
+    ids = _c(ids, np.int32)
+    topk_w = _c(topk_w, np.float32)
+    T, k = ids.shape
+    assert x.shape == (T, H)
+    S = T * k
+    P = S + n_shared * T
+    d = _Dims(T, H, I, E, k, wfmt, n_shared)
+    w13 = np.ascontiguousarray(w13)
+    s13 = np.ascontiguousarray(s13)
+    w2 = np.ascontiguousarray(w2)
+    s2 = np.ascontiguousarray(s2)
+    mask = None
+    if token_mask is not None:
+        mask = _c(np.asarray(token_mask, dtype=np.uint8), np.uint8)
+        assert mask.shape == (T,)
+    out_f32 = np.full((T, H), np.nan, np.float32)
+    out_bf16 = np.zeros((T, H), np.uint16)
+    dbg = {}
+    if debug:
+        dbg = dict(xq=np.zeros((T, H), np.uint8), xs=np.zeros((T, H // 128), np.float32),
+                   hq=np.zeros((max(P, 1), I), np.uint8),
+                   hs=np.zeros((max(P, 1), I // 128), np.float32))
+    rc = lib().orc_forward(ctypes.byref(d), _p(x), _p(ids), _p(topk_w), _p(w13), _p(s13),
+                           _p(w2), _p(s2), _p(mask), _p(out_f32), _p(out_bf16),
+                           _p(dbg.get("xq")), _p(dbg.get("xs")), _p(dbg.get("hq")),
+                           _p(dbg.get("hs")))
+    if rc < 0:
+        raise ValueError("oracle rejected the arguments")
+    res = dict(out_f32=out_f32, out_bf16=out_bf16, dropped=rc)
+    if debug:
+        dbg["hq"] = dbg["hq"][:P]
+        dbg["hs"] = dbg["hs"][:P]
+        res.update(dbg)
+    return res

@@ -1,0 +1,108 @@
+/*
+ * moe_oracle.h -- plain, slow CPU oracle for the decode-regime MoE layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path may include, link or
+ * call this file: only the tests, the smoke check and the benchmark's CPU
+ * baseline leg use it.  It shares no code, header, table or constant with the
+ * CUDA library.
+ *
+ * What it computes (sources):
+ *  - "GC-MoE: Overlapping Expert-Parallel Token Dispatch with FP8/FP4 Grouped
+ *    GEMM via CUDA Green Contexts", abstract: per layer, token dispatch to
+ *    experts, grouped GEMMs on FP8/FP4 block-scaled weights, fused SwiGLU with
+ *    requantisation, optional shared experts, and a combine step.
+ *  - FusedDeepMoE unified-execution-flow page (Ascend fused family analysis):
+ *    QuantToken (per-token dynamic activation quantisation), OpDequant
+ *    (accumulator x weight scale x per-token scale), OpSwiglu (gate = first
+ *    half, x_left * sigmoid(x_left) * x_right), OpBlockQuant (abs -> max ->
+ *    scale -> quant of the SwiGLU output), OpCombineSend / ReducePermute
+ *    (prefix-summed per-expert ranges, accumulate expert outputs per token),
+ *    and the shared-expert rank that treats all tokens as one group.
+ *  - Number formats, which the pages name but do not define: OCP 8-bit
+ *    floating point spec (E4M3, "e4m3fn": bias 7, no infinities, S.1111.111 is
+ *    NaN, max 448) and OCP Microscaling (MX) v1.0 (E2M1 elements, E8M0 shared
+ *    scale per 32 elements, 0xFF = NaN).
+ *
+ * Precision: fp32 arithmetic throughout (the layer's own accumulate and
+ * scale precision), partial sums of one 128-wide K block in ascending k,
+ * blocks promoted in ascending order.  No blocking or reordering beyond that.
+ *
+ * Parity pins live in tests/test_oracle_pins.py (codec tables against torch's
+ * float8 dtype and the OCP tables, routing against numpy's stable argsort,
+ * the one-expert/dense-FFN reduction, fp64 brute force on tiny shapes,
+ * linearity in the combine weights, zero input).
+ */
+#ifndef MOE_ORACLE_H
+#define MOE_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1 };
+
+/* ---- codecs (OCP FP8 / OCP MX v1.0) ---------------------------------- */
+float   orc_e4m3_decode(uint8_t code);          /* exact value, NaN for S.1111.111 */
+uint8_t orc_e4m3_encode(float v);               /* round-to-nearest-even, saturate to +-448 */
+float   orc_e2m1_decode(uint8_t nibble);        /* low 4 bits used */
+float   orc_e8m0_decode(uint8_t code);          /* 2^(code-127), NaN for 0xFF */
+float   orc_bf16_decode(uint16_t bits);
+uint16_t orc_bf16_encode(float v);              /* round-to-nearest-even */
+
+/* Vector forms for the tests (n elements). */
+void orc_e4m3_decode_n(const uint8_t* in, float* out, int64_t n);
+void orc_e4m3_encode_n(const float* in, uint8_t* out, int64_t n);
+void orc_e2m1_decode_n(const uint8_t* in, float* out, int64_t n);
+
+/* ---- step 1: routing (counting sort of slots by expert) -------------- */
+/* ids [T*k] expert ids, slot s = t*k + j.  With n_shared == 1 the shared
+ * expert is group E holding every token t as virtual slot S + t.
+ * Outputs: counts [E+n_shared], offsets [E+n_shared+1] (exclusive scan,
+ * routed groups first), perm [S + n_shared*T] (position -> slot),
+ * inv [S + n_shared*T] (slot -> position, -1 for a dropped slot).
+ * Returns the number of slots dropped because their id is outside [0,E). */
+int orc_route(int T, int k, int E, int n_shared, const int32_t* ids,
+              int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv);
+
+/* ---- step 2: per-token, per-128-column activation quantisation ------- */
+/* x bf16 [T,H] -> xq E4M3 [T,H], xs fp32 [T,H/128] with s = amax/448
+ * (s = 1 when the group is all zero) and q = e4m3(x / s). */
+void orc_quant_act(int T, int H, const uint16_t* x, uint8_t* xq, float* xs);
+
+/* Same rule on an fp32 row (used for the SwiGLU output requantisation). */
+void orc_quant_row_f32(int K, const float* v, uint8_t* q, float* s);
+
+/* ---- steps 1-8: the whole layer -------------------------------------- */
+typedef struct {
+  int T, H, I, E, k;
+  int wfmt;       /* ORC_WFMT_FP8 or ORC_WFMT_MXFP4 */
+  int n_shared;   /* 0 or 1: shared expert stored as expert index E */
+} orc_dims;
+
+/* Weight layouts (row-major, K contiguous), NE = E + n_shared experts:
+ *  FP8:   w13 u8 [NE, 2I, H] (rows 0..I-1 gate, I..2I-1 up), s13 f32 [NE, 2I/128, H/128]
+ *         w2  u8 [NE, H, I],                               s2  f32 [NE, H/128, I/128]
+ *  MXFP4: w13 u8 [NE, 2I, H/2] (element 2c in the low nibble of byte c),
+ *         s13 u8 E8M0 [NE, 2I, H/32]; w2 u8 [NE, H, I/2], s2 u8 [NE, H, I/32]
+ * token_mask [T] (1 = compute this token) or NULL for all tokens.
+ * Outputs for masked-in tokens: out_f32 [T,H] fp32 combine result and
+ * out_bf16 [T,H] its bf16 rounding (either may be NULL).  Other rows are
+ * left untouched.  Optional debug outputs (NULL to skip): xq/xs per token
+ * [T,H] / [T,H/128]; hq/hs per slot position (routing order of orc_route)
+ * [S + n_shared*T, I] / [.., I/128].
+ * Returns the number of dropped slots (as orc_route), or -1 on bad arguments. */
+int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
+                const float* topk_w, const void* w13, const void* s13,
+                const void* w2, const void* s2, const uint8_t* token_mask,
+                float* out_f32, uint16_t* out_bf16,
+                uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs);
+
+/* OpenMP threads the oracle will use (1 when built without OpenMP). */
+int orc_num_threads(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
