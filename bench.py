@@ -1,0 +1,435 @@
+#!/usr/bin/env python
+"""Benchmark of the decode-regime MoE layer on B200.
+
+One step = one full MoE layer (route, activation quant, GEMM1 + SwiGLU +
+requant, GEMM2 + weighted combine, bf16 output) over one batch of seeded
+synthetic inputs, through the C ABI.  Default workload: the FP8 decode layer
+T=32, H=7168, E=256, top-k=8, I=2048.  Metric: weight-stream GB/s (bytes of
+the weights and scales of every expert the step touches, divided by the step
+time); microseconds per layer and TFLOP/s ride along.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload IDX] [--impl reference]
+
+With N > 1 (launched by torchrun) every rank runs an independent replica of
+the layer on its own GPU (the single-GPU path has no exchange step); the
+value is the sum over ranks of the bytes streamed divided by the slowest
+rank's time.  Rank 0 prints one JSON line on stdout.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MoE layer µs and weight-stream HBM GB/s (vs ~8 TB/s) at T=1–256; TFLOP/s at T=4096"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+GEMM_SOURCES = ["fp4_block_scaled_route_b200/csrc/moe_gemm.cu", "fp4_block_scaled_route_b200/csrc/moe_ptx.cuh"]
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ---------------------------------------------------------------------------
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", type=int, default=1, help="index into synth.CONFIGS")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for rel in GEMM_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name: str):
+    """Per-launch DRAM bytes of the GEMM1 kernel from the committed ncu summary,
+    or None when there is none or the kernel sources changed since."""
+    path = os.path.join(ROOT, "profiles", f"gemm1_{workload_name}_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith("#"):
+                k, v = line.split(":", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_source_sha256_16") != gemm_source_hash():
+        return None
+    try:
+        return float(vals["dram_bytes_per_launch_full_size"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str | None):
+        self.lines = []
+        self.proc = None
+        try:
+            cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+            if gpu_id:
+                cmd += ["-i", gpu_id]
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def wait_first(self, timeout=3.0):
+        t0 = time.time()
+        while self.proc and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=2)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [l for (t, l) in self.lines if t0 <= t <= t1]
+        if not rows:
+            rows = [l for (t, l) in self.lines if t0 - 0.1 <= t <= t1 + 0.1]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            parts = [p.strip() for p in r.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def gpu_uuid(dev):
+    import torch
+    try:
+        u = str(torch.cuda.get_device_properties(dev).uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------------
+def weight_bytes_per_expert(L) -> int:
+    H, I = L.H, L.I
+    if L.wfmt == 0:
+        return 2 * I * H + (2 * I // 128) * (H // 128) * 4 + H * I + (H // 128) * (I // 128) * 4
+    return 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
+
+
+def gemm1_weight_bytes_per_expert(L) -> int:
+    H, I = L.H, L.I
+    if L.wfmt == 0:
+        return 2 * I * H + (2 * I // 128) * (H // 128) * 4
+    return 2 * I * H // 2 + 2 * I * H // 32
+
+
+def touched_experts(ids: np.ndarray, E: int) -> int:
+    v = ids[(ids >= 0) & (ids < E)]
+    return int(np.unique(v).size)
+
+
+def workload_stats(L, ids_np):
+    n_exp = touched_experts(ids_np, L.E) + L.n_shared
+    P = L.T * L.k + L.n_shared * L.T
+    wbytes = n_exp * weight_bytes_per_expert(L)
+    flops = 2.0 * P * 3 * L.I * L.H
+    g1 = n_exp * gemm1_weight_bytes_per_expert(L) + P * L.H + P * (L.H // 128) * 4 + P * L.I + P * (L.I // 128) * 4
+    return dict(experts_touched=n_exp, weight_bytes=wbytes, flops=flops, gemm1_bytes=g1, positions=P)
+
+
+def build_layer(cfg_idx, device):
+    from fp4_block_scaled_route_b200 import moe, synth
+    cfg = synth.CONFIGS[cfg_idx]
+    L = synth.make_layer(cfg, synth.config_seed(cfg_idx), device=device)
+    return cfg, L
+
+
+# ---------------------------------------------------------------------------
+def cpu_baseline_sample(L, n_slots: int):
+    """Oracle on the first n_slots (token, expert) pairs of the workload."""
+    import oracle
+    import torch
+    from fp4_block_scaled_route_b200 import synth
+    ids = L.ids.cpu().numpy()
+    w = L.topk_w.cpu().numpy()
+    slots = [(t, j) for t in range(L.T) for j in range(L.k)][:n_slots]
+    experts = sorted({int(ids[t, j]) for (t, j) in slots})
+    idx = torch.tensor(experts, device=L.w13.device)
+    pick = lambda a: a.index_select(0, idx).cpu().numpy()
+    w13, s13, w2, s2 = pick(L.w13), pick(L.s13), pick(L.w2), pick(L.s2)
+    remap = {e: i for i, e in enumerate(experts)}
+    toks = sorted({t for (t, _) in slots})
+    x = synth.bf16_bits(L.x[toks])
+    ids_s = np.full((len(toks), L.k), -1, np.int32)
+    w_s = np.zeros((len(toks), L.k), np.float32)
+    for (t, j) in slots:
+        ids_s[toks.index(t), j] = remap[int(ids[t, j])]
+        w_s[toks.index(t), j] = w[t, j]
+    t0 = time.perf_counter()
+    oracle.forward(x, ids_s, w_s, w13, s13, w2, s2, H=L.H, I=L.I, E=len(experts), wfmt=L.wfmt, n_shared=0)
+    dt = time.perf_counter() - t0
+    nbytes = len(experts) * weight_bytes_per_expert(L)
+    return dt, nbytes, len(experts), oracle.num_threads()
+
+
+def run_reference(args):
+    """The oracle, as it stands, on the host cores (rank 0 only)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+    from fp4_block_scaled_route_b200 import synth
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    cfg, L = build_layer(args.workload, dev)
+    # per step: one (token, expert) slot, the smallest unit of the workload
+    times, nb = [], 0
+    for i in range(args.warmup + args.steps):
+        dt, nbytes, _, cores = cpu_baseline_sample(L, 1)
+        if i >= args.warmup:
+            times.append(dt)
+            nb += nbytes
+    total = sum(times)
+    value = nb / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic (seeded)",
+        "config": {"workload": cfg["name"], "T": cfg["T"], "H": cfg["H"], "E": cfg["E"], "k": cfg["k"],
+                   "I": cfg["I"], "wfmt": ["fp8", "mxfp4"][cfg["wfmt"]], "parallelism": "replicas"},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": "per step one (token, expert) slot of the workload: one expert FFN on one token"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    from fp4_block_scaled_route_b200 import build as moe_build
+    from fp4_block_scaled_route_b200 import moe, synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        moe_build.build()
+    if dist:
+        dist.barrier()
+
+    cfg, L = build_layer(args.workload, dev)
+    ids_np = L.ids.cpu().numpy()
+    st = workload_stats(L, ids_np)
+    layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
+    if L.wfmt == synth.WFMT_MXFP4:
+        w13, s13, w2, s2 = L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2)
+    else:
+        w13, s13, w2, s2 = L.w13, L.s13, L.w2, L.s2
+    out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        layer.forward(L.x, L.ids, L.topk_w, w13, s13, w2, s2, out=out, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if layer.device_status() != moe.MOE_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    # ---- timed region (device events, max over ranks) ----
+    sampler = ClockSampler(gpu_uuid(dev))
+    sampler.wait_first()
+    moe.moe_profile_enable(layer.ctx, 1)
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    tw0 = time.time()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    tw1 = time.time()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
+    moe.moe_profile_enable(layer.ctx, 0)
+    clocks = sampler.summary(tw0, tw1)
+    sampler.stop()
+    if layer.device_status() != moe.MOE_OK:
+        raise RuntimeError("device status not OK after the timed region")
+    if dist:
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_step = ms / args.steps
+    value = world * st["weight_bytes"] / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end through the C ABI with host buffers ----
+    e2e = None
+    if not args.no_e2e:
+        x_h = L.x.cpu().pin_memory()
+        ids_h = L.ids.cpu().pin_memory()
+        w_h = L.topk_w.cpu().pin_memory()
+        out_h = torch.empty(L.T, L.H, dtype=torch.bfloat16).pin_memory()
+        x_d, ids_d, w_d = torch.empty_like(L.x), torch.empty_like(L.ids), torch.empty_like(L.topk_w)
+
+        def step_e2e():
+            x_d.copy_(x_h, non_blocking=True)
+            ids_d.copy_(ids_h, non_blocking=True)
+            w_d.copy_(w_h, non_blocking=True)
+            layer.forward(x_d, ids_d, w_d, w13, s13, w2, s2, out=out, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+
+        for _ in range(3):
+            step_e2e()
+        torch.cuda.synchronize(dev)
+        if dist:
+            dist.barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step_e2e()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        ms_e = ev0.elapsed_time(ev1)
+        if dist:
+            t = torch.tensor([ms_e], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms_e = float(t.item())
+        h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
+        e2e = {"value": world * st["weight_bytes"] / (ms_e / args.steps * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_h.numel() * 2,
+               "ms_per_step": ms_e / args.steps}
+
+    # ---- roofline of the dominant kernel (GEMM1 + SwiGLU + requant) ----
+    hbm_peak, bf16_peak, peak_src = peaks()
+    g1_ms = stage_ms[2]
+    g1_gbs = st["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9 if g1_ms > 0 else None
+    roofline = {"kernel": "moe_gemm_kernel<GEMM1> (grouped GEMM1 + SwiGLU + FP8 requant)", "bound": "hbm",
+                "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
+                "frac": (g1_gbs / hbm_peak) if g1_gbs else None,
+                "traffic": recorded_traffic(cfg["name"]),
+                "algorithmic_bytes_per_launch": st["gemm1_bytes"], "avg_launch_ms": g1_ms,
+                "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
+                "launches_timed": ncalls}
+
+    if dist:
+        dist.barrier()
+    if rank != 0:
+        if dist:
+            dist.destroy_process_group()
+        return
+
+    cpu = None
+    if world == 1 and not args.no_cpu_baseline:
+        dt, nbytes, nexp, cores = cpu_baseline_sample(L, 2 * L.k)
+        cpu = {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": f"first {2 * L.k} (token, expert) slots of the workload ({nexp} expert FFNs, "
+                         f"{nbytes / 1e9:.2f} GB of weights), timed once",
+               "seconds": dt}
+
+    frac_step = value / world / hbm_peak
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if L.wfmt == 0 else "mxfp4_e2m1 x fp8_e4m3",
+        "data": "synthetic (seeded: x~N(0,1) bf16, uniform/zipf top-k, weights N(0,0.02) quantised)",
+        "config": {"workload": cfg["name"], "T": L.T, "H": L.H, "E": L.E, "k": L.k, "I": L.I,
+                   "wfmt": ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32"][L.wfmt], "n_shared": L.n_shared,
+                   "experts_touched": st["experts_touched"], "weight_bytes_per_step": st["weight_bytes"],
+                   "l2": "inputs larger than L2 (weights streamed per step exceed the 126 MB L2); no flush",
+                   "parallelism": "replicas" if world > 1 else "single GPU"},
+        "us_per_layer": ms_step * 1e3,
+        "tflops": st["flops"] / (ms_step * 1e-3) / 1e12,
+        "hbm_frac_of_step": frac_step,
+        "stage_ms": dict(zip(moe.STAGE_NAMES, stage_ms)),
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": moe.MOE_NUM_STAGES * args.steps,
+        "clocks": clocks,
+    }
+    print(json.dumps(line), flush=True)
+    if dist:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

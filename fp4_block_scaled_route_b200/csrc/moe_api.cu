@@ -1,0 +1,389 @@
+// moe_api.cu -- the C ABI (include/moe.h): context, workspace, tensor maps
+// and the launch sequence of one MoE layer.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "moe.h"
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+using moe::GemmParams;
+using moe::QuantParams;
+using moe::RouteParams;
+
+struct moe_ctx {
+  int H, I, E, k, wfmt, max_T, n_shared, NG;
+  int dev, num_sms;
+  int S_max, P_max, S_pad, max_tiles;
+  void* ws_base;
+  int32_t *counts, *offsets, *perm, *inv, *num_tiles, *status;
+  int4* tiles;
+  uint8_t *xq, *hq;
+  float *xs, *hs, *out_acc;
+  // tensor-map cache
+  const void* c_w13;
+  const void* c_w2;
+  int c_bn;
+  CUtensorMap tm_w13, tm_w2, tm_xq, tm_hq;
+  // last call
+  int last_T, last_bn, last_grid;
+  // profiling: events[call][stage boundary]
+  int prof_on, prof_calls;
+  cudaEvent_t* prof_ev;
+};
+
+namespace {
+constexpr int kProfMaxCalls = 4096;
+constexpr int kProfEvents = MOE_NUM_STAGES + 1;
+}
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D map over a row-major matrix [rows, inner] (inner contiguous), box
+// {128 elements, box_rows}, 128-byte swizzle.
+bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
+              uint64_t row_bytes, uint32_t box_rows, CUtensorMapL2promotion l2) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gdim[2] = {inner, rows};
+  cuuint64_t gstride[1] = {row_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int pick_tile_n(const moe_ctx* c, int T) {
+  const double avg = (double)T * c->k / c->E;  // expected tokens per routed expert
+  int bn = avg <= 8 ? 16 : avg <= 20 ? 32 : avg <= 48 ? 64 : 128;
+  if (c->wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 && bn > 64) bn = 64;
+  return bn;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported shape, format or device";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_NO_MEMORY: return "out of device memory";
+    case MOE_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case MOE_ERR_BAD_ROUTING: return "expert id out of range (slot dropped)";
+  }
+  return "unknown status";
+}
+
+moe_status moe_create(int H, int I, int E, int k, int wfmt, moe_ctx** out) {
+  return moe_create_ex(H, I, E, k, wfmt, 4096, 0, out);
+}
+
+moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_shared, moe_ctx** out) {
+  if (!out) return MOE_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || max_T <= 0 || n_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (H % 128 || I % 128 || H > 8192 || I > 8192 || E > 1024 || k > moe::kMaxK || n_shared > 1)
+    return MOE_ERR_UNSUPPORTED;
+  if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32) return MOE_ERR_UNSUPPORTED;
+  if ((long long)max_T * (k + n_shared) > (1LL << 26)) return MOE_ERR_UNSUPPORTED;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  int major = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (major != 10) return MOE_ERR_UNSUPPORTED;
+  if (!encode_fn()) return MOE_ERR_CUDA;
+  if (moe::gemm_setup(wfmt) != cudaSuccess) return MOE_ERR_CUDA;
+
+  moe_ctx* c = new (std::nothrow) moe_ctx();
+  if (!c) return MOE_ERR_NO_MEMORY;
+  c->H = H; c->I = I; c->E = E; c->k = k; c->wfmt = wfmt; c->max_T = max_T; c->n_shared = n_shared;
+  c->NG = E + n_shared;
+  c->dev = dev;
+  c->num_sms = sms;
+  c->S_max = max_T * k;
+  c->P_max = c->S_max + n_shared * max_T;
+  c->S_pad = c->P_max + 128;
+  c->max_tiles = c->P_max / 16 + c->NG + 1;
+
+  const size_t HB = H / 128, IB = I / 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  const size_t o_counts = take(sizeof(int32_t) * c->NG);
+  const size_t o_offsets = take(sizeof(int32_t) * (c->NG + 1));
+  const size_t o_perm = take(sizeof(int32_t) * c->P_max);
+  const size_t o_inv = take(sizeof(int32_t) * c->P_max);
+  const size_t o_ntiles = take(sizeof(int32_t) * 4);
+  const size_t o_status = take(sizeof(int32_t) * 4);
+  const size_t o_tiles = take(sizeof(int4) * c->max_tiles);
+  const size_t o_xq = take((size_t)c->S_pad * H);
+  const size_t o_hq = take((size_t)c->S_pad * I);
+  const size_t o_xs = take(sizeof(float) * (size_t)c->S_pad * HB);
+  const size_t o_hs = take(sizeof(float) * (size_t)c->S_pad * IB);
+  const size_t o_acc = take(sizeof(float) * (size_t)max_T * H);
+  void* base = nullptr;
+  if (cudaMalloc(&base, off) != cudaSuccess) {
+    delete c;
+    cudaGetLastError();
+    return MOE_ERR_NO_MEMORY;
+  }
+  if (cudaMemset(base, 0, off) != cudaSuccess) {
+    cudaFree(base);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
+  char* b = static_cast<char*>(base);
+  c->ws_base = base;
+  c->counts = reinterpret_cast<int32_t*>(b + o_counts);
+  c->offsets = reinterpret_cast<int32_t*>(b + o_offsets);
+  c->perm = reinterpret_cast<int32_t*>(b + o_perm);
+  c->inv = reinterpret_cast<int32_t*>(b + o_inv);
+  c->num_tiles = reinterpret_cast<int32_t*>(b + o_ntiles);
+  c->status = reinterpret_cast<int32_t*>(b + o_status);
+  c->tiles = reinterpret_cast<int4*>(b + o_tiles);
+  c->xq = reinterpret_cast<uint8_t*>(b + o_xq);
+  c->hq = reinterpret_cast<uint8_t*>(b + o_hq);
+  c->xs = reinterpret_cast<float*>(b + o_xs);
+  c->hs = reinterpret_cast<float*>(b + o_hs);
+  c->out_acc = reinterpret_cast<float*>(b + o_acc);
+  *out = c;
+  return MOE_OK;
+}
+
+static void prof_free(moe_ctx* c) {
+  if (!c->prof_ev) return;
+  for (int i = 0; i < kProfMaxCalls * kProfEvents; ++i) cudaEventDestroy(c->prof_ev[i]);
+  delete[] c->prof_ev;
+  c->prof_ev = nullptr;
+}
+
+void moe_destroy(moe_ctx* c) {
+  if (!c) return;
+  cudaDeviceSynchronize();
+  prof_free(c);
+  cudaFree(c->ws_base);
+  delete c;
+}
+
+moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w, const void* w13,
+                       const void* s13, const void* w2, const void* s2, void* out, void* stream) {
+  if (!c || T < 0 || T > c->max_T) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  if (!x || !ids || !topk_w || !w13 || !s13 || !w2 || !s2 || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(w13, 128) || !aligned(w2, 128) || !aligned(s13, 16) ||
+      !aligned(s2, 16) || !aligned(ids, 4) || !aligned(topk_w, 4))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int H = c->H, I = c->I, NE = c->NG;
+  const int S = T * c->k;
+  const int BN = pick_tile_n(c, T);
+  const int grid = c->num_sms;
+  const bool fp8 = (c->wfmt == MOE_WFMT_FP8_E4M3_B128);
+
+  // weight maps (re-encoded only when the caller's pointers change)
+  if (w13 != c->c_w13) {
+    const bool ok = fp8 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H, (uint64_t)NE * 2 * I, H, 128,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                        : make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13, H, (uint64_t)NE * 2 * I,
+                                   H / 2, 128, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (!ok) {
+      c->c_w13 = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    c->c_w13 = w13;
+  }
+  if (w2 != c->c_w2) {
+    const bool ok = fp8 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I, (uint64_t)NE * H, I, 128,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                        : make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2, I, (uint64_t)NE * H, I / 2,
+                                   128, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+    if (!ok) {
+      c->c_w2 = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    c->c_w2 = w2;
+  }
+  if (BN != c->c_bn) {
+    if (!make_map(&c->tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H, c->S_pad, H, BN,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !make_map(&c->tm_hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hq, I, c->S_pad, I, BN,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
+      c->c_bn = 0;
+      return MOE_ERR_CUDA;
+    }
+    c->c_bn = BN;
+  }
+
+  cudaEvent_t* ev = nullptr;
+  if (c->prof_on && c->prof_calls < kProfMaxCalls) ev = c->prof_ev + (size_t)c->prof_calls++ * kProfEvents;
+  auto mark = [&](int i) {
+    if (ev) cudaEventRecord(ev[i], s);
+  };
+
+  RouteParams rp;
+  rp.T = T; rp.k = c->k; rp.E = c->E; rp.n_shared = c->n_shared; rp.BN = BN;
+  rp.ids = ids; rp.counts = c->counts; rp.offsets = c->offsets; rp.perm = c->perm; rp.inv = c->inv;
+  rp.tiles = c->tiles; rp.num_tiles = c->num_tiles; rp.status = c->status;
+  mark(MOE_STAGE_ROUTE);
+  if (moe::launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  QuantParams qp;
+  qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
+  qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs; qp.out_acc = c->out_acc;
+  mark(MOE_STAGE_QUANT);
+  if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  GemmParams g;
+  g.H = H; g.I = I; g.k = c->k; g.S = S;
+  g.kblocks = H / 128;
+  g.wscale = static_cast<const float*>(s13);
+  g.ascale = c->xs;
+  g.hq = c->hq; g.hs = c->hs;
+  g.perm = c->perm; g.topk_w = topk_w; g.out_acc = c->out_acc;
+  g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
+  mark(MOE_STAGE_GEMM1);
+  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  g.kblocks = I / 128;
+  g.wscale = static_cast<const float*>(s2);
+  g.ascale = c->hs;
+  mark(MOE_STAGE_GEMM2);
+  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+
+  mark(MOE_STAGE_FINALIZE);
+  if (moe::launch_finalize(c->out_acc, static_cast<uint16_t*>(out), (long long)T * H, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  mark(MOE_NUM_STAGES);
+  c->last_T = T;
+  c->last_bn = BN;
+  c->last_grid = grid;
+  return MOE_OK;
+}
+
+moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream) {
+  if (!src || !dst || src == dst || rows <= 0 || K <= 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+  if (moe::launch_pack_e8m0(src, dst, rows, K / 32, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
+moe_status moe_get_routing(moe_ctx* c, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                           void* stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
+  cudaError_t e = cudaSuccess;
+  if (counts && e == cudaSuccess) e = cudaMemcpy(counts, c->counts, sizeof(int32_t) * c->NG, cudaMemcpyDefault);
+  if (offsets && e == cudaSuccess)
+    e = cudaMemcpy(offsets, c->offsets, sizeof(int32_t) * (c->NG + 1), cudaMemcpyDefault);
+  if (perm && P && e == cudaSuccess) e = cudaMemcpy(perm, c->perm, sizeof(int32_t) * P, cudaMemcpyDefault);
+  if (inv && P && e == cudaSuccess) e = cudaMemcpy(inv, c->inv, sizeof(int32_t) * P, cudaMemcpyDefault);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, float* hs, void* stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
+  cudaError_t e = cudaSuccess;
+  if (xq && P && e == cudaSuccess) e = cudaMemcpy(xq, c->xq, P * c->H, cudaMemcpyDefault);
+  if (xs && P && e == cudaSuccess) e = cudaMemcpy(xs, c->xs, sizeof(float) * P * (c->H / 128), cudaMemcpyDefault);
+  if (hq && P && e == cudaSuccess) e = cudaMemcpy(hq, c->hq, P * c->I, cudaMemcpyDefault);
+  if (hs && P && e == cudaSuccess) e = cudaMemcpy(hs, c->hs, sizeof(float) * P * (c->I / 128), cudaMemcpyDefault);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_device_status(moe_ctx* c, void* stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+  int32_t v = 0;
+  if (cudaMemcpy(&v, c->status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (cudaMemset(c->status, 0, sizeof(int32_t)) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v & moe::DEV_TIMEOUT) return MOE_ERR_TIMEOUT;
+  if (v & moe::DEV_BAD_ROUTING) return MOE_ERR_BAD_ROUTING;
+  return MOE_OK;
+}
+
+moe_status moe_profile_enable(moe_ctx* c, int on) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (on && !c->prof_ev) {
+    c->prof_ev = new (std::nothrow) cudaEvent_t[kProfMaxCalls * kProfEvents];
+    if (!c->prof_ev) return MOE_ERR_NO_MEMORY;
+    for (int i = 0; i < kProfMaxCalls * kProfEvents; ++i) {
+      if (cudaEventCreate(&c->prof_ev[i]) != cudaSuccess) {
+        for (int j = 0; j < i; ++j) cudaEventDestroy(c->prof_ev[j]);
+        delete[] c->prof_ev;
+        c->prof_ev = nullptr;
+        return MOE_ERR_CUDA;
+      }
+    }
+  }
+  if (!on) prof_free(c);
+  c->prof_on = on ? 1 : 0;
+  c->prof_calls = 0;
+  return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_ctx* c, float* avg_ms, int* calls) {
+  if (!c || !avg_ms) return MOE_ERR_INVALID_ARG;
+  double sum[MOE_NUM_STAGES] = {0};
+  const int n = c->prof_calls;
+  for (int i = 0; i < n; ++i) {
+    cudaEvent_t* ev = c->prof_ev + (size_t)i * kProfEvents;
+    if (cudaEventSynchronize(ev[MOE_NUM_STAGES]) != cudaSuccess) return MOE_ERR_CUDA;
+    for (int st = 0; st < MOE_NUM_STAGES; ++st) {
+      float ms = 0.0f;
+      if (cudaEventElapsedTime(&ms, ev[st], ev[st + 1]) != cudaSuccess) return MOE_ERR_CUDA;
+      sum[st] += ms;
+    }
+  }
+  for (int st = 0; st < MOE_NUM_STAGES; ++st) avg_ms[st] = n ? (float)(sum[st] / n) : 0.0f;
+  if (calls) *calls = n;
+  c->prof_calls = 0;
+  return MOE_OK;
+}
+
+moe_status moe_last_config(moe_ctx* c, int* tile_n, int* grid) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (tile_n) *tile_n = c->last_bn;
+  if (grid) *grid = c->last_grid;
+  return MOE_OK;
+}
+
+}  // extern "C"

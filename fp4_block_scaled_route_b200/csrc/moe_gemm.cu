@@ -1,0 +1,457 @@
+// moe_gemm.cu -- grouped expert GEMMs on tcgen05 tensor cores (sm_100a).
+//
+// One persistent kernel template serves both GEMMs of the layer:
+//   GEMM1 (steps 3-5): per expert, G = Xq_e * W13[e]^T over K = H, then
+//          SwiGLU (gate = first I rows) and FP8 requantisation per token per
+//          128 channels, written as the GEMM2 activations hq / hs.
+//   GEMM2 (steps 6-7): per expert, Y = Hq_e * W2[e]^T over K = I, then the
+//          top-k weighted combine: out_acc[token] += w * Y (fp32 atomics).
+// Sources: GC-MoE abstract (operand-swapped tcgen05 block-scaled MMA, fused
+// SwiGLU + requantisation, optional shared experts); FusedDeepMoE page
+// (GmmDeqSwigluQuant and GmmDeq with the combine as epilogue callback;
+// BlockEpilogue order: dequant by weight scale and per-token scale, SwiGLU,
+// block quant).
+//
+// Operand swap: the expert's weight rows fill the 128-row M side of the MMA
+// and the (few) tokens of the expert are the N side (BN = 16 .. 128), so a
+// decode step with 1-16 tokens per expert still issues full-height MMAs while
+// the weights stream through shared memory exactly once.
+//
+// Work unit = (row tile rt of 128 weight rows [GEMM1: 128 gate + 128 up
+// rows], token tile of <= BN positions of one expert).  Units are spread over
+// a grid of one CTA per SM; every CTA walks units u = blockIdx.x + i*grid.
+//
+// Warp roles (one CTA per SM):
+//   warp 0     TMA producer: weight tiles (128 rows x 128 K bytes, 128-byte
+//              swizzle, L2 evict-first) and the token tile, STAGES deep.
+//   warp 1     allocates TMEM; one lane issues tcgen05.mma (K = 32 per
+//              instruction, 4 per 128-wide K block) into one of two TMEM
+//              accumulators per K block and commits to mbarriers.
+//   warps 2..  epilogue: per K block, tcgen05.ld the block's fp32 partial and
+//              promote it with the block's scales (FP8: weight block scale x
+//              per-token activation scale; MXFP4: the E8M0 weight scales are
+//              applied by the MMA and only the activation scale is promoted),
+//              then the fused SwiGLU/requant or combine tail.
+// Per-128-K promotion is required because the fp32 FP8 scales (amax/448) are
+// not powers of two and so cannot be fed to the block-scaled MMA.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+template <int KIND, int BN, int WFMT>
+struct GemmCfg {
+  static constexpr int NA = (KIND == 1) ? 2 : 1;          // weight tiles per stage (gate + up)
+  static constexpr int A_BYTES = 128 * 128;               // 128 rows x 128 K bytes (E2M1 padded to 8 bits)
+  static constexpr int B_BYTES = BN * 128;
+  static constexpr int SF_BYTES = (WFMT == 1) ? NA * 512 : 0;
+  static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
+  static constexpr int KB_MAX = 64;                       // K <= 8192
+  static constexpr int CG = (BN <= 32) ? 1 : BN / 32;     // epilogue column groups
+  static constexpr int CPT = BN / CG;                     // columns per epilogue thread
+  static constexpr int EPI_THREADS = 128 * CG;
+  static constexpr int THREADS = 64 + EPI_THREADS;
+  static constexpr int MAX_STAGES = 12;
+  static constexpr int NBARS = 2 * MAX_STAGES + 5;
+  static constexpr int AUX_BYTES = ((BN * KB_MAX + NA * KB_MAX + 6 * BN) * 4 + NBARS * 8 + 16 + 15) / 16 * 16;
+  static constexpr int SMEM_LIMIT = 232448;
+  static constexpr int FIT = (SMEM_LIMIT - 1024 - AUX_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+  static constexpr int ACC_COLS = 2 * NA * BN;            // two accumulators (K-block parity)
+  static constexpr int SFA_COL = ACC_COLS;                // MXFP4: 2 parities x NA x 4 columns
+  static constexpr int SFB_COL = SFA_COL + 2 * NA * 4;    // MXFP4: 4 columns of unit scales
+  static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : ACC_COLS;
+  static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
+                                 : USED_COLS <= 256 ? 256 : 512;
+  static constexpr int TX_BYTES = STAGE_BYTES;
+  static_assert(STAGES >= 2, "shared memory too small");
+  static_assert(USED_COLS <= 512, "TMEM too small");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "BN");
+};
+
+// Bounded wait that ignores the abort word (used to drain in-flight copies
+// and MMAs before the CTA releases its shared memory and TMEM).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) break;
+  }
+}
+
+template <int KIND, int BN, int WFMT>
+__global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const GemmParams p) {
+  using C = GemmCfg<KIND, BN, WFMT>;
+  constexpr int NA = C::NA, STAGES = C::STAGES, KB_MAX = C::KB_MAX, CPT = C::CPT;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = sA + STAGES * NA * C::A_BYTES;
+  uint8_t* sSF = sB + STAGES * C::B_BYTES;
+  float* asc = reinterpret_cast<float*>(sSF + STAGES * C::SF_BYTES);  // [BN][KB_MAX] activation scales
+  float* wsc = asc + BN * KB_MAX;                                     // [NA][KB_MAX] FP8 weight scales
+  float* red = wsc + NA * KB_MAX;                                     // [4][BN] per-quarter amax
+  int* slot_tok = reinterpret_cast<int*>(red + 4 * BN);               // [BN] GEMM2: token of column
+  float* slot_w = reinterpret_cast<float*>(slot_tok + BN);            // [BN] GEMM2: combine weight
+  uint64_t* bars = reinterpret_cast<uint64_t*>(slot_w + BN);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* done = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
+  volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KB = p.kblocks;
+  const int num_tiles = *p.num_tiles;
+  const int rows_e = (KIND == 1) ? 2 * p.I : p.H;      // weight rows per expert
+  const int NRT = ((KIND == 1) ? p.I : p.H) / 128;     // row tiles per expert
+  const int RB = rows_e / 128;                          // 128-row scale blocks per expert
+  const int total = num_tiles * NRT;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], C::EPI_THREADS);
+    }
+    mbar_init(done, 1);
+    *abort = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA);
+    tma_prefetch_map(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  if constexpr (WFMT == 1) {
+    // B-side scale factors: all 1.0 (E8M0 127); the activation scales are
+    // promoted in the epilogue instead.
+    if (warp >= 2 && warp < 6) {
+      const uint32_t q = warp & 3;
+      tmem_st4(tmem + ((q * 32) << 16) + C::SFB_COL, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  }
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, last_par = 0;  // per-stage bitmasks for the final drain
+      bool ok = true;
+      for (int u = blockIdx.x; u < total; u += gridDim.x) {
+        const int rt = u / num_tiles, ti = u % num_tiles;
+        const int4 tile = p.tiles[ti];
+        const int e = tile.x, p0 = tile.y;
+        const int row0 = e * rows_e + rt * 128;
+        const int row1 = row0 + p.I;  // GEMM1 up rows
+        for (int kb = 0; kb < KB; ++kb) {
+          if (ok) ok = mbar_wait(&empty[stage], phase ^ 1u, abort);
+          if (ok) {
+            mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+            uint8_t* a = sA + stage * NA * C::A_BYTES;
+            tma_load_2d(&tmA, &full[stage], a, kb * 128, row0, pol_w);
+            if constexpr (KIND == 1) tma_load_2d(&tmA, &full[stage], a + C::A_BYTES, kb * 128, row1, pol_w);
+            tma_load_2d(&tmB, &full[stage], sB + stage * C::B_BYTES, kb * 128, p0, pol_a);
+            if constexpr (WFMT == 1) {
+              const uint8_t* sf = reinterpret_cast<const uint8_t*>(p.wscale);
+              uint8_t* d = sSF + stage * C::SF_BYTES;
+              bulk_load(d, sf + ((size_t)(row0 / 128) * KB + kb) * 512, 512, &full[stage], pol_w);
+              if constexpr (KIND == 1)
+                bulk_load(d + 512, sf + ((size_t)(row1 / 128) * KB + kb) * 512, 512, &full[stage], pol_w);
+            }
+            issued |= 1u << stage;
+            last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      for (int s = 0; s < STAGES; ++s)
+        if (issued & (1u << s)) drain_wait(&full[s], (last_par >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    constexpr int AF = (WFMT == 1) ? 5 : 0;  // E2M1 : E4M3
+    int stage = 0, buf = 0;
+    uint32_t phase = 0, tphase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (ok) ok = mbar_wait(&tempty[buf], tphase ^ 1u, abort);
+        if (ok) ok = mbar_wait(&full[stage], phase, abort);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (ok) {
+          tc_fence_after();
+          if (lane == 0) {
+            const uint32_t d0 = tmem + buf * (NA * BN);
+            const uint64_t ad = sdesc_k_sw128(smem_u32(sA + stage * NA * C::A_BYTES));
+            const uint64_t bd = sdesc_k_sw128(smem_u32(sB + stage * C::B_BYTES));
+            if constexpr (WFMT == 0) {
+              constexpr uint32_t idesc = idesc_f8f6f4(128, BN, AF, 0);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                mma_f8f6f4(d0, ad + 2 * kk, bd + 2 * kk, idesc, kk > 0);
+                if constexpr (KIND == 1)
+                  mma_f8f6f4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * kk, bd + 2 * kk, idesc, kk > 0);
+              }
+            } else {
+              // scale factors of this K block: smem atoms -> TMEM (parity buf)
+              const uint32_t sfa = tmem + C::SFA_COL + buf * (NA * 4);
+              const uint32_t sfb = tmem + C::SFB_COL;
+              uint8_t* sfs = sSF + stage * C::SF_BYTES;
+#pragma unroll
+              for (int a = 0; a < NA; ++a) {
+                uint64_t sd = 0;
+                sd |= static_cast<uint64_t>((smem_u32(sfs + a * 512) & 0x3FFFFu) >> 4);
+                sd |= static_cast<uint64_t>(128 >> 4) << 32;  // 8 rows x 16 bytes per core group
+                sd |= static_cast<uint64_t>(1) << 46;
+                tmem_cp_32x128b_warpx4(sfa + a * 4, sd);
+              }
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint32_t idesc = idesc_mxf8f6f4(128, BN, AF, 0, kk, 0);
+                mma_mxf8f6f4(d0, ad + 2 * kk, bd + 2 * kk, idesc, sfa, sfb, kk > 0);
+                if constexpr (KIND == 1)
+                  mma_mxf8f6f4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * kk, bd + 2 * kk, idesc, sfa + 4, sfb, kk > 0);
+              }
+            }
+            mma_commit(&empty[stage]);
+            mma_commit(&tfull[buf]);
+          }
+          __syncwarp();
+        }
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+        buf ^= 1;
+        if (buf == 0) tphase ^= 1u;
+      }
+    }
+    if (lane == 0) mma_commit(done);
+    __syncwarp();
+    drain_wait(done, 0);
+  } else {
+    // ---------------- epilogue ----------------
+    const int ew = warp - 2;
+    const int q = warp & 3;        // TMEM lane quarter this warp may access
+    const int cg = ew >> 2;        // column group
+    const int row = q * 32 + lane; // weight row within the tile = TMEM lane
+    const int etid = threadIdx.x - 64;
+    const int S = p.S;
+    int buf = 0;
+    uint32_t tphase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      const int rt = u / num_tiles, ti = u % num_tiles;
+      const int4 tile = p.tiles[ti];
+      const int e = tile.x, p0 = tile.y, nv = tile.z;
+      for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
+        const int j = i / KB, kb = i % KB;
+        asc[j * KB_MAX + kb] = p.ascale[(size_t)(p0 + j) * KB + kb];
+      }
+      if constexpr (WFMT == 0) {
+        for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
+          const int a = i / KB, kb = i % KB;
+          const int rb = (a == 0) ? rt : p.I / 128 + rt;
+          wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + rb) * KB + kb];
+        }
+      }
+      if constexpr (KIND == 2) {
+        for (int j = etid; j < BN; j += C::EPI_THREADS) {
+          int tok = 0;
+          float w = 0.0f;
+          if (j < nv) {
+            const int slot = p.perm[p0 + j];
+            tok = (slot < S) ? slot / p.k : slot - S;
+            w = (slot < S) ? p.topk_w[slot] : 1.0f;
+          }
+          slot_tok[j] = tok;
+          slot_w[j] = w;
+        }
+      }
+      named_sync(1, C::EPI_THREADS);
+
+      float acc0[CPT], acc1[CPT];
+#pragma unroll
+      for (int c = 0; c < CPT; ++c) {
+        acc0[c] = 0.0f;
+        acc1[c] = 0.0f;
+      }
+      for (int kb = 0; kb < KB; ++kb) {
+        if (ok) ok = mbar_wait(&tfull[buf], tphase, abort);
+        ok = __all_sync(0xFFFFFFFFu, ok);
+        if (ok) {
+          tc_fence_after();
+          const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + buf * (NA * BN) + cg * CPT;
+          const float w0 = (WFMT == 0) ? wsc[kb] : 1.0f;
+          const float w1 = (WFMT == 0 && KIND == 1) ? wsc[KB_MAX + kb] : 1.0f;
+#pragma unroll
+          for (int c0 = 0; c0 < CPT; c0 += 16) {
+            float d0[16], d1[16];
+            tmem_ld16(tb + c0, d0);
+            if constexpr (KIND == 1) tmem_ld16(tb + BN + c0, d1);
+            tmem_wait_ld();
+            if (c0 + 16 >= CPT) {
+              tc_fence_before();
+              mbar_arrive(&tempty[buf]);
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float sa = asc[(cg * CPT + c0 + i) * KB_MAX + kb];
+              acc0[c0 + i] = fmaf(d0[i], sa * w0, acc0[c0 + i]);
+              if constexpr (KIND == 1) acc1[c0 + i] = fmaf(d1[i], sa * w1, acc1[c0 + i]);
+            }
+          }
+        }
+        buf ^= 1;
+        if (buf == 0) tphase ^= 1u;
+      }
+
+      if constexpr (KIND == 1) {
+        // SwiGLU (gate rows 0..I-1 of W13, up rows I..2I-1: same channel),
+        // then FP8 requantisation per token over the tile's 128 channels.
+        float h[CPT];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          const float g = acc0[c];
+          const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+          h[c] = g * sig * acc1[c];
+          float m = fabsf(h[c]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          if (lane == 0) red[q * BN + cg * CPT + c] = m;
+        }
+        named_sync(1, C::EPI_THREADS);
+        if (ok) {
+          const int ch = rt * 128 + row;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            const int j = cg * CPT + c;
+            const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
+            const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+            if (j < nv) {
+              p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[c], sc)));
+              if (row == 0) p.hs[(size_t)(p0 + j) * (p.I / 128) + rt] = sc;
+            }
+          }
+        }
+      } else {
+        if (ok) {
+          const int ch = rt * 128 + row;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            const int j = cg * CPT + c;
+            if (j < nv) atomicAdd(p.out_acc + (size_t)slot_tok[j] * p.H + ch, slot_w[j] * acc0[c]);
+          }
+        }
+      }
+      named_sync(1, C::EPI_THREADS);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+  if (threadIdx.x == 0 && *abort) atomicOr(p.status, DEV_TIMEOUT);
+}
+
+// ---------------------------------------------------------------------------
+template <int KIND, int BN, int WFMT>
+static cudaError_t set_attr() {
+  using C = GemmCfg<KIND, BN, WFMT>;
+  return cudaFuncSetAttribute(moe_gemm_kernel<KIND, BN, WFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              C::SMEM_BYTES);
+}
+
+template <int KIND, int BN, int WFMT>
+static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
+                          cudaStream_t s) {
+  using C = GemmCfg<KIND, BN, WFMT>;
+  moe_gemm_kernel<KIND, BN, WFMT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_setup(int wfmt) {
+  cudaError_t e = cudaSuccess;
+#define MOE_SET(K, B, W) \
+  if (e == cudaSuccess) e = set_attr<K, B, W>();
+  if (wfmt == 0) {
+    MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0) MOE_SET(1, 128, 0)
+    MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0) MOE_SET(2, 128, 0)
+  } else {
+    MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
+    MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
+  }
+#undef MOE_SET
+  return e;
+}
+
+cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& tx,
+                         const GemmParams& p, cudaStream_t s) {
+  if (wfmt == 0) {
+    switch (BN) {
+      case 16: return launch<1, 16, 0>(grid, tw, tx, p, s);
+      case 32: return launch<1, 32, 0>(grid, tw, tx, p, s);
+      case 64: return launch<1, 64, 0>(grid, tw, tx, p, s);
+      case 128: return launch<1, 128, 0>(grid, tw, tx, p, s);
+    }
+  } else {
+    switch (BN) {
+      case 16: return launch<1, 16, 1>(grid, tw, tx, p, s);
+      case 32: return launch<1, 32, 1>(grid, tw, tx, p, s);
+      case 64: return launch<1, 64, 1>(grid, tw, tx, p, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
+                         const GemmParams& p, cudaStream_t s) {
+  if (wfmt == 0) {
+    switch (BN) {
+      case 16: return launch<2, 16, 0>(grid, tw, th, p, s);
+      case 32: return launch<2, 32, 0>(grid, tw, th, p, s);
+      case 64: return launch<2, 64, 0>(grid, tw, th, p, s);
+      case 128: return launch<2, 128, 0>(grid, tw, th, p, s);
+    }
+  } else {
+    switch (BN) {
+      case 16: return launch<2, 16, 1>(grid, tw, th, p, s);
+      case 32: return launch<2, 32, 1>(grid, tw, th, p, s);
+      case 64: return launch<2, 64, 1>(grid, tw, th, p, s);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

@@ -1,0 +1,62 @@
+// moe_internal.h -- parameter blocks and launchers shared by the library's
+// translation units (not part of the public C ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace moe {
+
+constexpr int kMaxK = 32;        // largest top-k accepted
+constexpr int kMaxGroups = 1025; // routed experts + shared expert
+constexpr int kRouteThreads = 1024;
+
+struct RouteParams {
+  int T, k, E, n_shared, BN;
+  const int32_t* ids;     // [T*k]
+  int32_t* counts;        // [E + n_shared]
+  int32_t* offsets;       // [E + n_shared + 1]
+  int32_t* perm;          // [P]   position -> slot (shared: S + t)
+  int32_t* inv;           // [P]   slot -> position (-1: dropped)
+  int4* tiles;            // (group, first position, valid rows, 0)
+  int32_t* num_tiles;     // [1]
+  int32_t* status;        // [1]
+};
+
+struct QuantParams {
+  int T, H, k, n_shared;
+  const uint16_t* x;      // bf16 [T, H]
+  const int32_t* inv;     // [P]
+  uint8_t* xq;            // E4M3 [S_pad, H]   rows in routing order
+  float* xs;              // [S_pad, H/128]
+  float* out_acc;         // [T, H] zeroed here
+};
+
+struct GemmParams {
+  int H, I, k, S;         // S = T*k routed slots
+  int kblocks;            // K / 128
+  const float* wscale;    // FP8: fp32 [NE, rows/128, K/128]; MXFP4: packed E8M0 atoms
+  const float* ascale;    // activation scales [S_pad, K/128]
+  uint8_t* hq;            // GEMM1: E4M3 [S_pad, I]
+  float* hs;              // GEMM1: [S_pad, I/128]
+  const int32_t* perm;    // GEMM2: position -> slot
+  const float* topk_w;    // GEMM2: [T*k]
+  float* out_acc;         // GEMM2: fp32 [T, H]
+  const int4* tiles;
+  const int32_t* num_tiles;
+  int32_t* status;
+};
+
+size_t route_smem_bytes(int n_groups);
+cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
+cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);
+cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s);
+cudaError_t gemm_setup(int wfmt);  // raise shared-memory limits once per process
+cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& tx,
+                         const GemmParams& p, cudaStream_t s);
+cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
+                         const GemmParams& p, cudaStream_t s);
+cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,259 @@
+// moe_route.cu -- routing, activation quantisation and output kernels.
+//
+// route_kernel   step 1: per-expert token counts, exclusive prefix sum,
+//                stable scatter of slots into expert-contiguous positions
+//                (perm) and its inverse (inv), plus the GEMM tile list.
+//                GC-MoE abstract (token dispatch); FusedDeepMoE page
+//                (per-expert counts, group list, expand index, prefix-summed
+//                ranges in OpCombineSend).
+// quant_kernel   step 2: per token, per 128 columns, s = amax/448 and
+//                q = e4m3(x/s), written to every position the token is routed
+//                to.  FusedDeepMoE QuantToken, with the E4M3 maximum in
+//                place of the int8 127.
+// finalize       fp32 combine accumulator -> bf16 output.
+#include <cuda_bf16.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+
+// ---------------------------------------------------------------------------
+// One CTA of 1024 threads.  Warp w owns the contiguous slot range
+// [w*chunk, (w+1)*chunk); __match_any_sync groups equal expert ids within a
+// 32-slot step, so a slot's position is
+//   offsets[e] + (slots of e in earlier warps) + (earlier steps of this warp)
+//   + (lower lanes with the same id in this step),
+// which is exactly the stable counting-sort position.
+__global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) {
+  extern __shared__ int sm[];
+  const int E = p.E, NG = p.E + p.n_shared;
+  const int S = p.T * p.k, P = S + p.n_shared * p.T;
+  int* cnt = sm;                 // [NG]
+  int* off = cnt + NG;           // [NG + 1]
+  int* toff = off + NG + 1;      // [NG + 1]
+  int* wc = toff + NG + 1;       // [32][NG]: per-warp counts, then per-warp bases
+  __shared__ int s_bad;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int i = tid; i < 32 * NG; i += kRouteThreads) wc[i] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+
+  const int chunk = (((S + 31) / 32) + 31) & ~31;
+  const int beg = min(S, warp * chunk), end = min(S, beg + chunk);
+
+  // pass A: per-warp, per-expert counts
+  for (int base = beg; base < end; base += 32) {
+    const int s = base + lane;
+    int e = -1;
+    if (s < end) {
+      e = p.ids[s];
+      if (e < 0 || e >= E) {
+        e = -1;
+        s_bad = 1;
+      }
+    }
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+
+  // per expert: total count, and counts of earlier warps (exclusive over warps)
+  for (int e = tid; e < E; e += kRouteThreads) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int c = wc[w * NG + e];
+      wc[w * NG + e] = run;
+      run += c;
+    }
+    cnt[e] = run;
+  }
+  if (p.n_shared && tid == 0) cnt[E] = p.T;
+  __syncthreads();
+
+  // exclusive scans: group offsets, and tile offsets (ceil(count / BN) tiles)
+  if (warp == 0 || warp == 1) {
+    const int per = (NG + 31) / 32;
+    const int b = min(NG, lane * per), en = min(NG, b + per);
+    int local = 0;
+    for (int i = b; i < en; ++i) local += (warp == 0) ? cnt[i] : (cnt[i] + p.BN - 1) / p.BN;
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    int run = incl - local;
+    int* dst = (warp == 0) ? off : toff;
+    for (int i = b; i < en; ++i) {
+      dst[i] = run;
+      run += (warp == 0) ? cnt[i] : (cnt[i] + p.BN - 1) / p.BN;
+    }
+    if (lane == 31) dst[NG] = incl;
+  }
+  __syncthreads();
+
+  for (int g = tid; g < NG; g += kRouteThreads) p.counts[g] = cnt[g];
+  for (int g = tid; g <= NG; g += kRouteThreads) p.offsets[g] = off[g];
+
+  // pass B: stable scatter
+  for (int base = beg; base < end; base += 32) {
+    const int s = base + lane;
+    int e = -1;
+    if (s < end) {
+      e = p.ids[s];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(peers & ((1u << lane) - 1u));
+    if (s < end) {
+      if (e >= 0) {
+        const int pos = off[e] + wc[warp * NG + e] + rank;
+        p.perm[pos] = s;
+        p.inv[s] = pos;
+      } else {
+        p.inv[s] = -1;
+      }
+    }
+    __syncwarp();
+    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
+    __syncwarp();
+  }
+
+  // shared expert: every token, as virtual slot S + t, after the routed groups
+  if (p.n_shared) {
+    for (int t = tid; t < p.T; t += kRouteThreads) {
+      const int pos = off[E] + t;
+      p.perm[pos] = S + t;
+      p.inv[S + t] = pos;
+    }
+  }
+  for (int i = off[NG] + tid; i < P; i += kRouteThreads) p.perm[i] = -1;  // tail left by dropped slots
+
+  // tile list: tiles[toff[g] + j] covers positions off[g] + j*BN ..
+  for (int g = tid; g < NG; g += kRouteThreads) {
+    const int n = cnt[g];
+    for (int j = 0; j * p.BN < n; ++j)
+      p.tiles[toff[g] + j] = make_int4(g, off[g] + j * p.BN, min(p.BN, n - j * p.BN), 0);
+  }
+  if (tid == 0) {
+    *p.num_tiles = toff[NG];
+    if (s_bad) atomicOr(p.status, DEV_BAD_ROUTING);
+  }
+}
+
+size_t route_smem_bytes(int n_groups) { return sizeof(int) * (3 * (size_t)n_groups + 2 + 32 * (size_t)n_groups); }
+
+cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
+  const size_t smem = route_smem_bytes(p.E + p.n_shared);
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)route_smem_bytes(kMaxGroups));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  route_kernel<<<1, kRouteThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// One CTA per token, 8 warps; warp w quantises column groups w, w+8, ...
+// Each lane holds 4 consecutive bf16 values of the 128-column group.
+constexpr int kQuantThreads = 256;
+
+__global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
+  const int t = blockIdx.x;
+  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  __shared__ int rows[kMaxK + 1];
+  __shared__ int nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int r = p.inv[t * p.k + j];
+      if (r >= 0) rows[n++] = r;
+    }
+    if (p.n_shared) rows[n++] = p.inv[S + t];
+    nrows = n;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xr = p.x + (size_t)t * H;
+  for (int g = warp; g < HB; g += kQuantThreads / 32) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    float f[4];
+    f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
+    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
+    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) packed |= f32_to_e4m3(__fdiv_rn(f[i], sc)) << (8 * i);
+    for (int r = 0; r < nrows; ++r) {
+      *reinterpret_cast<uint32_t*>(p.xq + (size_t)rows[r] * H + g * 128 + lane * 4) = packed;
+      if (lane == 0) p.xs[(size_t)rows[r] * HB + g] = sc;
+    }
+  }
+  float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
+  for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
+  quant_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+__global__ void finalize_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, long long n4) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 v = acc[i];
+    const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(v.z, v.w);
+    out[i] = make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+  }
+}
+
+cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s) {
+  const long long n4 = n / 4;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  long long blocks = (n4 + 255) / 256;
+  if (blocks > 4LL * sms) blocks = 4LL * sms;
+  if (blocks < 1) blocks = 1;
+  finalize_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(acc), reinterpret_cast<uint2*>(out), n4);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// E8M0 scales, plain layout [rows, kgroups] (one byte per 32 K elements) ->
+// the block-scaled MMA layout: for each 128-row block and each 128-wide K
+// block, one 512-byte atom with row m's 4 scales at byte
+// (m % 32) * 16 + (m / 32) * 4 + (k-group within the K block).
+__global__ void pack_e8m0_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int rows, int kgroups) {
+  const long long total = (long long)rows * kgroups;
+  const int kblocks = kgroups / 4;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+    const int r = (int)(i / kgroups), kg = (int)(i % kgroups);
+    const int rb = r / 128, m = r % 128, kb = kg / 4, kk = kg % 4;
+    const long long o = ((long long)rb * kblocks + kb) * 512 + (m % 32) * 16 + (m / 32) * 4 + kk;
+    dst[o] = src[i];
+  }
+}
+
+cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s) {
+  const long long total = (long long)rows * kgroups;
+  long long blocks = (total + 255) / 256;
+  if (blocks > 65535) blocks = 65535;
+  if (blocks < 1) blocks = 1;
+  pack_e8m0_kernel<<<(int)blocks, 256, 0, s>>>(src, dst, rows, kgroups);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

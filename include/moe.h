@@ -1,0 +1,171 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) decode-regime MoE layer library
+ * (libmoe.so).
+ *
+ * The operation (one MoE layer, single GPU):
+ *   given hidden states x[T,H] (bf16) and the router's top-k choice per token
+ *   (expert ids [T,k], combine weights [T,k]), compute
+ *     out[t] = sum_j topk_w[t,j] * FFN_{ids[t,j]}(x[t])  (+ FFN_shared(x[t]))
+ *   with FFN_e(x) = W2_e * (silu(W1_e x) * (W3_e x)) evaluated in the layer's
+ *   quantised form: activations quantised to FP8 E4M3 per token per 128
+ *   columns (scale amax/448), FP8 (128x128 block-scaled) or MXFP4 expert
+ *   weights, fp32 accumulation, SwiGLU output requantised to FP8 per token per
+ *   128 channels, fp32 combine, bf16 output.
+ * Sources:
+ *   - "GC-MoE: Overlapping Expert-Parallel Token Dispatch with FP8/FP4 Grouped
+ *     GEMM via CUDA Green Contexts", abstract: dispatch -> grouped GEMMs ->
+ *     combine; operand-swapped tcgen05 block-scaled MMA; fused SwiGLU and
+ *     requantisation; optional shared experts.
+ *   - FusedDeepMoE execution-flow page (Ascend fused family): the step math
+ *     (QuantToken, OpDequant, OpSwiglu with gate = first half, OpBlockQuant,
+ *     prefix-summed expert ranges, ReducePermute combine, shared expert as one
+ *     group of all tokens).
+ *   - OCP FP8 (E4M3) and OCP MX v1.0 (E2M1 + E8M0 per 32) define the formats.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named d_* or documented as "device" are CUDA device pointers on
+ *     the context's device; the library never frees memory it did not allocate.
+ *   - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *     enqueued asynchronously on it; no entry point synchronises the device
+ *     unless documented.
+ *   - Errors detectable on the host are returned synchronously and nothing is
+ *     enqueued.  Errors detected on the device (bad expert id, a pipeline wait
+ *     that gave up) are OR-ed into a device status word that
+ *     moe_get_device_status() reads.
+ *   - The calls are not thread-safe on one context; use one context per
+ *     host thread or serialise.
+ */
+#ifndef FP4_BLOCK_SCALED_ROUTE_B200_MOE_H
+#define FP4_BLOCK_SCALED_ROUTE_B200_MOE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct moe_ctx moe_ctx;
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned pointer */
+  MOE_ERR_UNSUPPORTED = 2,  /* shape/format outside what the kernels handle, or not an sm_100 GPU */
+  MOE_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  MOE_ERR_NO_MEMORY = 4,    /* workspace allocation failed */
+  MOE_ERR_TIMEOUT = 5,      /* device: a pipeline wait gave up (no hang; outputs invalid) */
+  MOE_ERR_BAD_ROUTING = 6   /* device: an expert id outside [0,E); that slot was dropped */
+} moe_status;
+
+/* Expert weight formats. */
+enum {
+  /* w13 u8 E4M3 [NE, 2I, H], rows 0..I-1 = gate (W1), I..2I-1 = up (W3);
+   * s13 f32 [NE, 2I/128, H/128] one scale per 128x128 block;
+   * w2 u8 E4M3 [NE, H, I]; s2 f32 [NE, H/128, I/128]. */
+  MOE_WFMT_FP8_E4M3_B128 = 0,
+  /* w13 u8 [NE, 2I, H/2]: E2M1 nibbles, element 2c in the low nibble of byte c;
+   * w2 u8 [NE, H, I/2]; scales are E8M0 (2^(e-127)) per 32 elements along K,
+   * plain layout [NE, rows, K/32], converted once with moe_pack_mxfp4_scales()
+   * into the layout moe_forward() reads. */
+  MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1
+};
+
+/* moe_create -- context for a layer with hidden size H, expert intermediate
+ * size I, E routed experts, top-k = k, weight format wfmt (MOE_WFMT_*), no
+ * shared expert, up to 4096 tokens per call.  Same as
+ * moe_create_ex(H, I, E, k, wfmt, 4096, 0, out). */
+moe_status moe_create(int H, int I, int E, int k, int wfmt, moe_ctx** out);
+
+/* moe_create_ex -- as moe_create, with the token capacity max_T (>= 1) and
+ * n_shared (0 or 1) always-on shared experts at combine weight 1.0 (GC-MoE
+ * abstract "optional shared experts"; FusedDeepMoE: the shared expert takes
+ * every token as one group).  The shared expert's weights are expert index E
+ * of the weight arrays (NE = E + n_shared) and share I.
+ * Requirements: H and I multiples of 128, 128 <= H, I <= 8192; 1 <= E <= 1024;
+ * 1 <= k <= 32.  The GPU must be sm_100 (B200).  The context owns its
+ * workspace (device memory sized by max_T) on the current device; *out is
+ * set to NULL on failure. */
+moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_shared, moe_ctx** out);
+
+/* moe_destroy -- frees the context and its workspace (synchronises the
+ * device first).  NULL is a no-op. */
+void moe_destroy(moe_ctx* ctx);
+
+/* moe_forward -- one MoE layer.
+ *   T          tokens, 0 <= T <= max_T (T = 0 enqueues nothing)
+ *   x          device bf16 [T, H], 16-byte aligned
+ *   topk_ids   device int32 [T, k]; ids outside [0, E) drop their slot and
+ *              raise MOE_ERR_BAD_ROUTING in the device status
+ *   topk_w     device fp32 [T, k], used as given (no renormalisation)
+ *   w13, s13, w2, s2   device expert weights in the context's format (see
+ *              MOE_WFMT_*), weights 128-byte aligned, scales 16-byte aligned
+ *   out        device bf16 [T, H], overwritten, 16-byte aligned
+ * Steps, all in this library's CUDA kernels on `stream`: route (counts,
+ * prefix sum, stable permutation + inverse), activation FP8 quantisation,
+ * GEMM1 with fused SwiGLU + requantisation, GEMM2 with fused weighted
+ * combine, bf16 output.  The workspace is reused by the next call on the same
+ * context, so calls on one context must be stream-ordered. */
+moe_status moe_forward(moe_ctx* ctx, int T, const void* x, const int32_t* topk_ids, const float* topk_w,
+                       const void* w13, const void* s13, const void* w2, const void* s2, void* out,
+                       void* stream);
+
+/* moe_pack_mxfp4_scales -- converts E8M0 scales from the plain layout
+ * [rows, K/32] (rows = NE*2I for s13, NE*H for s2) into the 128x128 atom
+ * layout moe_forward() reads for MOE_WFMT_MXFP4_E2M1_E8M0_K32 (same byte
+ * count).  src and dst are distinct device buffers; rows % 128 == 0 and
+ * K % 128 == 0.  Weight-load-time step, asynchronous on `stream`. */
+moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream);
+
+/* moe_get_routing -- copies the routing of the last moe_forward() (after a
+ * stream synchronisation) into caller buffers (host or device):
+ *   counts  int32 [E + n_shared]     tokens per expert (shared expert: T)
+ *   offsets int32 [E + n_shared + 1] exclusive prefix sum of counts
+ *   perm    int32 [T*k + n_shared*T] position -> slot t*k+j (shared: T*k + t), -1 past the end
+ *   inv     int32 [T*k + n_shared*T] slot -> position, -1 for a dropped slot
+ * Any pointer may be NULL.  Debug / test entry point. */
+moe_status moe_get_routing(moe_ctx* ctx, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
+                           void* stream);
+
+/* moe_get_activations -- copies the quantised activations of the last call
+ * (after a stream synchronisation), rows in routing-position order:
+ *   xq u8 E4M3 [P, H], xs fp32 [P, H/128]  (GEMM1 input, P = T*k + n_shared*T)
+ *   hq u8 E4M3 [P, I], hs fp32 [P, I/128]  (GEMM2 input)
+ * Rows of dropped positions are unspecified.  Any pointer may be NULL. */
+moe_status moe_get_activations(moe_ctx* ctx, uint8_t* xq, float* xs, uint8_t* hq, float* hs, void* stream);
+
+/* moe_get_device_status -- synchronises `stream`, returns MOE_OK,
+ * MOE_ERR_TIMEOUT or MOE_ERR_BAD_ROUTING (timeout wins) for all calls since
+ * the last status read, and clears the status word. */
+moe_status moe_get_device_status(moe_ctx* ctx, void* stream);
+
+/* moe_last_config -- tile width (tokens per MMA N tile) and grid size the
+ * last moe_forward() used; debug / benchmark entry point. */
+moe_status moe_last_config(moe_ctx* ctx, int* tile_n, int* grid);
+
+/* Kernel stages of one moe_forward(), in launch order (profiling index). */
+enum {
+  MOE_STAGE_ROUTE = 0,     /* counts, prefix sum, permutation, tile list */
+  MOE_STAGE_QUANT = 1,     /* activation FP8 quantisation (+ clears the fp32 combine buffer) */
+  MOE_STAGE_GEMM1 = 2,     /* grouped GEMM1 + SwiGLU + FP8 requantisation */
+  MOE_STAGE_GEMM2 = 3,     /* grouped GEMM2 + top-k weighted combine */
+  MOE_STAGE_FINALIZE = 4,  /* fp32 -> bf16 output */
+  MOE_NUM_STAGES = 5
+};
+
+/* moe_profile_enable -- on != 0: every following moe_forward() also records
+ * CUDA events around each of its kernels on the caller's stream (up to 4096
+ * calls are kept); on == 0: stop and discard.  Profiling entry point. */
+moe_status moe_profile_enable(moe_ctx* ctx, int on);
+
+/* moe_profile_read -- synchronises the recorded events and writes the mean
+ * duration in milliseconds of each stage over the calls recorded since
+ * profiling was enabled (or last read) into avg_ms[MOE_NUM_STAGES]; *calls
+ * receives their number.  Resets the record. */
+moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
+
+/* moe_status_string -- static description of a status code. */
+const char* moe_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,74 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads without a GPU,
+exports every entry point include/moe.h declares, and the product path never
+touches the oracle."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from fp4_block_scaled_route_b200 import build as moe_build
+from fp4_block_scaled_route_b200 import moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(moe_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def libmoe():
+    moe_build.build()
+    return moe.lib()
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ("moe_create", "moe_forward", "moe_destroy"):
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol(libmoe):
+    for name in declared_symbols():
+        assert hasattr(libmoe, name), name
+    raw = ctypes.CDLL(moe.LIB_PATH)
+    for name in declared_symbols():
+        assert getattr(raw, name) is not None
+
+
+def test_binding_covers_every_declared_symbol():
+    assert sorted(moe.SIGNATURES) == declared_symbols()
+
+
+def test_status_strings(libmoe):
+    assert moe.status_string(0) == "ok"
+    assert "range" in moe.status_string(moe.MOE_ERR_BAD_ROUTING)
+
+
+def test_host_argument_checks_without_gpu(libmoe):
+    ctx = ctypes.c_void_p()
+    assert libmoe.moe_create(100, 128, 8, 2, 0, ctypes.byref(ctx)) == moe.MOE_ERR_UNSUPPORTED
+    assert libmoe.moe_create_ex(256, 128, 8, 2, 7, 16, 0, ctypes.byref(ctx)) == moe.MOE_ERR_UNSUPPORTED
+    assert libmoe.moe_create_ex(256, 128, 8, 2, 0, 0, 0, ctypes.byref(ctx)) == moe.MOE_ERR_INVALID_ARG
+    assert libmoe.moe_create(256, 128, 8, 2, 0, None) == moe.MOE_ERR_INVALID_ARG
+    assert libmoe.moe_forward(None, 1, None, None, None, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
+    assert libmoe.moe_pack_mxfp4_scales(None, None, 128, 128, None) == moe.MOE_ERR_INVALID_ARG
+
+
+def test_product_path_does_not_use_the_oracle():
+    pkg = os.path.join(ROOT, "fp4_block_scaled_route_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle", text, flags=re.M), f
+                assert "moe_oracle" not in text and "orc_" not in text, f
+
+
+def test_sources_are_sm100a_only():
+    src = open(os.path.join(ROOT, "fp4_block_scaled_route_b200", "build.py")).read()
+    assert "arch=compute_100a,code=sm_100a" in src
