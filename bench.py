@@ -49,6 +49,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", type=int, default=1, help="index into synth.CONFIGS")
+    ap.add_argument("--shape", default=None,
+                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4) instead of --workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -196,10 +198,18 @@ def workload_stats(L, ids_np):
     return dict(experts_touched=n_exp, weight_bytes=wbytes, flops=flops, gemm1_bytes=g1, positions=P)
 
 
-def build_layer(cfg_idx, device):
-    from fp4_block_scaled_route_b200 import moe, synth
-    cfg = synth.CONFIGS[cfg_idx]
-    L = synth.make_layer(cfg, synth.config_seed(cfg_idx), device=device)
+def build_layer(args, device):
+    from fp4_block_scaled_route_b200 import synth
+    if args.shape:
+        f = args.shape.split(",")
+        T, H, E, k, I = (int(v) for v in f[:5])
+        wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4}[f[5]]
+        nsh = int(f[6]) if len(f) > 6 else 0
+        cfg = dict(name=f"custom_T{T}_H{H}_E{E}_k{k}_I{I}_{f[5]}" + ("_shared" if nsh else ""), T=T, H=H, E=E,
+                   k=k, I=I, wfmt=wfmt, routing="uniform", n_shared=nsh)
+        return cfg, synth.make_layer(cfg, 2000, device=device)
+    cfg = synth.CONFIGS[args.workload]
+    L = synth.make_layer(cfg, synth.config_seed(args.workload), device=device)
     return cfg, L
 
 
@@ -239,7 +249,7 @@ def run_reference(args):
     import torch
     from fp4_block_scaled_route_b200 import synth
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    cfg, L = build_layer(args.workload, dev)
+    cfg, L = build_layer(args, dev)
     # per step: one (token, expert) slot, the smallest unit of the workload
     times, nb = [], 0
     for i in range(args.warmup + args.steps):
@@ -290,7 +300,7 @@ def main():
     if dist:
         dist.barrier()
 
-    cfg, L = build_layer(args.workload, dev)
+    cfg, L = build_layer(args, dev)
     ids_np = L.ids.cpu().numpy()
     st = workload_stats(L, ids_np)
     layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)

@@ -66,7 +66,10 @@ struct GemmCfg {
   static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : ACC_COLS;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                  : USED_COLS <= 256 ? 256 : 512;
-  static constexpr int TX_BYTES = STAGE_BYTES;
+  // Transaction bytes per stage: a packed-E2M1 weight tile moves 64 bytes per
+  // row from global memory although it lands as 128 padded bytes in smem.
+  static constexpr int A_TX = (WFMT == 1) ? A_BYTES / 2 : A_BYTES;
+  static constexpr int TX_BYTES = NA * A_TX + B_BYTES + SF_BYTES;
   static_assert(STAGES >= 2, "shared memory too small");
   static_assert(USED_COLS <= 512, "TMEM too small");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "BN");

@@ -43,6 +43,7 @@ SIGNATURES = {
     "moe_last_config": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "moe_profile_enable": (_i, [_vp, _i]),
     "moe_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i)]),
+    "moe_forward_noalloc": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
 }
 
@@ -99,6 +100,12 @@ def moe_destroy(ctx) -> None:
 
 def moe_forward(ctx, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, stream) -> int:
     return lib().moe_forward(ctx, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, stream)
+
+
+def moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, d_status,
+                        stream) -> int:
+    return lib().moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13, s13, w2, s2, out,
+                                     d_status, stream)
 
 
 def moe_pack_mxfp4_scales(src, dst, rows, K, stream) -> int:

@@ -162,6 +162,39 @@ moe_status moe_profile_enable(moe_ctx* ctx, int on);
  * receives their number.  Resets the record. */
 moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
 
+/* Size of the fixed device scratch array used by moe_forward_noalloc(). */
+#define MOE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* moe_forward_noalloc -- the same layer as moe_forward(), for callers that
+ * cannot allocate device memory: code running under a host framework that
+ * owns every device allocation (its allocator may not be bypassed), code that
+ * must not allocate while a stream is being captured, or a memory-pool-locked
+ * process.  No context is needed and nothing is allocated: no cudaMalloc,
+ * cudaFree or allocating library routine.  The scratch (routing arrays, tile
+ * list, quantised activations, fp32 combine buffer) is one file-scope device
+ * array of MOE_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
+ * keeps until the process exits.  The paper has no counterpart of this entry
+ * point; it exists only for such callers.
+ *   H, I, E, k, wfmt, n_shared   the layer, as in moe_create_ex()
+ *   T, x, topk_ids, topk_w, w13, s13, w2, s2, out   as in moe_forward()
+ *   d_status   optional device int32 (caller memory): cleared, then receives
+ *              the device status bits of this call (1 = expert id out of
+ *              range, 2 = pipeline wait timed out); NULL keeps them in the
+ *              scratch, where they are not readable.
+ * The scratch needed grows with T*(k + n_shared)*(H + I) plus T*H*4 bytes
+ * (FP8 decode T=32, H=7168, I=2048, k=8 needs about 5 MB; T=128 about
+ * 15 MB); a shape that needs more than MOE_NOALLOC_SCRATCH_BYTES returns
+ * MOE_ERR_UNSUPPORTED before any device work.
+ * The first call on a device performs a one-time set-up on the current
+ * device (looks up the array's device address, sets kernel attributes);
+ * make that first call before any stream capture.  Every call, on every
+ * stream, shares the one array and leaves its contents behind: calls whose
+ * execution overlaps on the GPU race and corrupt each other's results, so
+ * order them (one stream, or events). */
+moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, int n_shared, int T, const void* x,
+                               const int32_t* topk_ids, const float* topk_w, const void* w13, const void* s13,
+                               const void* w2, const void* s2, void* out, int32_t* d_status, void* stream);
+
 /* moe_status_string -- static description of a status code. */
 const char* moe_status_string(int status);
 
