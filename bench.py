@@ -323,7 +323,6 @@ def main():
     # ---- timed region (device events, max over ranks) ----
     sampler = ClockSampler(gpu_uuid(dev))
     sampler.wait_first()
-    moe.moe_profile_enable(layer.ctx, 1)
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
     if dist:
@@ -339,10 +338,21 @@ def main():
     if dist:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
-    stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
-    moe.moe_profile_enable(layer.ctx, 0)
     clocks = sampler.summary(tw0, tw1)
     sampler.stop()
+
+    # ---- second timed region: the same K steps with CUDA events around each
+    # kernel of the layer (on the launching stream), for the per-kernel times ----
+    moe.moe_profile_enable(layer.ctx, 1)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(args.steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_prof = ev0.elapsed_time(ev1)
+    stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
+    moe.moe_profile_enable(layer.ctx, 0)
     if layer.device_status() != moe.MOE_OK:
         raise RuntimeError("device status not OK after the timed region")
     if dist:
@@ -430,10 +440,11 @@ def main():
         "tflops": st["flops"] / (ms_step * 1e-3) / 1e12,
         "hbm_frac_of_step": frac_step,
         "stage_ms": dict(zip(moe.STAGE_NAMES, stage_ms)),
+        "ms_per_step_profiled": ms_prof / args.steps,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": moe.MOE_NUM_STAGES * args.steps,
+        "gpu_launches": moe.MOE_NUM_STAGES * args.steps,  # per timed region
         "clocks": clocks,
     }
     print(json.dumps(line), flush=True)

@@ -54,15 +54,19 @@ struct GemmCfg {
   static constexpr int EPI_THREADS = 128 * CG;
   static constexpr int THREADS = 64 + EPI_THREADS;
   static constexpr int MAX_STAGES = 12;
-  static constexpr int NBARS = 2 * MAX_STAGES + 5;
+  // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
+  // the promoting epilogue (short K steps would otherwise be latency bound).
+  static constexpr int NBUF_RAW = 256 / (NA * BN);
+  static constexpr int NBUF = NBUF_RAW < 2 ? 2 : (NBUF_RAW > 8 ? 8 : NBUF_RAW);
+  static constexpr int NBARS = 2 * MAX_STAGES + 2 * 8 + 1;
   static constexpr int AUX_BYTES = ((BN * KB_MAX + NA * KB_MAX + 6 * BN) * 4 + NBARS * 8 + 16 + 15) / 16 * 16;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int FIT = (SMEM_LIMIT - 1024 - AUX_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
-  static constexpr int ACC_COLS = 2 * NA * BN;            // two accumulators (K-block parity)
-  static constexpr int SFA_COL = ACC_COLS;                // MXFP4: 2 parities x NA x 4 columns
-  static constexpr int SFB_COL = SFA_COL + 2 * NA * 4;    // MXFP4: 4 columns of unit scales
+  static constexpr int ACC_COLS = NBUF * NA * BN;         // NBUF accumulators
+  static constexpr int SFA_COL = ACC_COLS;                // MXFP4: NBUF x NA x 4 columns
+  static constexpr int SFB_COL = SFA_COL + NBUF * NA * 4; // MXFP4: 4 columns of unit scales
   static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : ACC_COLS;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                  : USED_COLS <= 256 ? 256 : 512;
@@ -103,9 +107,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(slot_w + BN);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
+  constexpr int NBUF = C::NBUF;
   uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* done = tempty + 2;
+  uint64_t* tempty = tfull + NBUF;
+  uint64_t* done = tempty + NBUF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -122,7 +127,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NBUF; ++b) {
       mbar_init(&tfull[b], 1);
       mbar_init(&tempty[b], C::EPI_THREADS);
     }
@@ -142,6 +147,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  // The next kernel may be scheduled as soon as SMs free up; it waits for this
+  // grid's completion before it reads anything this grid writes.
+  griddep_launch_dependents();
 
   if constexpr (WFMT == 1) {
     // B-side scale factors: all 1.0 (E8M0 127); the activation scales are
@@ -165,20 +173,40 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0, last_par = 0;  // per-stage bitmasks for the final drain
       bool ok = true;
+      // The weights (and the tile list, written before the previous kernel
+      // started) do not depend on the previous kernel: the first ring pass of
+      // weight tiles is issued before waiting for it; the token tiles of that
+      // pass follow once the previous kernel's output is visible.
+      bool waited = false;
+      int npend = 0;
+      int pend_c0[STAGES], pend_p0[STAGES];
+      int it = 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const int rt = u / num_tiles, ti = u % num_tiles;
         const int4 tile = p.tiles[ti];
         const int e = tile.x, p0 = tile.y;
         const int row0 = e * rows_e + rt * 128;
         const int row1 = row0 + p.I;  // GEMM1 up rows
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          if (!waited && it == STAGES) {
+            griddep_wait();
+            for (int i = 0; i < npend; ++i)
+              tma_load_2d(&tmB, &full[i], sB + i * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
+            waited = true;
+          }
           if (ok) ok = mbar_wait(&empty[stage], phase ^ 1u, abort);
           if (ok) {
             mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
             uint8_t* a = sA + stage * NA * C::A_BYTES;
             tma_load_2d(&tmA, &full[stage], a, kb * 128, row0, pol_w);
             if constexpr (KIND == 1) tma_load_2d(&tmA, &full[stage], a + C::A_BYTES, kb * 128, row1, pol_w);
-            tma_load_2d(&tmB, &full[stage], sB + stage * C::B_BYTES, kb * 128, p0, pol_a);
+            if (waited) {
+              tma_load_2d(&tmB, &full[stage], sB + stage * C::B_BYTES, kb * 128, p0, pol_a);
+            } else {
+              pend_c0[npend] = kb * 128;
+              pend_p0[npend] = p0;
+              ++npend;
+            }
             if constexpr (WFMT == 1) {
               const uint8_t* sf = reinterpret_cast<const uint8_t*>(p.wscale);
               uint8_t* d = sSF + stage * C::SF_BYTES;
@@ -194,6 +222,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             phase ^= 1u;
           }
         }
+      }
+      if (!waited) {
+        griddep_wait();
+        for (int i = 0; i < npend; ++i)
+          tma_load_2d(&tmB, &full[i], sB + i * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
       }
       for (int s = 0; s < STAGES; ++s)
         if (issued & (1u << s)) drain_wait(&full[s], (last_par >> s) & 1u);
@@ -225,7 +258,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
               }
             } else {
               // scale factors of this K block: smem atoms -> TMEM (parity buf)
-              const uint32_t sfa = tmem + C::SFA_COL + buf * (NA * 4);
+              const uint32_t sfa = tmem + C::SFA_COL + buf * (NA * 4);  // per accumulator buffer
               const uint32_t sfb = tmem + C::SFB_COL;
               uint8_t* sfs = sSF + stage * C::SF_BYTES;
 #pragma unroll
@@ -253,8 +286,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
           stage = 0;
           phase ^= 1u;
         }
-        buf ^= 1;
-        if (buf == 0) tphase ^= 1u;
+        if (++buf == NBUF) {
+          buf = 0;
+          tphase ^= 1u;
+        }
       }
     }
     if (lane == 0) mma_commit(done);
@@ -271,6 +306,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     int buf = 0;
     uint32_t tphase = 0;
     bool ok = true;
+    griddep_wait();  // activation scales / combine buffer come from earlier kernels
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const int rt = u / num_tiles, ti = u % num_tiles;
       const int4 tile = p.tiles[ti];
@@ -333,8 +369,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             }
           }
         }
-        buf ^= 1;
-        if (buf == 0) tphase ^= 1u;
+        if (++buf == NBUF) {
+          buf = 0;
+          tphase ^= 1u;
+        }
       }
 
       if constexpr (KIND == 1) {
@@ -400,8 +438,17 @@ template <int KIND, int BN, int WFMT>
 static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
                           cudaStream_t s) {
   using C = GemmCfg<KIND, BN, WFMT>;
-  moe_gemm_kernel<KIND, BN, WFMT><<<grid, C::THREADS, C::SMEM_BYTES, s>>>(ta, tb, p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT>, ta, tb, p);
 }
 
 cudaError_t gemm_setup(int wfmt) {

@@ -221,6 +221,16 @@ __device__ __forceinline__ void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// ---- programmatic dependent launch -----------------------------------------------
+// Let the next kernel in the stream be scheduled now (its pre-wait prologue
+// overlaps this kernel); a no-op when it was not launched for overlap.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+// Wait until the preceding kernel of the stream has completed and its memory
+// is visible; a no-op when this kernel was launched without overlap.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---- FP8 conversion --------------------------------------------------------------
 // fp32 -> E4M3 with round-to-nearest-even and saturation to +-448.
 __device__ __forceinline__ uint32_t f32_to_e4m3(float v) {

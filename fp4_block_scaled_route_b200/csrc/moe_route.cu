@@ -165,6 +165,7 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
 constexpr int kQuantThreads = 256;
 
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
+  griddep_launch_dependents();  // GEMM1 may start its weight prefetch now
   const int t = blockIdx.x;
   const int H = p.H, HB = p.H / 128, S = p.T * p.k;
   __shared__ int rows[kMaxK + 1];
@@ -211,6 +212,7 @@ cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
 
 // ---------------------------------------------------------------------------
 __global__ void finalize_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, long long n4) {
+  griddep_wait();  // the combine buffer is complete once GEMM2 has finished
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
     const float4 v = acc[i];
     const __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y);
@@ -227,8 +229,17 @@ cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaSt
   long long blocks = (n4 + 255) / 256;
   if (blocks > 4LL * sms) blocks = 4LL * sms;
   if (blocks < 1) blocks = 1;
-  finalize_kernel<<<(int)blocks, 256, 0, s>>>(reinterpret_cast<const float4*>(acc), reinterpret_cast<uint2*>(out), n4);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)blocks);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, finalize_kernel, reinterpret_cast<const float4*>(acc), reinterpret_cast<uint2*>(out),
+                            n4);
 }
 
 // ---------------------------------------------------------------------------
