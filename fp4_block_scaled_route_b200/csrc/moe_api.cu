@@ -35,7 +35,12 @@ struct moe_ctx {
   // profiling: events[call][stage boundary]
   int prof_on, prof_calls;
   cudaEvent_t* prof_ev;
+  int tile_n_override;  // MOE_TILE_N environment variable (16/32/64/128), 0 = automatic
+  float* y_rows;        // [S_pad, H] fp32 per-position expert outputs (MOE_COMBINE=rows only)
+  int combine_mode;     // MOE_COMBINE: 0/1 fused fp32 reductions (default), 2 stored rows
 };
+
+
 
 namespace {
 constexpr int kProfMaxCalls = 4096;
@@ -82,6 +87,7 @@ bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p
 int pick_tile_n(const moe_ctx* c, int T) {
   const double avg = (double)T * c->k / c->E;  // expected tokens per routed expert
   int bn = avg <= 8 ? 16 : avg <= 20 ? 32 : avg <= 48 ? 64 : 128;
+  if (c->tile_n_override) bn = c->tile_n_override;
   if (c->wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 && bn > 64) bn = 64;
   return bn;
 }
@@ -136,6 +142,14 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->P_max = c->S_max + n_shared * max_T;
   c->S_pad = c->P_max + 128;
   c->max_tiles = c->P_max / 16 + c->NG + 1;
+  if (const char* env = getenv("MOE_COMBINE")) {
+    if (!strcmp(env, "atomic")) c->combine_mode = 1;
+    if (!strcmp(env, "rows")) c->combine_mode = 2;
+  }
+  if (const char* env = getenv("MOE_TILE_N")) {
+    const int v = atoi(env);
+    if (v == 16 || v == 32 || v == 64 || (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128)) c->tile_n_override = v;
+  }
 
   const size_t HB = H / 128, IB = I / 128;
   size_t off = 0;
@@ -156,6 +170,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_xs = take(sizeof(float) * (size_t)c->S_pad * HB);
   const size_t o_hs = take(sizeof(float) * (size_t)c->S_pad * IB);
   const size_t o_acc = take(sizeof(float) * (size_t)max_T * H);
+  const bool want_rows = c->combine_mode == 2;
+  const size_t o_rows = want_rows ? take(sizeof(float) * (size_t)c->S_pad * H) : 0;
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     delete c;
@@ -181,6 +197,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->xs = reinterpret_cast<float*>(b + o_xs);
   c->hs = reinterpret_cast<float*>(b + o_hs);
   c->out_acc = reinterpret_cast<float*>(b + o_acc);
+  c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
   *out = c;
   return MOE_OK;
 }
@@ -216,11 +233,12 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   const bool fp8 = (c->wfmt == MOE_WFMT_FP8_E4M3_B128);
 
   // weight maps (re-encoded only when the caller's pointers change)
+  const CUtensorMapL2promotion wpromo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
   if (w13 != c->c_w13) {
     const bool ok = fp8 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H, (uint64_t)NE * 2 * I, H, 128,
-                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                                   wpromo)
                         : make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13, H, (uint64_t)NE * 2 * I,
-                                   H / 2, 128, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+                                   H / 2, 128, wpromo);
     if (!ok) {
       c->c_w13 = nullptr;
       return MOE_ERR_CUDA;
@@ -229,9 +247,9 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   }
   if (w2 != c->c_w2) {
     const bool ok = fp8 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I, (uint64_t)NE * H, I, 128,
-                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B)
+                                   wpromo)
                         : make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2, I, (uint64_t)NE * H, I / 2,
-                                   128, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+                                   128, wpromo);
     if (!ok) {
       c->c_w2 = nullptr;
       return MOE_ERR_CUDA;
@@ -262,9 +280,14 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   mark(MOE_STAGE_ROUTE);
   if (moe::launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
+  const int P = S + c->n_shared * T;
+  const bool rows = c->y_rows != nullptr;
+  (void)P;
+
   QuantParams qp;
   qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
-  qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs; qp.out_acc = c->out_acc;
+  qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs;
+  qp.out_acc = rows ? nullptr : c->out_acc;
   mark(MOE_STAGE_QUANT);
   if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -276,6 +299,7 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.hq = c->hq; g.hs = c->hs;
   g.perm = c->perm; g.topk_w = topk_w; g.out_acc = c->out_acc;
   g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
+  g.y_rows = nullptr;
   mark(MOE_STAGE_GEMM1);
   if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -283,11 +307,18 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.wscale = static_cast<const float*>(s2);
   g.ascale = c->hs;
   mark(MOE_STAGE_GEMM2);
+  g.y_rows = rows ? c->y_rows : nullptr;
   if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
 
   mark(MOE_STAGE_FINALIZE);
-  if (moe::launch_finalize(c->out_acc, static_cast<uint16_t*>(out), (long long)T * H, s) != cudaSuccess)
+  if (rows) {
+    moe::CombineParams cp;
+    cp.T = T; cp.H = H; cp.k = c->k; cp.n_shared = c->n_shared;
+    cp.y_rows = c->y_rows; cp.inv = c->inv; cp.topk_w = topk_w; cp.out = static_cast<uint16_t*>(out);
+    if (moe::launch_combine(cp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (moe::launch_finalize(c->out_acc, static_cast<uint16_t*>(out), (long long)T * H, s) != cudaSuccess) {
     return MOE_ERR_CUDA;
+  }
   mark(MOE_NUM_STAGES);
   c->last_T = T;
   c->last_bn = BN;

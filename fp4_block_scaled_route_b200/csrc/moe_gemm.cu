@@ -49,7 +49,7 @@ struct GemmCfg {
   static constexpr int SF_BYTES = (WFMT == 1) ? NA * 512 : 0;
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int KB_MAX = 64;                       // K <= 8192
-  static constexpr int CG = (BN <= 32) ? 1 : BN / 32;     // epilogue column groups
+  static constexpr int CG = (BN <= 64) ? 1 : BN / 64;     // epilogue column groups
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
   static constexpr int THREADS = 64 + EPI_THREADS;
@@ -99,7 +99,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * NA * C::A_BYTES;
   uint8_t* sSF = sB + STAGES * C::B_BYTES;
-  float* asc = reinterpret_cast<float*>(sSF + STAGES * C::SF_BYTES);  // [BN][KB_MAX] activation scales
+  float* asc = reinterpret_cast<float*>(sSF + STAGES * C::SF_BYTES);  // [KB_MAX][BN] activation scales
   float* wsc = asc + BN * KB_MAX;                                     // [NA][KB_MAX] FP8 weight scales
   float* red = wsc + NA * KB_MAX;                                     // [4][BN] per-quarter amax
   int* slot_tok = reinterpret_cast<int*>(red + 4 * BN);               // [BN] GEMM2: token of column
@@ -313,7 +313,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       const int e = tile.x, p0 = tile.y, nv = tile.z;
       for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
         const int j = i / KB, kb = i % KB;
-        asc[j * KB_MAX + kb] = p.ascale[(size_t)(p0 + j) * KB + kb];
+        asc[kb * BN + j] = p.ascale[(size_t)(p0 + j) * KB + kb];
       }
       if constexpr (WFMT == 0) {
         for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
@@ -351,21 +351,51 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
           const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + buf * (NA * BN) + cg * CPT;
           const float w0 = (WFMT == 0) ? wsc[kb] : 1.0f;
           const float w1 = (WFMT == 0 && KIND == 1) ? wsc[KB_MAX + kb] : 1.0f;
+          // acc += D_kb * (activation scale x weight block scale), two
+          // columns per paired fp32 multiply-add
+          if constexpr (KIND == 1 && CPT >= 64) {
+            // wide tiles: gate and up chunks one after the other, so only 16
+            // loaded values are live next to the 2 x CPT accumulators
 #pragma unroll
-          for (int c0 = 0; c0 < CPT; c0 += 16) {
-            float d0[16], d1[16];
-            tmem_ld16(tb + c0, d0);
-            if constexpr (KIND == 1) tmem_ld16(tb + BN + c0, d1);
-            tmem_wait_ld();
-            if (c0 + 16 >= CPT) {
-              tc_fence_before();
-              mbar_arrive(&tempty[buf]);
+            for (int c0 = 0; c0 < 2 * CPT; c0 += 16) {
+              float d[16];
+              const bool up = c0 >= CPT;
+              const int cc = up ? c0 - CPT : c0;
+              tmem_ld16(tb + (up ? BN : 0) + cc, d);
+              tmem_wait_ld();
+              if (c0 + 16 >= 2 * CPT) {
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);
+              }
+              const float2 wk = make_float2(up ? w1 : w0, up ? w1 : w0);
+              const float2* sa2 = reinterpret_cast<const float2*>(asc + kb * BN + cg * CPT + cc);
+              float2* a2 = reinterpret_cast<float2*>(up ? acc1 + cc : acc0 + cc);
+#pragma unroll
+              for (int i = 0; i < 8; ++i)
+                a2[i] = __ffma2_rn(make_float2(d[2 * i], d[2 * i + 1]), __fmul2_rn(sa2[i], wk), a2[i]);
             }
+          } else {
+            const float2 wg = make_float2(w0, w0), wu = make_float2(w1, w1);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float sa = asc[(cg * CPT + c0 + i) * KB_MAX + kb];
-              acc0[c0 + i] = fmaf(d0[i], sa * w0, acc0[c0 + i]);
-              if constexpr (KIND == 1) acc1[c0 + i] = fmaf(d1[i], sa * w1, acc1[c0 + i]);
+            for (int c0 = 0; c0 < CPT; c0 += 16) {
+              float d0[16], d1[16];
+              tmem_ld16(tb + c0, d0);
+              if constexpr (KIND == 1) tmem_ld16(tb + BN + c0, d1);
+              tmem_wait_ld();
+              if (c0 + 16 >= CPT) {
+                tc_fence_before();
+                mbar_arrive(&tempty[buf]);
+              }
+              const float2* sa2 = reinterpret_cast<const float2*>(asc + kb * BN + cg * CPT + c0);
+              float2* g2 = reinterpret_cast<float2*>(acc0 + c0);
+              float2* u2 = reinterpret_cast<float2*>(acc1 + c0);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float2 sa = sa2[i];
+                g2[i] = __ffma2_rn(make_float2(d0[2 * i], d0[2 * i + 1]), __fmul2_rn(sa, wg), g2[i]);
+                if constexpr (KIND == 1)
+                  u2[i] = __ffma2_rn(make_float2(d1[2 * i], d1[2 * i + 1]), __fmul2_rn(sa, wu), u2[i]);
+              }
             }
           }
         }
@@ -378,7 +408,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       if constexpr (KIND == 1) {
         // SwiGLU (gate rows 0..I-1 of W13, up rows I..2I-1: same channel),
         // then FP8 requantisation per token over the tile's 128 channels.
-        float h[CPT];
+        float* h = acc0;  // h overwrites the gate accumulator in place
 #pragma unroll
         for (int c = 0; c < CPT; ++c) {
           const float g = acc0[c];
@@ -406,10 +436,20 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       } else {
         if (ok) {
           const int ch = rt * 128 + row;
+          if (p.y_rows) {
+            // unfused combine: keep this position's expert output row
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            const int j = cg * CPT + c;
-            if (j < nv) atomicAdd(p.out_acc + (size_t)slot_tok[j] * p.H + ch, slot_w[j] * acc0[c]);
+            for (int c = 0; c < CPT; ++c) {
+              const int j = cg * CPT + c;
+              if (j < nv) p.y_rows[(size_t)(p0 + j) * p.H + ch] = acc0[c];
+            }
+          } else {
+            // fused combine: out_acc[token] += w * y (fp32 reductions in L2)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+              const int j = cg * CPT + c;
+              if (j < nv) atomicAdd(p.out_acc + (size_t)slot_tok[j] * p.H + ch, slot_w[j] * acc0[c]);
+            }
           }
         }
       }

@@ -30,7 +30,7 @@ struct QuantParams {
   const int32_t* inv;     // [P]
   uint8_t* xq;            // E4M3 [S_pad, H]   rows in routing order
   float* xs;              // [S_pad, H/128]
-  float* out_acc;         // [T, H] zeroed here
+  float* out_acc;         // [T, H] zeroed here (null: not needed)
 };
 
 struct GemmParams {
@@ -46,6 +46,15 @@ struct GemmParams {
   const int4* tiles;
   const int32_t* num_tiles;
   int32_t* status;
+  float* y_rows;          // GEMM2: non-null = store fp32 rows [S_pad, H] instead of the fused combine
+};
+
+struct CombineParams {
+  int T, H, k, n_shared;
+  const float* y_rows;    // [S_pad, H] expert output per routing position
+  const int32_t* inv;     // slot -> position (-1: dropped)
+  const float* topk_w;    // [T*k]
+  uint16_t* out;          // bf16 [T, H]
 };
 
 size_t route_smem_bytes(int n_groups);
@@ -53,10 +62,12 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s);
 cudaError_t gemm_setup(int wfmt);  // raise shared-memory limits once per process
+// tw: weight tiles; tx / th: token tiles.
 cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& tx,
                          const GemmParams& p, cudaStream_t s);
 cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
                          const GemmParams& p, cudaStream_t s);
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s);
 
 }  // namespace moe

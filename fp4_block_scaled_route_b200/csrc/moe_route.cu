@@ -201,8 +201,10 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
       if (lane == 0) p.xs[(size_t)rows[r] * HB + g] = sc;
     }
   }
-  float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
-  for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.out_acc) {
+    float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
+    for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
@@ -240,6 +242,66 @@ cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaSt
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, finalize_kernel, reinterpret_cast<const float4*>(acc), reinterpret_cast<uint2*>(out),
                             n4);
+}
+
+// ---------------------------------------------------------------------------
+// Unfused combine (step 7) for large token counts: one CTA per token,
+// out[t] = sum_j w[t,j] * y[inv[t*k+j]] (ascending j) + y[inv[S+t]] (shared
+// expert, weight 1), in fp32, then bf16.  FusedDeepMoE ReducePermute
+// (accumulate the expert outputs of each token), in the same order as the
+// CPU reference and without atomics.
+__global__ void __launch_bounds__(256) combine_kernel(CombineParams p) {
+  griddep_wait();  // the expert output rows are complete once GEMM2 has finished
+  const int t = blockIdx.x, S = p.T * p.k;
+  __shared__ int rows[kMaxK + 1];
+  __shared__ float wts[kMaxK + 1];
+  __shared__ int nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int r = p.inv[t * p.k + j];
+      if (r >= 0) {
+        rows[n] = r;
+        wts[n] = p.topk_w[t * p.k + j];
+        ++n;
+      }
+    }
+    if (p.n_shared) {
+      rows[n] = p.inv[S + t];
+      wts[n] = 1.0f;
+      ++n;
+    }
+    nrows = n;
+  }
+  __syncthreads();
+  for (int h = threadIdx.x * 4; h < p.H; h += 256 * 4) {
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < nrows; ++r) {
+      const float4 y = *reinterpret_cast<const float4*>(p.y_rows + (size_t)rows[r] * p.H + h);
+      const float w = wts[r];
+      o.x += w * y.x;
+      o.y += w * y.y;
+      o.z += w * y.z;
+      o.w += w * y.w;
+    }
+    const __nv_bfloat162 a = __floats2bfloat162_rn(o.x, o.y);
+    const __nv_bfloat162 b = __floats2bfloat162_rn(o.z, o.w);
+    *reinterpret_cast<uint2*>(p.out + (size_t)t * p.H + h) =
+        make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
+  }
+}
+
+cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)p.T);
+  cfg.blockDim = dim3(256);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, combine_kernel, p);
 }
 
 // ---------------------------------------------------------------------------

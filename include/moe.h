@@ -83,7 +83,14 @@ moe_status moe_create(int H, int I, int E, int k, int wfmt, moe_ctx** out);
  * Requirements: H and I multiples of 128, 128 <= H, I <= 8192; 1 <= E <= 1024;
  * 1 <= k <= 32.  The GPU must be sm_100 (B200).  The context owns its
  * workspace (device memory sized by max_T) on the current device; *out is
- * set to NULL on failure. */
+ * set to NULL on failure.  Tuning: the environment variable MOE_TILE_N
+ * (16, 32, 64, or 128 for FP8), read here, fixes the token-tile width the
+ * GEMMs use instead of the automatic choice from T*k/E, and MOE_COMBINE
+ * ("atomic" or "rows") fixes how the top-k combine is done: fused into GEMM2
+ * as fp32 reductions (default), or from stored per-position fp32 expert
+ * outputs in a separate, deterministic pass that sums each token's experts
+ * in ascending j (the context then holds an extra [positions, H] fp32
+ * buffer). */
 moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_shared, moe_ctx** out);
 
 /* moe_destroy -- frees the context and its workspace (synchronises the
@@ -147,7 +154,7 @@ enum {
   MOE_STAGE_QUANT = 1,     /* activation FP8 quantisation (+ clears the fp32 combine buffer) */
   MOE_STAGE_GEMM1 = 2,     /* grouped GEMM1 + SwiGLU + FP8 requantisation */
   MOE_STAGE_GEMM2 = 3,     /* grouped GEMM2 + top-k weighted combine */
-  MOE_STAGE_FINALIZE = 4,  /* fp32 -> bf16 output */
+  MOE_STAGE_FINALIZE = 4,  /* fp32 -> bf16 output (or the unfused combine + bf16 output) */
   MOE_NUM_STAGES = 5
 };
 

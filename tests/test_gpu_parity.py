@@ -260,3 +260,24 @@ def test_full_size_sampled(cfg_idx):
     P = L.T * L.k + L.n_shared * L.T
     assert np.array_equal(inv[perm[:P]], np.arange(P))
     assert counts.sum() == P
+
+
+# ---- both combine paths (fused fp32 reductions / stored rows + combine pass) ----
+@pytest.mark.parametrize("mode", ["atomic", "rows"])
+def test_combine_paths(mode, monkeypatch):
+    monkeypatch.setenv("MOE_COMBINE", mode)
+    cfg = dict(T=150, H=256, I=256, E=8, k=4, wfmt=0, n_shared=1)
+    L = synth.make_layer(cfg, 61, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.device_status() == moe.MOE_OK
+    assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], f"combine {mode}")
+
+
+@pytest.mark.parametrize("bn", ["16", "32", "64", "128"])
+def test_every_tile_width(bn, monkeypatch):
+    monkeypatch.setenv("MOE_TILE_N", bn)
+    cfg = dict(T=90, H=384, I=256, E=6, k=3, wfmt=0)
+    L = synth.make_layer(cfg, 62, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.last_config()[0] == int(bn)
+    assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], f"tile {bn}")
