@@ -52,14 +52,22 @@ struct GemmCfg {
   static constexpr int CG = (BN <= 64) ? 1 : BN / 64;     // epilogue column groups
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
-  static constexpr int THREADS = 64 + EPI_THREADS;
+  // Warpgroup 0: NPROD TMA producer warps (warp p issues all loads of the
+  // pipeline iterations it with it % NPROD == p) and the MMA warp.  One
+  // issuing thread fills shared memory through TMA at only ~47 GB/s, so the
+  // iterations are spread over three issuers.  Warpgroups 1..CG: the epilogue.
+  static constexpr int NPROD = 3;
+  static constexpr int MMA_WARP = 3;
+  static constexpr int EPI_WARP0 = 4;
+  static constexpr int THREADS = 128 + EPI_THREADS;
   static constexpr int MAX_STAGES = 12;
   // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
   // the promoting epilogue (short K steps would otherwise be latency bound).
   static constexpr int NBUF_RAW = 256 / (NA * BN);
   static constexpr int NBUF = NBUF_RAW < 2 ? 2 : (NBUF_RAW > 8 ? 8 : NBUF_RAW);
   static constexpr int NBARS = 2 * MAX_STAGES + 2 * 8 + 1;
-  static constexpr int AUX_BYTES = ((BN * KB_MAX + NA * KB_MAX + 6 * BN) * 4 + NBARS * 8 + 16 + 15) / 16 * 16;
+  static constexpr int AUX_BYTES =
+      ((BN * KB_MAX + NA * KB_MAX + 6 * BN + 2 * NA * BN) * 4 + NBARS * 8 + 16 + 15) / 16 * 16;
   static constexpr int SMEM_LIMIT = 232448;
   static constexpr int FIT = (SMEM_LIMIT - 1024 - AUX_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
@@ -104,7 +112,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   float* red = wsc + NA * KB_MAX;                                     // [4][BN] per-quarter amax
   int* slot_tok = reinterpret_cast<int*>(red + 4 * BN);               // [BN] GEMM2: token of column
   float* slot_w = reinterpret_cast<float*>(slot_tok + BN);            // [BN] GEMM2: combine weight
-  uint64_t* bars = reinterpret_cast<uint64_t*>(slot_w + BN);
+  float* cs = slot_w + BN;                                            // [2][NA][BN] combined scales ring
+  uint64_t* bars = reinterpret_cast<uint64_t*>(cs + 2 * NA * BN);
   uint64_t* full = bars;
   uint64_t* empty = bars + STAGES;
   constexpr int NBUF = C::NBUF;
@@ -139,7 +148,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     tma_prefetch_map(&tmA);
     tma_prefetch_map(&tmB);
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -154,7 +163,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   if constexpr (WFMT == 1) {
     // B-side scale factors: all 1.0 (E8M0 127); the activation scales are
     // promoted in the epilogue instead.
-    if (warp >= 2 && warp < 6) {
+    if (warp >= C::EPI_WARP0 && warp < C::EPI_WARP0 + 4) {
       const uint32_t q = warp & 3;
       tmem_st4(tmem + ((q * 32) << 16) + C::SFB_COL, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu, 0x7F7F7F7Fu);
       tmem_wait_st();
@@ -164,22 +173,25 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     tc_fence_after();
   }
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
+  if (warp < C::NPROD) {
+    // ---------------- TMA producers ----------------
+    // Producer pr fills the stages of the pipeline iterations it (one per
+    // (unit, K block)) with it % NPROD == pr: stage it % STAGES, phase
+    // (it / STAGES) & 1.  The MMA warp consumes the iterations in order.
     if (lane == 0) {
+      const int pr = warp;
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t issued = 0, last_par = 0;  // per-stage bitmasks for the final drain
+      uint32_t issued = 0, last_par = 0;  // per-stage bitmasks for the abort drain
       bool ok = true;
       // The weights (and the tile list, written before the previous kernel
       // started) do not depend on the previous kernel: the first ring pass of
       // weight tiles is issued before waiting for it; the token tiles of that
       // pass follow once the previous kernel's output is visible.
       bool waited = false;
+      constexpr int NPEND = (STAGES + C::NPROD - 1) / C::NPROD;
       int npend = 0;
-      int pend_c0[STAGES], pend_p0[STAGES];
+      int pend_c0[NPEND], pend_p0[NPEND], pend_st[NPEND];
       int it = 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const int rt = u / num_tiles, ti = u % num_tiles;
@@ -188,10 +200,13 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         const int row0 = e * rows_e + rt * 128;
         const int row1 = row0 + p.I;  // GEMM1 up rows
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          if (!waited && it == STAGES) {
+          if (it % C::NPROD != pr) continue;
+          const int stage = it % STAGES;
+          const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
+          if (!waited && it >= STAGES) {
             griddep_wait();
             for (int i = 0; i < npend; ++i)
-              tma_load_2d(&tmB, &full[i], sB + i * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
+              tma_load_2d(&tmB, &full[pend_st[i]], sB + pend_st[i] * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
             waited = true;
           }
           if (ok) ok = mbar_wait(&empty[stage], phase ^ 1u, abort);
@@ -205,6 +220,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             } else {
               pend_c0[npend] = kb * 128;
               pend_p0[npend] = p0;
+              pend_st[npend] = stage;
               ++npend;
             }
             if constexpr (WFMT == 1) {
@@ -217,21 +233,21 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             issued |= 1u << stage;
             last_par = (last_par & ~(1u << stage)) | (phase << stage);
           }
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
         }
       }
       if (!waited) {
         griddep_wait();
         for (int i = 0; i < npend; ++i)
-          tma_load_2d(&tmB, &full[i], sB + i * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
+          tma_load_2d(&tmB, &full[pend_st[i]], sB + pend_st[i] * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
       }
-      for (int s = 0; s < STAGES; ++s)
-        if (issued & (1u << s)) drain_wait(&full[s], (last_par >> s) & 1u);
+      // Without an abort every issued load was consumed by the MMA warp.  After
+      // one, wait (bounded) for this producer's last load into each stage; a
+      // later phase issued by another producer only shortens that wait.
+      if (*abort)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) drain_wait(&full[s], (last_par >> s) & 1u);
     }
-  } else if (warp == 1) {
+  } else if (warp == C::MMA_WARP) {
     // ---------------- MMA issuer ----------------
     constexpr int AF = (WFMT == 1) ? 5 : 0;  // E2M1 : E4M3
     int stage = 0, buf = 0;
@@ -295,13 +311,13 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     if (lane == 0) mma_commit(done);
     __syncwarp();
     drain_wait(done, 0);
-  } else {
+  } else if (warp >= C::EPI_WARP0) {
     // ---------------- epilogue ----------------
-    const int ew = warp - 2;
+    const int ew = warp - C::EPI_WARP0;
     const int q = warp & 3;        // TMEM lane quarter this warp may access
     const int cg = ew >> 2;        // column group
     const int row = q * 32 + lane; // weight row within the tile = TMEM lane
-    const int etid = threadIdx.x - 64;
+    const int etid = threadIdx.x - 32 * C::EPI_WARP0;
     const int S = p.S;
     int buf = 0;
     uint32_t tphase = 0;
@@ -343,16 +359,29 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         acc0[c] = 0.0f;
         acc1[c] = 0.0f;
       }
+      // Combined scale of K block kb per tile column, shared by all 128 rows:
+      // cs[kb & 1][a][j] = activation scale (column j, kb) x weight block
+      // scale (tile a, kb) (MXFP4: the activation scale alone).  Filled one K
+      // block ahead by the epilogue threads, one named barrier per K block.
+      auto fill_cs = [&](int kb) {
+        float* dst = cs + (kb & 1) * (NA * BN);
+        for (int i = etid; i < NA * BN; i += C::EPI_THREADS) {
+          const int a = i / BN, j = i - (i / BN) * BN;
+          dst[i] = (WFMT == 0) ? asc[kb * BN + j] * wsc[a * KB_MAX + kb] : asc[kb * BN + j];
+        }
+      };
+      fill_cs(0);
+      named_sync(1, C::EPI_THREADS);
       for (int kb = 0; kb < KB; ++kb) {
+        if (kb + 1 < KB) fill_cs(kb + 1);
         if (ok) ok = mbar_wait(&tfull[buf], tphase, abort);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (ok) {
           tc_fence_after();
           const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + buf * (NA * BN) + cg * CPT;
-          const float w0 = (WFMT == 0) ? wsc[kb] : 1.0f;
-          const float w1 = (WFMT == 0 && KIND == 1) ? wsc[KB_MAX + kb] : 1.0f;
-          // acc += D_kb * (activation scale x weight block scale), two
-          // columns per paired fp32 multiply-add
+          const float* csg = cs + (kb & 1) * (NA * BN) + cg * CPT;
+          const float* csu = csg + (NA - 1) * BN;
+          // acc += D_kb * combined scale, two columns per paired fp32 FMA
           if constexpr (KIND == 1 && CPT >= 64) {
             // wide tiles: gate and up chunks one after the other, so only 16
             // loaded values are live next to the 2 x CPT accumulators
@@ -367,15 +396,12 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
                 tc_fence_before();
                 mbar_arrive(&tempty[buf]);
               }
-              const float2 wk = make_float2(up ? w1 : w0, up ? w1 : w0);
-              const float2* sa2 = reinterpret_cast<const float2*>(asc + kb * BN + cg * CPT + cc);
+              const float2* s2 = reinterpret_cast<const float2*>((up ? csu : csg) + cc);
               float2* a2 = reinterpret_cast<float2*>(up ? acc1 + cc : acc0 + cc);
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                a2[i] = __ffma2_rn(make_float2(d[2 * i], d[2 * i + 1]), __fmul2_rn(sa2[i], wk), a2[i]);
+              for (int i = 0; i < 8; ++i) a2[i] = __ffma2_rn(make_float2(d[2 * i], d[2 * i + 1]), s2[i], a2[i]);
             }
           } else {
-            const float2 wg = make_float2(w0, w0), wu = make_float2(w1, w1);
 #pragma unroll
             for (int c0 = 0; c0 < CPT; c0 += 16) {
               float d0[16], d1[16];
@@ -386,19 +412,19 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
                 tc_fence_before();
                 mbar_arrive(&tempty[buf]);
               }
-              const float2* sa2 = reinterpret_cast<const float2*>(asc + kb * BN + cg * CPT + c0);
+              const float2* sg = reinterpret_cast<const float2*>(csg + c0);
+              const float2* su = reinterpret_cast<const float2*>(csu + c0);
               float2* g2 = reinterpret_cast<float2*>(acc0 + c0);
               float2* u2 = reinterpret_cast<float2*>(acc1 + c0);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float2 sa = sa2[i];
-                g2[i] = __ffma2_rn(make_float2(d0[2 * i], d0[2 * i + 1]), __fmul2_rn(sa, wg), g2[i]);
-                if constexpr (KIND == 1)
-                  u2[i] = __ffma2_rn(make_float2(d1[2 * i], d1[2 * i + 1]), __fmul2_rn(sa, wu), u2[i]);
+                g2[i] = __ffma2_rn(make_float2(d0[2 * i], d0[2 * i + 1]), sg[i], g2[i]);
+                if constexpr (KIND == 1) u2[i] = __ffma2_rn(make_float2(d1[2 * i], d1[2 * i + 1]), su[i], u2[i]);
               }
             }
           }
         }
+        named_sync(1, C::EPI_THREADS);  // cs slot kb+1 written, slot kb consumed
         if (++buf == NBUF) {
           buf = 0;
           tphase ^= 1u;
@@ -459,7 +485,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
