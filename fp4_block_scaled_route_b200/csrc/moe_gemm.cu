@@ -53,11 +53,15 @@ struct GemmCfg {
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
   // Warpgroup 0: NPROD TMA producer warps (warp p issues all loads of the
-  // pipeline iterations it with it % NPROD == p) and the MMA warp.  One
-  // issuing thread fills shared memory through TMA at only ~47 GB/s, so the
-  // iterations are spread over three issuers.  Warpgroups 1..CG: the epilogue.
-  static constexpr int NPROD = 3;
-  static constexpr int MMA_WARP = 3;
+  // pipeline iterations it with it % NPROD == p) and NMMA MMA warps (MMA warp
+  // m issues all MMAs of the iterations with it % NMMA == m, each iteration
+  // into its own TMEM accumulator).  One issuing thread fills shared memory
+  // through TMA at only ~47 GB/s, and one thread issues a tcgen05.mma only
+  // every ~100 cycles whatever N is, which for 4-bit weights is below the
+  // HBM rate; two of each double both.  Warpgroups 1..CG: the epilogue.
+  static constexpr int NPROD = 2;
+  static constexpr int NMMA = 2;
+  static constexpr int MMA_WARP = NPROD;  // first MMA warp; allocates TMEM
   static constexpr int EPI_WARP0 = 4;
   static constexpr int THREADS = 128 + EPI_THREADS;
   static constexpr int MAX_STAGES = 12;
@@ -114,11 +118,18 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   float* slot_w = reinterpret_cast<float*>(slot_tok + BN);            // [BN] GEMM2: combine weight
   float* cs = slot_w + BN;                                            // [2][NA][BN] combined scales ring
   uint64_t* bars = reinterpret_cast<uint64_t*>(cs + 2 * NA * BN);
-  uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
+  // full[s]: TMA bytes of stage s landed.  mdone[i % NMD]: the MMAs of
+  // pipeline iteration i completed -- one tcgen05.commit per iteration tells
+  // the producers that the stage is free and the epilogue that the TMEM
+  // accumulator is ready (each commit costs the tensor pipe several hundred
+  // cycles, so a second one per iteration would halve the decode rate).
+  // tempty[b]: the epilogue has read TMEM accumulator b.  NMD = STAGES +
+  // NBUF keeps every waiter within one phase of the barrier it polls.
   constexpr int NBUF = C::NBUF;
-  uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + NBUF;
+  constexpr int NMD = STAGES + NBUF;
+  uint64_t* full = bars;
+  uint64_t* mdone = bars + STAGES;
+  uint64_t* tempty = mdone + NMD;
   uint64_t* done = tempty + NBUF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(done + 1);
   volatile int* abort = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -132,15 +143,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   const int total = num_tiles * NRT;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < NBUF; ++b) {
-      mbar_init(&tfull[b], 1);
-      mbar_init(&tempty[b], C::EPI_THREADS);
-    }
-    mbar_init(done, 1);
+    for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
+    for (int i = 0; i < NMD; ++i) mbar_init(&mdone[i], 1);
+    for (int b = 0; b < NBUF; ++b) mbar_init(&tempty[b], C::EPI_THREADS);
+    mbar_init(done, C::NMMA);
     *abort = 0;
     mbar_fence_init();
   }
@@ -209,7 +215,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
               tma_load_2d(&tmB, &full[pend_st[i]], sB + pend_st[i] * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
             waited = true;
           }
-          if (ok) ok = mbar_wait(&empty[stage], phase ^ 1u, abort);
+          if (ok && it >= STAGES) {  // the stage's previous iteration has been consumed
+            const int prev = it - STAGES;
+            ok = mbar_wait(&mdone[prev % NMD], (uint32_t)(prev / NMD) & 1u, abort);
+          }
           if (ok) {
             mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
             uint8_t* a = sA + stage * NA * C::A_BYTES;
@@ -247,14 +256,17 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         for (int s = 0; s < STAGES; ++s)
           if (issued & (1u << s)) drain_wait(&full[s], (last_par >> s) & 1u);
     }
-  } else if (warp == C::MMA_WARP) {
-    // ---------------- MMA issuer ----------------
+  } else if (warp < C::MMA_WARP + C::NMMA) {
+    // ---------------- MMA issuers ----------------
     constexpr int AF = (WFMT == 1) ? 5 : 0;  // E2M1 : E4M3
-    int stage = 0, buf = 0;
-    uint32_t phase = 0, tphase = 0;
+    const int mw = warp - C::MMA_WARP;
     bool ok = true;
+    int mit = 0;  // pipeline iteration
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < KB; ++kb, ++mit) {
+        if (mit % C::NMMA != mw) continue;
+        const int stage = mit % STAGES, buf = mit % NBUF;
+        const uint32_t phase = (uint32_t)(mit / STAGES) & 1u, tphase = (uint32_t)(mit / NBUF) & 1u;
         if (ok) ok = mbar_wait(&tempty[buf], tphase ^ 1u, abort);
         if (ok) ok = mbar_wait(&full[stage], phase, abort);
         ok = __all_sync(0xFFFFFFFFu, ok);
@@ -293,18 +305,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
                   mma_mxf8f6f4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * kk, bd + 2 * kk, idesc, sfa + 4, sfb, kk > 0);
               }
             }
-            mma_commit(&empty[stage]);
-            mma_commit(&tfull[buf]);
+            mma_commit(&mdone[mit % NMD]);
           }
           __syncwarp();
-        }
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
-        }
-        if (++buf == NBUF) {
-          buf = 0;
-          tphase ^= 1u;
         }
       }
     }
@@ -322,6 +325,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     int buf = 0;
     uint32_t tphase = 0;
     bool ok = true;
+    int eit = 0;  // pipeline iteration
     griddep_wait();  // activation scales / combine buffer come from earlier kernels
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const int rt = u / num_tiles, ti = u % num_tiles;
@@ -372,9 +376,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       };
       fill_cs(0);
       named_sync(1, C::EPI_THREADS);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int kb = 0; kb < KB; ++kb, ++eit) {
         if (kb + 1 < KB) fill_cs(kb + 1);
-        if (ok) ok = mbar_wait(&tfull[buf], tphase, abort);
+        if (ok) ok = mbar_wait(&mdone[eit % NMD], (uint32_t)(eit / NMD) & 1u, abort);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (ok) {
           tc_fence_after();
