@@ -38,6 +38,7 @@ struct moe_ctx {
   int tile_n_override;  // MOE_TILE_N environment variable (16/32/64/128), 0 = automatic
   float* y_rows;        // [S_pad, H] fp32 per-position expert outputs (MOE_COMBINE=rows only)
   int combine_mode;     // MOE_COMBINE: 0/1 fused fp32 reductions (default), 2 stored rows
+  int inject;           // moe_set_fault_injection mode
 };
 
 
@@ -300,6 +301,7 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.perm = c->perm; g.topk_w = topk_w; g.out_acc = c->out_acc;
   g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
   g.y_rows = nullptr;
+  g.inject = c->inject;
   mark(MOE_STAGE_GEMM1);
   if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -407,6 +409,12 @@ moe_status moe_profile_read(moe_ctx* c, float* avg_ms, int* calls) {
   for (int st = 0; st < MOE_NUM_STAGES; ++st) avg_ms[st] = n ? (float)(sum[st] / n) : 0.0f;
   if (calls) *calls = n;
   c->prof_calls = 0;
+  return MOE_OK;
+}
+
+moe_status moe_set_fault_injection(moe_ctx* c, int mode) {
+  if (!c || mode < 0 || mode > 1) return MOE_ERR_INVALID_ARG;
+  c->inject = mode;
   return MOE_OK;
 }
 

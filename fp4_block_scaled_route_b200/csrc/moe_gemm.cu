@@ -220,7 +220,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             ok = mbar_wait(&mdone[prev % NMD], (uint32_t)(prev / NMD) & 1u, abort);
           }
           if (ok) {
-            mbar_arrive_expect_tx(&full[stage], C::TX_BYTES);
+            // Failure-injection hook: CTA 0's first stage expects 16 bytes that
+            // never arrive, so the MMA warp's bounded wait runs out (the load
+            // itself completes; nothing is left in flight).
+            const uint32_t extra = (p.inject == 1 && KIND == 1 && it == 0 && blockIdx.x == 0) ? 16u : 0u;
+            mbar_arrive_expect_tx(&full[stage], C::TX_BYTES + extra);
             uint8_t* a = sA + stage * NA * C::A_BYTES;
             tma_load_2d(&tmA, &full[stage], a, kb * 128, row0, pol_w);
             if constexpr (KIND == 1) tma_load_2d(&tmA, &full[stage], a + C::A_BYTES, kb * 128, row1, pol_w);

@@ -47,6 +47,7 @@ struct GemmParams {
   const int32_t* num_tiles;
   int32_t* status;
   float* y_rows;          // GEMM2: non-null = store fp32 rows [S_pad, H] instead of the fused combine
+  int inject;             // failure-injection test hook (0 in normal use), see moe_set_fault_injection
 };
 
 struct CombineParams {

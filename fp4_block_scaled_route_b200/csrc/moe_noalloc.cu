@@ -185,6 +185,7 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   g.perm = rp.perm; g.topk_w = topk_w; g.out_acc = acc;
   g.tiles = rp.tiles; g.num_tiles = rp.num_tiles; g.status = status;
   g.y_rows = nullptr;  // fused combine into the fp32 accumulator
+  g.inject = 0;
   if (moe::launch_gemm1(wfmt, BN, g_num_sms[dev], tw13, txq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
   g.kblocks = I / 128;
   g.wscale = static_cast<const float*>(s2);

@@ -41,6 +41,7 @@ SIGNATURES = {
     "moe_get_activations": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_last_config": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "moe_set_fault_injection": (_i, [_vp, _i]),
     "moe_profile_enable": (_i, [_vp, _i]),
     "moe_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i)]),
     "moe_forward_noalloc": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
@@ -132,6 +133,10 @@ def moe_last_config(ctx):
 
 MOE_NUM_STAGES = 5
 STAGE_NAMES = ("route", "quant", "gemm1_swiglu_requant", "gemm2_combine", "finalize")
+
+
+def moe_set_fault_injection(ctx, mode) -> int:
+    return lib().moe_set_fault_injection(ctx, mode)
 
 
 def moe_profile_enable(ctx, on) -> int:

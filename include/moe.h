@@ -148,6 +148,15 @@ moe_status moe_get_device_status(moe_ctx* ctx, void* stream);
  * last moe_forward() used; debug / benchmark entry point. */
 moe_status moe_last_config(moe_ctx* ctx, int* tile_n, int* grid);
 
+/* moe_set_fault_injection -- failure-detection test hook.  mode 1: every
+ * following moe_forward() on this context makes one pipeline wait of its
+ * GEMM1 run out (CTA 0's first stage expects 16 bytes that never arrive), so
+ * the bounded wait gives up after about a second, the kernel drains, frees
+ * its tensor memory and returns, and moe_get_device_status() reports
+ * MOE_ERR_TIMEOUT; that call's output is invalid.  mode 0 (default) turns
+ * it off; the context stays usable.  Nothing faults, traps or hangs. */
+moe_status moe_set_fault_injection(moe_ctx* ctx, int mode);
+
 /* Kernel stages of one moe_forward(), in launch order (profiling index). */
 enum {
   MOE_STAGE_ROUTE = 0,     /* counts, prefix sum, permutation, tile list */

@@ -57,6 +57,7 @@ def test_host_argument_checks_without_gpu(libmoe):
     assert libmoe.moe_create(256, 128, 8, 2, 0, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_forward(None, 1, None, None, None, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_pack_mxfp4_scales(None, None, 128, 128, None) == moe.MOE_ERR_INVALID_ARG
+    assert libmoe.moe_set_fault_injection(None, 1) == moe.MOE_ERR_INVALID_ARG
 
 
 def test_product_path_does_not_use_the_oracle():
