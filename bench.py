@@ -214,6 +214,22 @@ def build_layer(args, device):
 
 
 # ---------------------------------------------------------------------------
+def replica_throughput(dist, device, local_ms: float, local_bytes: float, steps: int):
+    """Whole-job rate of independent replicas: the slowest rank's device time
+    (max over ranks) and the bytes all ranks streamed (sum over ranks).
+    Returns (ms_max, bytes_total, GB/s)."""
+    ms, nbytes = float(local_ms), float(local_bytes)
+    if dist is not None:
+        import torch
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        b = torch.tensor([nbytes], device=device, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        dist.all_reduce(b, op=dist.ReduceOp.SUM)
+        ms, nbytes = float(t.item()), float(b.item())
+    return ms, nbytes, nbytes / (ms / steps * 1e-3) / 1e9
+
+
+# ---------------------------------------------------------------------------
 def cpu_baseline(L, min_seconds=10.0, max_slots=None):
     """The oracle on a bounded sample of the workload, repeated until about
     min_seconds of CPU time: the first n (token, expert) slots, n doubling from
@@ -378,12 +394,8 @@ def main():
     moe.moe_profile_enable(layer.ctx, 0)
     if layer.device_status() != moe.MOE_OK:
         raise RuntimeError("device status not OK after the timed region")
-    if dist:
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms, _, value = replica_throughput(dist, dev, ms, st["weight_bytes"], args.steps)
     ms_step = ms / args.steps
-    value = world * st["weight_bytes"] / (ms_step * 1e-3) / 1e9
 
     # ---- end to end through the C ABI with host buffers ----
     e2e = None
@@ -411,13 +423,9 @@ def main():
             step_e2e()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
-        ms_e = ev0.elapsed_time(ev1)
-        if dist:
-            t = torch.tensor([ms_e], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms_e = float(t.item())
+        ms_e, _, e2e_value = replica_throughput(dist, dev, ev0.elapsed_time(ev1), st["weight_bytes"], args.steps)
         h2d = x_h.numel() * 2 + ids_h.numel() * 4 + w_h.numel() * 4
-        e2e = {"value": world * st["weight_bytes"] / (ms_e / args.steps * 1e-3) / 1e9, "unit": "GB/s",
+        e2e = {"value": e2e_value, "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": out_h.numel() * 2,
                "ms_per_step": ms_e / args.steps}
 
