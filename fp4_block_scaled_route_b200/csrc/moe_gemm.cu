@@ -59,11 +59,15 @@ struct GemmCfg {
   // through TMA at only ~47 GB/s, and one thread issues a tcgen05.mma only
   // every ~100 cycles whatever N is, which for 4-bit weights is below the
   // HBM rate; two of each double both.  Warpgroups 1..CG: the epilogue.
-  static constexpr int NPROD = 2;
+  // The epilogue warps need not start at a warpgroup boundary: TMEM lane
+  // access depends only on the warp index mod 4, and any 4 consecutive warps
+  // cover the 4 lane quarters.  Tiles of 64 tokens or more keep two producers
+  // so that the epilogue's accumulators fit in the per-thread registers.
+  static constexpr int NPROD = (BN >= 64) ? 2 : 3;
   static constexpr int NMMA = 2;
   static constexpr int MMA_WARP = NPROD;  // first MMA warp; allocates TMEM
-  static constexpr int EPI_WARP0 = 4;
-  static constexpr int THREADS = 128 + EPI_THREADS;
+  static constexpr int EPI_WARP0 = NPROD + NMMA;
+  static constexpr int THREADS = 32 * EPI_WARP0 + EPI_THREADS;
   static constexpr int MAX_STAGES = 12;
   // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
   // the promoting epilogue (short K steps would otherwise be latency bound).
