@@ -288,6 +288,7 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   QuantParams qp;
   qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs;
+  qp.xs_ld = c->S_pad;
   qp.out_acc = rows ? nullptr : c->out_acc;
   mark(MOE_STAGE_QUANT);
   if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
@@ -297,6 +298,7 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.kblocks = H / 128;
   g.wscale = static_cast<const float*>(s13);
   g.ascale = c->xs;
+  g.scale_ld = c->S_pad;
   g.hq = c->hq; g.hs = c->hs;
   g.perm = c->perm; g.topk_w = topk_w; g.out_acc = c->out_acc;
   g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
@@ -355,9 +357,33 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
   const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
   cudaError_t e = cudaSuccess;
   if (xq && P && e == cudaSuccess) e = cudaMemcpy(xq, c->xq, P * c->H, cudaMemcpyDefault);
-  if (xs && P && e == cudaSuccess) e = cudaMemcpy(xs, c->xs, sizeof(float) * P * (c->H / 128), cudaMemcpyDefault);
   if (hq && P && e == cudaSuccess) e = cudaMemcpy(hq, c->hq, P * c->I, cudaMemcpyDefault);
-  if (hs && P && e == cudaSuccess) e = cudaMemcpy(hs, c->hs, sizeof(float) * P * (c->I / 128), cudaMemcpyDefault);
+  // The scales are stored K-block major on the device ([K/128][S_pad]); the
+  // caller gets them position major ([P][K/128]).
+  auto scales = [&](float* dst, const float* src, int kb) {
+    if (!dst || !P || e != cudaSuccess) return;
+    float* tmp = new (std::nothrow) float[(size_t)kb * P];
+    if (!tmp) {
+      e = cudaErrorMemoryAllocation;
+      return;
+    }
+    e = cudaMemcpy2D(tmp, P * sizeof(float), src, (size_t)c->S_pad * sizeof(float), P * sizeof(float), kb,
+                     cudaMemcpyDeviceToHost);
+    if (e == cudaSuccess) {
+      float* stage = new (std::nothrow) float[(size_t)kb * P];
+      if (!stage) {
+        e = cudaErrorMemoryAllocation;
+      } else {
+        for (size_t i = 0; i < P; ++i)
+          for (int b = 0; b < kb; ++b) stage[i * kb + b] = tmp[(size_t)b * P + i];
+        e = cudaMemcpy(dst, stage, sizeof(float) * kb * P, cudaMemcpyDefault);
+        delete[] stage;
+      }
+    }
+    delete[] tmp;
+  };
+  scales(xs, c->xs, c->H / 128);
+  scales(hs, c->hs, c->I / 128);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

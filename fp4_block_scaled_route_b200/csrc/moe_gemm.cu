@@ -100,7 +100,7 @@ struct GemmCfg {
   static constexpr int TX_BYTES = NA * A_TX + B_BYTES + SF_BYTES;
   static_assert(STAGES >= 2, "shared memory too small");
   static_assert(USED_COLS <= 512, "TMEM too small");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 128, "BN");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 64, "BN");
 };
 
 // Bounded wait that ignores the abort word (used to drain in-flight copies
@@ -357,8 +357,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       const int4 tile = p.tiles[ti];
       const int e = tile.x, p0 = tile.y, nv = tile.z;
       for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
-        const int j = i / KB, kb = i % KB;
-        asc[kb * BN + j] = p.ascale[(size_t)(p0 + j) * KB + kb];
+        const int kb = i / BN, j = i % BN;
+        asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
       }
       if constexpr (WFMT == 0) {
         for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
             if (j < nv) {
               p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[c], sc)));
-              if (row == 0) p.hs[(size_t)(p0 + j) * (p.I / 128) + rt] = sc;
+              if (row == 0) p.hs[(size_t)rt * p.scale_ld + p0 + j] = sc;
             }
           }
         }
@@ -551,8 +551,9 @@ cudaError_t gemm_setup(int wfmt) {
 #define MOE_SET(K, B, W) \
   if (e == cudaSuccess) e = set_attr<K, B, W>();
   if (wfmt == 0) {
-    MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0) MOE_SET(1, 128, 0)
-    MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0) MOE_SET(2, 128, 0)
+    MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0)
+    MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0)
+    if (e == cudaSuccess) e = gemm_tm_setup();
   } else {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
     MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
@@ -568,7 +569,7 @@ cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 16: return launch<1, 16, 0>(grid, tw, tx, p, s);
       case 32: return launch<1, 32, 0>(grid, tw, tx, p, s);
       case 64: return launch<1, 64, 0>(grid, tw, tx, p, s);
-      case 128: return launch<1, 128, 0>(grid, tw, tx, p, s);
+      case 128: return launch_gemm1_tm(grid, tw, tx, p, s);
     }
   } else {
     switch (BN) {
@@ -587,7 +588,7 @@ cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 16: return launch<2, 16, 0>(grid, tw, th, p, s);
       case 32: return launch<2, 32, 0>(grid, tw, th, p, s);
       case 64: return launch<2, 64, 0>(grid, tw, th, p, s);
-      case 128: return launch<2, 128, 0>(grid, tw, th, p, s);
+      case 128: return launch_gemm2_tm(grid, tw, th, p, s);
     }
   } else {
     switch (BN) {

@@ -29,7 +29,8 @@ struct QuantParams {
   const uint16_t* x;      // bf16 [T, H]
   const int32_t* inv;     // [P]
   uint8_t* xq;            // E4M3 [S_pad, H]   rows in routing order
-  float* xs;              // [S_pad, H/128]
+  float* xs;              // [H/128, xs_ld]    K-block major: one row of position scales per K block
+  int xs_ld;              // = S_pad
   float* out_acc;         // [T, H] zeroed here (null: not needed)
 };
 
@@ -37,9 +38,10 @@ struct GemmParams {
   int H, I, k, S;         // S = T*k routed slots
   int kblocks;            // K / 128
   const float* wscale;    // FP8: fp32 [NE, rows/128, K/128]; MXFP4: packed E8M0 atoms
-  const float* ascale;    // activation scales [S_pad, K/128]
+  const float* ascale;    // activation scales [K/128, scale_ld], K-block major
+  int scale_ld;           // = S_pad (row length of ascale and hs)
   uint8_t* hq;            // GEMM1: E4M3 [S_pad, I]
-  float* hs;              // GEMM1: [S_pad, I/128]
+  float* hs;              // GEMM1: [I/128, scale_ld]
   const int32_t* perm;    // GEMM2: position -> slot
   const float* topk_w;    // GEMM2: [T*k]
   float* out_acc;         // GEMM2: fp32 [T, H]
@@ -68,6 +70,12 @@ cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
                          const GemmParams& p, cudaStream_t s);
 cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
                          const GemmParams& p, cudaStream_t s);
+// Token-major kernels for 128-token tiles (FP8 weights), moe_gemm_tm.cu.
+cudaError_t gemm_tm_setup();
+cudaError_t launch_gemm1_tm(int grid, const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
+                            cudaStream_t s);
+cudaError_t launch_gemm2_tm(int grid, const CUtensorMap& tw, const CUtensorMap& th, const GemmParams& p,
+                            cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s);
 

@@ -174,6 +174,7 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   moe::QuantParams qp;
   qp.T = T; qp.H = H; qp.k = k; qp.n_shared = n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = rp.inv; qp.xq = xq; qp.xs = xs; qp.out_acc = acc;
+  qp.xs_ld = (int)S_pad;
   if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::GemmParams g;
@@ -181,6 +182,7 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   g.kblocks = H / 128;
   g.wscale = static_cast<const float*>(s13);
   g.ascale = xs;
+  g.scale_ld = (int)S_pad;
   g.hq = hq; g.hs = hs;
   g.perm = rp.perm; g.topk_w = topk_w; g.out_acc = acc;
   g.tiles = rp.tiles; g.num_tiles = rp.num_tiles; g.status = status;

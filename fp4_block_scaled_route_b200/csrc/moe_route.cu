@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
     for (int i = 0; i < 4; ++i) packed |= f32_to_e4m3(__fdiv_rn(f[i], sc)) << (8 * i);
     for (int r = 0; r < nrows; ++r) {
       *reinterpret_cast<uint32_t*>(p.xq + (size_t)rows[r] * H + g * 128 + lane * 4) = packed;
-      if (lane == 0) p.xs[(size_t)rows[r] * HB + g] = sc;
+      if (lane == 0) p.xs[(size_t)g * p.xs_ld + rows[r]] = sc;
     }
   }
   if (p.out_acc) {
