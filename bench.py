@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--green-ctx", type=int, default=0,
+                    help="run the dispatch kernels in a green context of >= N SMs and the GEMMs on the rest")
     return ap.parse_args()
 
 
@@ -343,6 +345,7 @@ def main():
     ids_np = L.ids.cpu().numpy()
     st = workload_stats(L, ids_np)
     layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
+    green = layer.set_green_ctx(args.green_ctx) if args.green_ctx else None
     if L.wfmt == synth.WFMT_MXFP4:
         w13, s13, w2, s2 = L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2)
     else:
@@ -469,7 +472,8 @@ def main():
                    "wfmt": ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32"][L.wfmt], "n_shared": L.n_shared,
                    "experts_touched": st["experts_touched"], "weight_bytes_per_step": st["weight_bytes"],
                    "l2": "inputs larger than L2 (weights streamed per step exceed the 126 MB L2); no flush",
-                   "parallelism": "replicas" if world > 1 else "single GPU"},
+                   "parallelism": "replicas" if world > 1 else "single GPU",
+                   "green_ctx": {"dispatch_sms": green[0], "gemm_sms": green[1]} if green else None},
         "us_per_layer": ms_step * 1e3,
         "tflops": st["flops"] / (ms_step * 1e-3) / 1e12,
         "hbm_frac_of_step": frac_step,

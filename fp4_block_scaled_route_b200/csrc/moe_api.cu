@@ -39,6 +39,12 @@ struct moe_ctx {
   float* y_rows;        // [S_pad, H] fp32 per-position expert outputs (MOE_COMBINE=rows only)
   int combine_mode;     // MOE_COMBINE: 0/1 fused fp32 reductions (default), 2 stored rows
   int inject;           // moe_set_fault_injection mode
+  // Green-Context partition (moe_set_green_ctx): dispatch kernels on gc_sms
+  // SMs, the grouped GEMMs on the remaining gc_gemm_sms.
+  int gc_sms, gc_gemm_sms;
+  CUgreenCtx gc_small, gc_large;
+  CUstream gs_small, gs_large;
+  cudaEvent_t gev_in, gev_disp, gev_done;
 };
 
 
@@ -64,6 +70,44 @@ EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+// Green-Context driver entry points (CUDA 12.4+ drivers), fetched at run time
+// like cuTensorMapEncodeTiled so the library still loads without them.
+struct GreenFns {
+  CUresult (*device_get)(CUdevice*, int);
+  CUresult (*get_dev_resource)(CUdevice, CUdevResource*, CUdevResourceType);
+  CUresult (*split_by_count)(CUdevResource*, unsigned int*, const CUdevResource*, CUdevResource*, unsigned int,
+                             unsigned int);
+  CUresult (*generate_desc)(CUdevResourceDesc*, CUdevResource*, unsigned int);
+  CUresult (*create)(CUgreenCtx*, CUdevResourceDesc, CUdevice, unsigned int);
+  CUresult (*destroy)(CUgreenCtx);
+  CUresult (*stream_create)(CUstream*, CUgreenCtx, unsigned int, int);
+  CUresult (*stream_destroy)(CUstream);
+  bool ok;
+};
+
+template <typename F>
+bool driver_fn(const char* name, F* out) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return false;
+  *out = reinterpret_cast<F>(p);
+  return true;
+}
+
+const GreenFns& green_fns() {
+  static GreenFns g = [] {
+    GreenFns f = {};
+    f.ok = driver_fn("cuDeviceGet", &f.device_get) && driver_fn("cuDeviceGetDevResource", &f.get_dev_resource) &&
+           driver_fn("cuDevSmResourceSplitByCount", &f.split_by_count) &&
+           driver_fn("cuDevResourceGenerateDesc", &f.generate_desc) && driver_fn("cuGreenCtxCreate", &f.create) &&
+           driver_fn("cuGreenCtxDestroy", &f.destroy) && driver_fn("cuGreenCtxStreamCreate", &f.stream_create) &&
+           driver_fn("cuStreamDestroy", &f.stream_destroy);
+    return f;
+  }();
+  return g;
 }
 
 // 2-D map over a row-major matrix [rows, inner] (inner contiguous), box
@@ -147,6 +191,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
     if (!strcmp(env, "atomic")) c->combine_mode = 1;
     if (!strcmp(env, "rows")) c->combine_mode = 2;
   }
+  if (const char* env = getenv("MOE_GREEN_CTX")) c->gc_sms = atoi(env);  // applied below, once created
   if (const char* env = getenv("MOE_TILE_N")) {
     const int v = atoi(env);
     if (v == 16 || v == 32 || v == 64 || (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128)) c->tile_n_override = v;
@@ -199,6 +244,15 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->hs = reinterpret_cast<float*>(b + o_hs);
   c->out_acc = reinterpret_cast<float*>(b + o_acc);
   c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
+  const int want_green = c->gc_sms;
+  c->gc_sms = 0;
+  if (want_green > 0) {
+    const moe_status gs = moe_set_green_ctx(c, want_green);
+    if (gs != MOE_OK) {
+      moe_destroy(c);
+      return gs;
+    }
+  }
   *out = c;
   return MOE_OK;
 }
@@ -210,9 +264,68 @@ static void prof_free(moe_ctx* c) {
   c->prof_ev = nullptr;
 }
 
+static void green_free(moe_ctx* c) {
+  const GreenFns& g = green_fns();
+  if (c->gs_small) g.stream_destroy(c->gs_small);
+  if (c->gs_large) g.stream_destroy(c->gs_large);
+  if (c->gc_small) g.destroy(c->gc_small);
+  if (c->gc_large) g.destroy(c->gc_large);
+  if (c->gev_in) cudaEventDestroy(c->gev_in);
+  if (c->gev_disp) cudaEventDestroy(c->gev_disp);
+  if (c->gev_done) cudaEventDestroy(c->gev_done);
+  c->gs_small = c->gs_large = nullptr;
+  c->gc_small = c->gc_large = nullptr;
+  c->gev_in = c->gev_disp = c->gev_done = nullptr;
+  c->gc_sms = c->gc_gemm_sms = 0;
+}
+
+moe_status moe_set_green_ctx(moe_ctx* c, int dispatch_sms) {
+  if (!c || dispatch_sms < 0) return MOE_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+  green_free(c);
+  if (dispatch_sms == 0) return MOE_OK;
+  const GreenFns& g = green_fns();
+  if (!g.ok) return MOE_ERR_UNSUPPORTED;
+  CUdevice dev;
+  CUdevResource all = {}, small = {}, rest = {};
+  unsigned int groups = 1;
+  if (g.device_get(&dev, c->dev) != CUDA_SUCCESS ||
+      g.get_dev_resource(dev, &all, CU_DEV_RESOURCE_TYPE_SM) != CUDA_SUCCESS ||
+      g.split_by_count(&small, &groups, &all, &rest, 0, (unsigned int)dispatch_sms) != CUDA_SUCCESS || groups != 1)
+    return MOE_ERR_UNSUPPORTED;
+  if (small.sm.smCount == 0 || rest.sm.smCount < 8) return MOE_ERR_UNSUPPORTED;
+  CUdevResourceDesc dsmall = nullptr, drest = nullptr;
+  moe_status st = MOE_OK;
+  if (g.generate_desc(&dsmall, &small, 1) != CUDA_SUCCESS || g.generate_desc(&drest, &rest, 1) != CUDA_SUCCESS ||
+      g.create(&c->gc_small, dsmall, dev, CU_GREEN_CTX_DEFAULT_STREAM) != CUDA_SUCCESS ||
+      g.create(&c->gc_large, drest, dev, CU_GREEN_CTX_DEFAULT_STREAM) != CUDA_SUCCESS ||
+      g.stream_create(&c->gs_small, c->gc_small, CU_STREAM_NON_BLOCKING, 0) != CUDA_SUCCESS ||
+      g.stream_create(&c->gs_large, c->gc_large, CU_STREAM_NON_BLOCKING, 0) != CUDA_SUCCESS)
+    st = MOE_ERR_UNSUPPORTED;
+  if (st == MOE_OK && (cudaEventCreateWithFlags(&c->gev_in, cudaEventDisableTiming) != cudaSuccess ||
+                       cudaEventCreateWithFlags(&c->gev_disp, cudaEventDisableTiming) != cudaSuccess ||
+                       cudaEventCreateWithFlags(&c->gev_done, cudaEventDisableTiming) != cudaSuccess))
+    st = MOE_ERR_CUDA;
+  if (st != MOE_OK) {
+    green_free(c);
+    return st;
+  }
+  c->gc_sms = (int)small.sm.smCount;
+  c->gc_gemm_sms = (int)rest.sm.smCount;
+  return MOE_OK;
+}
+
+moe_status moe_green_ctx_sms(moe_ctx* c, int* dispatch_sms, int* gemm_sms) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (dispatch_sms) *dispatch_sms = c->gc_sms;
+  if (gemm_sms) *gemm_sms = c->gc_gemm_sms;
+  return MOE_OK;
+}
+
 void moe_destroy(moe_ctx* c) {
   if (!c) return;
   cudaDeviceSynchronize();
+  green_free(c);
   prof_free(c);
   cudaFree(c->ws_base);
   delete c;
@@ -230,7 +343,13 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   const int H = c->H, I = c->I, NE = c->NG;
   const int S = T * c->k;
   const int BN = pick_tile_n(c, T);
-  const int grid = c->num_sms;
+  // Green-Context partition: route + quant on the small partition's stream,
+  // GEMMs + output on the large one, ordered by events after the caller's
+  // stream and before its next work.  Otherwise everything runs on `s`.
+  const bool green = c->gc_small != nullptr;
+  cudaStream_t s_disp = green ? reinterpret_cast<cudaStream_t>(c->gs_small) : s;
+  cudaStream_t s_gemm = green ? reinterpret_cast<cudaStream_t>(c->gs_large) : s;
+  const int grid = green ? c->gc_gemm_sms : c->num_sms;
   const bool fp8 = (c->wfmt == MOE_WFMT_FP8_E4M3_B128);
 
   // weight maps (re-encoded only when the caller's pointers change)
@@ -271,15 +390,19 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   cudaEvent_t* ev = nullptr;
   if (c->prof_on && c->prof_calls < kProfMaxCalls) ev = c->prof_ev + (size_t)c->prof_calls++ * kProfEvents;
   auto mark = [&](int i) {
-    if (ev) cudaEventRecord(ev[i], s);
+    if (ev) cudaEventRecord(ev[i], i <= MOE_STAGE_QUANT ? s_disp : s_gemm);
   };
+  if (green) {
+    if (cudaEventRecord(c->gev_in, s) != cudaSuccess || cudaStreamWaitEvent(s_disp, c->gev_in, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
 
   RouteParams rp;
   rp.T = T; rp.k = c->k; rp.E = c->E; rp.n_shared = c->n_shared; rp.BN = BN;
   rp.ids = ids; rp.counts = c->counts; rp.offsets = c->offsets; rp.perm = c->perm; rp.inv = c->inv;
   rp.tiles = c->tiles; rp.num_tiles = c->num_tiles; rp.status = c->status;
   mark(MOE_STAGE_ROUTE);
-  if (moe::launch_route(rp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 
   const int P = S + c->n_shared * T;
   const bool rows = c->y_rows != nullptr;
@@ -291,7 +414,11 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   qp.xs_ld = c->S_pad;
   qp.out_acc = rows ? nullptr : c->out_acc;
   mark(MOE_STAGE_QUANT);
-  if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_quant(qp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
+  if (green) {
+    if (cudaEventRecord(c->gev_disp, s_disp) != cudaSuccess || cudaStreamWaitEvent(s_gemm, c->gev_disp, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
 
   GemmParams g;
   g.H = H; g.I = I; g.k = c->k; g.S = S;
@@ -305,25 +432,29 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.y_rows = nullptr;
   g.inject = c->inject;
   mark(MOE_STAGE_GEMM1);
-  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
   g.kblocks = I / 128;
   g.wscale = static_cast<const float*>(s2);
   g.ascale = c->hs;
   mark(MOE_STAGE_GEMM2);
   g.y_rows = rows ? c->y_rows : nullptr;
-  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
   mark(MOE_STAGE_FINALIZE);
   if (rows) {
     moe::CombineParams cp;
     cp.T = T; cp.H = H; cp.k = c->k; cp.n_shared = c->n_shared;
     cp.y_rows = c->y_rows; cp.inv = c->inv; cp.topk_w = topk_w; cp.out = static_cast<uint16_t*>(out);
-    if (moe::launch_combine(cp, s) != cudaSuccess) return MOE_ERR_CUDA;
-  } else if (moe::launch_finalize(c->out_acc, static_cast<uint16_t*>(out), (long long)T * H, s) != cudaSuccess) {
+    if (moe::launch_combine(cp, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (moe::launch_finalize(c->out_acc, static_cast<uint16_t*>(out), (long long)T * H, s_gemm) != cudaSuccess) {
     return MOE_ERR_CUDA;
   }
   mark(MOE_NUM_STAGES);
+  if (green) {
+    if (cudaEventRecord(c->gev_done, s_gemm) != cudaSuccess || cudaStreamWaitEvent(s, c->gev_done, 0) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
   c->last_T = T;
   c->last_bn = BN;
   c->last_grid = grid;

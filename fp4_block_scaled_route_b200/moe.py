@@ -45,6 +45,8 @@ SIGNATURES = {
     "moe_profile_enable": (_i, [_vp, _i]),
     "moe_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i)]),
     "moe_forward_noalloc": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_set_green_ctx": (_i, [_vp, _i]),
+    "moe_green_ctx_sms": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
 }
 
@@ -139,6 +141,16 @@ def moe_set_fault_injection(ctx, mode) -> int:
     return lib().moe_set_fault_injection(ctx, mode)
 
 
+def moe_set_green_ctx(ctx, dispatch_sms) -> int:
+    return lib().moe_set_green_ctx(ctx, dispatch_sms)
+
+
+def moe_green_ctx_sms(ctx):
+    d, g = _i(), _i()
+    _check(lib().moe_green_ctx_sms(ctx, ctypes.byref(d), ctypes.byref(g)), "moe_green_ctx_sms")
+    return d.value, g.value
+
+
 def moe_profile_enable(ctx, on) -> int:
     return lib().moe_profile_enable(ctx, on)
 
@@ -223,6 +235,11 @@ class MoeLayer:
 
     def last_config(self):
         return moe_last_config(self.ctx)
+
+    def set_green_ctx(self, dispatch_sms):
+        """Green-Context partition: dispatch kernels on >= dispatch_sms SMs, GEMMs on the rest (0 = off)."""
+        _check(moe_set_green_ctx(self.ctx, dispatch_sms), "moe_set_green_ctx")
+        return moe_green_ctx_sms(self.ctx)
 
 
 def pack_mxfp4_scales(s, stream=None):

@@ -157,6 +157,28 @@ moe_status moe_last_config(moe_ctx* ctx, int* tile_n, int* grid);
  * it off; the context stays usable.  Nothing faults, traps or hangs. */
 moe_status moe_set_fault_injection(moe_ctx* ctx, int mode);
 
+/* moe_set_green_ctx -- optional Green-Context partition of the GPU, the
+ * single-GPU form of the GC-MoE abstract's split into a small dispatch
+ * partition and a large compute partition (CUDA Green Contexts).
+ * dispatch_sms > 0: every following moe_forward() on this context runs the
+ * dispatch kernels (route, quant) in a green context of at least
+ * dispatch_sms SMs (the driver rounds up; a multiple of 8 on this GPU) and
+ * the grouped GEMMs and the output kernel in a green context of the
+ * remaining SMs, each on its own stream; events order them after the
+ * caller's stream and make the caller's stream wait for the result, so the
+ * call keeps its stream semantics.  The two partitions are ordered by events,
+ * not by flags polled across kernels: the driver does not guarantee that
+ * kernels of two green contexts run at the same time, so no kernel waits for
+ * another one while running.  dispatch_sms == 0 removes the partition
+ * (the default; the environment variable MOE_GREEN_CTX=<n> sets it at
+ * create time).  Synchronises the device.  Returns MOE_ERR_UNSUPPORTED when
+ * the driver has no green contexts or the split fails.  A measured option:
+ * the library's default is off. */
+moe_status moe_set_green_ctx(moe_ctx* ctx, int dispatch_sms);
+
+/* moe_green_ctx_sms -- SM counts of the current partition (0, 0 when off). */
+moe_status moe_green_ctx_sms(moe_ctx* ctx, int* dispatch_sms, int* gemm_sms);
+
 /* Kernel stages of one moe_forward(), in launch order (profiling index). */
 enum {
   MOE_STAGE_ROUTE = 0,     /* counts, prefix sum, permutation, tile list */
