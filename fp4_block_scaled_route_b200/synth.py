@@ -182,3 +182,12 @@ def make_layer(cfg: dict, seed: int, device="cpu", T: Optional[int] = None,
 def bf16_bits(x: torch.Tensor) -> np.ndarray:
     """bf16 tensor -> numpy uint16 bit patterns (host)."""
     return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def make_router(T: int, H: int, E: int, seed: int, device="cpu"):
+    """Seeded router inputs: x ~ N(0,1) and router weights ~ N(0, 1/H), both
+    rounded to bf16, so that the logits x . Wr^T have about unit variance."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    x = torch.randn(T, H, generator=g).to(torch.bfloat16)
+    wr = (torch.randn(E, H, generator=g) / float(np.sqrt(H))).to(torch.bfloat16)
+    return x.to(device), wr.to(device)

@@ -77,6 +77,8 @@ def lib() -> ctypes.CDLL:
             L.orc_quant_row_f32.argtypes = [ctypes.c_int, vp, vp, vp]
             L.orc_forward.restype = ctypes.c_int
             L.orc_forward.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 13
+            L.orc_router.restype = ctypes.c_int
+            L.orc_router.argtypes = [ctypes.c_int] * 4 + [vp] * 5
             L.orc_num_threads.restype = ctypes.c_int
             L.orc_num_threads.argtypes = []
             _lib = L
@@ -209,3 +211,23 @@ def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
         dbg["hs"] = dbg["hs"][:P]
         res.update(dbg)
     return res
+
+
+def router(x_bf16_bits, wr_bf16_bits, k: int, *, with_logits: bool = False):
+    """Fused router oracle: (ids [T,k] int32, w [T,k] fp32[, logits [T,E] fp32])."""
+    x = np.ascontiguousarray(x_bf16_bits, dtype=np.uint16)
+    wr = np.ascontiguousarray(wr_bf16_bits, dtype=np.uint16)
+    T, H = x.shape
+    E = wr.shape[0]
+    assert wr.shape[1] == H
+    ids = np.zeros((T, k), np.int32)
+    w = np.zeros((T, k), np.float32)
+    lg = np.zeros((T, E), np.float32) if with_logits else None
+    L = lib()
+    vp = ctypes.c_void_p
+    r = L.orc_router(T, H, E, k, x.ctypes.data_as(vp), wr.ctypes.data_as(vp),
+                     lg.ctypes.data_as(vp) if lg is not None else None, ids.ctypes.data_as(vp),
+                     w.ctypes.data_as(vp))
+    if r != 0:
+        raise ValueError("orc_router: bad arguments")
+    return (ids, w, lg) if with_logits else (ids, w)

@@ -396,3 +396,41 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   free(xq); free(xs); free(xd); free(Y);
   return dropped;
 }
+
+/* ----------------------------------------------------------------------- */
+/* Fused router: DeepGEMM 26/09 news page ("Mega Gate": routing GEMM + MoE
+ * routing ops in one kernel).  Reading: see moe_oracle.h.                   */
+int orc_router(int T, int H, int E, int k, const uint16_t* x, const uint16_t* wr,
+               float* logits, int32_t* ids, float* w) {
+  if (T < 0 || H <= 0 || E <= 0 || E > 1024 || k <= 0 || k > E) return -1;
+  int t;
+#pragma omp parallel for schedule(static)
+  for (t = 0; t < T; ++t) {
+    float lg[1024];
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += (double)orc_bf16_decode(x[(size_t)t * H + h]) * (double)orc_bf16_decode(wr[(size_t)e * H + h]);
+      lg[e] = (float)acc;
+      if (logits) logits[(size_t)t * E + e] = lg[e];
+    }
+    /* k rounds of "largest remaining, lowest index first" */
+    unsigned char taken[1024];
+    memset(taken, 0, sizeof(taken));
+    for (int j = 0; j < k; ++j) {
+      int best = -1;
+      for (int e = 0; e < E; ++e) {
+        if (taken[e]) continue;
+        if (best < 0 || lg[e] > lg[best]) best = e;
+      }
+      taken[best] = 1;
+      ids[(size_t)t * k + j] = best;
+    }
+    /* softmax over the chosen logits (max subtracted) */
+    const double m = (double)lg[ids[(size_t)t * k]];
+    double z = 0.0;
+    for (int j = 0; j < k; ++j) z += exp((double)lg[ids[(size_t)t * k + j]] - m);
+    for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = (float)(exp((double)lg[ids[(size_t)t * k + j]] - m) / z);
+  }
+  return 0;
+}

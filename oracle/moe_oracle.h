@@ -99,6 +99,21 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
                 float* out_f32, uint16_t* out_bf16,
                 uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs);
 
+/* ---- fused router (a "Mega Gate": routing GEMM + top-k in one step) ----
+ * DeepGEMM 26/09 news page: the router GEMM and the MoE routing ops fused
+ * into one kernel.  The page gives no formula; reading taken (plainest form
+ * consistent with the layer's inputs): logits = x . Wr^T with x bf16 [T,H]
+ * and Wr bf16 [E,H]; the k largest logits per token, ties to the lower expert
+ * index, in descending order; combine weights = softmax over the k chosen
+ * logits (equal to the full softmax renormalised over the chosen experts).
+ * Logits are the exact dot products (fp64 accumulation, one rounding to
+ * fp32); the selection compares those fp32 values; the weights are computed
+ * in fp64 from them and rounded to fp32.
+ * Outputs: logits [T,E] (may be NULL), ids [T,k], w [T,k].  Returns -1 on bad
+ * arguments (k > E, E > 1024), else 0. */
+int orc_router(int T, int H, int E, int k, const uint16_t* x, const uint16_t* wr,
+               float* logits, int32_t* ids, float* w);
+
 /* OpenMP threads the oracle will use (1 when built without OpenMP). */
 int orc_num_threads(void);
 
