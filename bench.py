@@ -54,6 +54,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--router", action="store_true",
+                    help="also time the fused router (moe_router_topk) on seeded router weights of this shape")
     ap.add_argument("--green-ctx", type=int, default=0,
                     help="run the dispatch kernels in a green context of >= N SMs and the GEMMs on the rest")
     return ap.parse_args()
@@ -315,6 +317,35 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------------------
+def time_router(args, L, layer, dev, stream):
+    """The fused router (logits GEMM + top-k + softmax, one kernel) on seeded
+    bf16 router weights of the layer's shape, timed with CUDA events; the
+    roofline is the larger of its HBM time (x and router weights read once)
+    and its bf16 tensor time."""
+    import torch
+    from fp4_block_scaled_route_b200 import synth
+    _, wr = synth.make_router(L.T, L.H, L.E, 4242, device=dev)
+    ids = torch.empty(L.T, L.k, dtype=torch.int32, device=dev)
+    w = torch.empty(L.T, L.k, dtype=torch.float32, device=dev)
+    for _ in range(5):
+        layer.router(L.x, wr, ids, w, stream=stream)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        layer.router(L.x, wr, ids, w, stream=stream)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = e0.elapsed_time(e1) / args.steps
+    hbm, bf16, src = peaks()
+    nbytes = L.T * L.H * 2 + L.E * L.H * 2 + L.T * L.k * 8
+    flops = 2.0 * L.T * L.H * L.E
+    floor_ms = max(nbytes / (hbm * 1e9), flops / (bf16 * 1e12)) * 1e3
+    return {"us": ms * 1e3, "bytes": nbytes, "GBps": nbytes / (ms * 1e-3) / 1e9, "tflops": flops / (ms * 1e-3) / 1e12,
+            "roofline_us": floor_ms * 1e3, "frac": floor_ms / ms, "peak_source": f"{src} hbm_gbs / bf16_tflops",
+            "launches_per_call": 1}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
@@ -458,6 +489,8 @@ def main():
             dist.destroy_process_group()
         return
 
+    router = time_router(args, L, layer, dev, stream) if args.router else None
+
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(L)
@@ -485,6 +518,8 @@ def main():
         "gpu_launches": moe.MOE_NUM_STAGES * args.steps,  # per timed region
         "clocks": clocks,
     }
+    if router:
+        line["router"] = router
     print(json.dumps(line), flush=True)
     if dist:
         dist.destroy_process_group()

@@ -45,6 +45,11 @@ struct moe_ctx {
   CUgreenCtx gc_small, gc_large;
   CUstream gs_small, gs_large;
   cudaEvent_t gev_in, gev_disp, gev_done;
+  // fused router (moe_router_topk): fp32 logit accumulators and tile counters
+  float* rt_logits;
+  int32_t* rt_counters;
+  const void* c_wr;
+  CUtensorMap tm_wr;
 };
 
 
@@ -111,14 +116,14 @@ const GreenFns& green_fns() {
 }
 
 // 2-D map over a row-major matrix [rows, inner] (inner contiguous), box
-// {128 elements, box_rows}, 128-byte swizzle.
+// {box_inner elements, box_rows}, 128-byte swizzle.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
-              uint64_t row_bytes, uint32_t box_rows, CUtensorMapL2promotion l2) {
+              uint64_t row_bytes, uint32_t box_rows, CUtensorMapL2promotion l2, uint32_t box_inner = 128) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {inner, rows};
   cuuint64_t gstride[1] = {row_bytes};
-  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -218,6 +223,11 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_acc = take(sizeof(float) * (size_t)max_T * H);
   const bool want_rows = c->combine_mode == 2;
   const size_t o_rows = want_rows ? take(sizeof(float) * (size_t)c->S_pad * H) : 0;
+  // fused router workspace (E <= 256, E % 4 == 0): logits of every token tile + a counter per tile
+  const bool want_router = E <= 256 && E % 4 == 0;
+  const size_t rt_tiles = ((size_t)max_T + 127) / 128;
+  const size_t o_rt_logits = want_router ? take(sizeof(float) * rt_tiles * 128 * E) : 0;
+  const size_t o_rt_counters = want_router ? take(sizeof(int32_t) * rt_tiles) : 0;
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     delete c;
@@ -244,6 +254,13 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->hs = reinterpret_cast<float*>(b + o_hs);
   c->out_acc = reinterpret_cast<float*>(b + o_acc);
   c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
+  c->rt_logits = want_router ? reinterpret_cast<float*>(b + o_rt_logits) : nullptr;
+  c->rt_counters = want_router ? reinterpret_cast<int32_t*>(b + o_rt_counters) : nullptr;
+  if (want_router && moe::router_setup(E) != cudaSuccess) {
+    cudaFree(base);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
   const int want_green = c->gc_sms;
   c->gc_sms = 0;
   if (want_green > 0) {
@@ -458,6 +475,47 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   c->last_T = T;
   c->last_bn = BN;
   c->last_grid = grid;
+  return MOE_OK;
+}
+
+moe_status moe_router_topk(moe_ctx* c, int T, const void* x, const void* wr, int32_t* topk_ids, float* topk_w,
+                           void* stream) {
+  if (!c || T < 0 || T > c->max_T) return MOE_ERR_INVALID_ARG;
+  if (!c->rt_logits) return MOE_ERR_UNSUPPORTED;  // E > 256 or E % 4 != 0
+  if (T == 0) return MOE_OK;
+  if (!x || !wr || !topk_ids || !topk_w || !aligned(x, 16) || !aligned(wr, 16) || !aligned(topk_ids, 4) ||
+      !aligned(topk_w, 4))
+    return MOE_ERR_INVALID_ARG;
+  const int H = c->H, E = c->E;
+  const int NP = (E + 15) / 16 * 16;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  CUtensorMap tx;
+  if (!make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, H, (uint64_t)T, (uint64_t)H * 2, 128,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 64))
+    return MOE_ERR_CUDA;
+  if (wr != c->c_wr) {
+    if (!make_map(&c->tm_wr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, wr, H, (uint64_t)E, (uint64_t)H * 2, NP,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 64)) {
+      c->c_wr = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    c->c_wr = wr;
+  }
+  moe::RouterParams rp;
+  rp.T = T; rp.H = H; rp.E = E; rp.k = c->k; rp.N = NP;
+  rp.kblocks = H / 64;
+  const int tiles = (T + 127) / 128;
+  // K splits fill the GPU, but keep at least 8 K blocks per split: every
+  // split adds its partial logits into the same rows with fp32 reductions.
+  int splits = c->num_sms / tiles;
+  if (splits > rp.kblocks / 8) splits = rp.kblocks / 8;
+  if (splits < 1) splits = 1;
+  rp.splits = splits;
+  rp.wbox_rows = NP;
+  rp.tmem_cols = NP <= 32 ? 32 : NP <= 64 ? 64 : NP <= 128 ? 128 : 256;
+  rp.logits = c->rt_logits; rp.counters = c->rt_counters;
+  rp.ids = topk_ids; rp.w = topk_w; rp.status = c->status;
+  if (moe::launch_router(tx, c->tm_wr, rp, s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;
 }
 

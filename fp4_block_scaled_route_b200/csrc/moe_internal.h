@@ -60,6 +60,24 @@ struct CombineParams {
   uint16_t* out;          // bf16 [T, H]
 };
 
+struct RouterParams {
+  int T, H, E, k;
+  int N;                  // MMA N: E rounded up to a multiple of 16 (<= 256)
+  int kblocks;            // H / 64
+  int splits;             // K splits per token tile (grid = tiles x splits)
+  int wbox_rows;          // rows of one router-weight TMA box (= N)
+  int tmem_cols;
+  float* logits;          // fp32 [tiles*128, E], zero between calls
+  int32_t* counters;      // [tiles], zero between calls
+  int32_t* ids;           // [T, k]
+  float* w;               // [T, k]
+  int32_t* status;
+};
+
+size_t router_smem_bytes(int E);
+cudaError_t router_setup(int E);
+cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, const RouterParams& p, cudaStream_t s);
+
 size_t route_smem_bytes(int n_groups);
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);

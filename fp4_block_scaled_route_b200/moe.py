@@ -45,6 +45,7 @@ SIGNATURES = {
     "moe_profile_enable": (_i, [_vp, _i]),
     "moe_profile_read": (_i, [_vp, ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_i)]),
     "moe_forward_noalloc": (_i, [_i, _i, _i, _i, _i, _i, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_router_topk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_set_green_ctx": (_i, [_vp, _i]),
     "moe_green_ctx_sms": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
@@ -141,6 +142,10 @@ def moe_set_fault_injection(ctx, mode) -> int:
     return lib().moe_set_fault_injection(ctx, mode)
 
 
+def moe_router_topk(ctx, T, x, wr, topk_ids, topk_w, stream) -> int:
+    return lib().moe_router_topk(ctx, T, x, wr, topk_ids, topk_w, stream)
+
+
 def moe_set_green_ctx(ctx, dispatch_sms) -> int:
     return lib().moe_set_green_ctx(ctx, dispatch_sms)
 
@@ -235,6 +240,21 @@ class MoeLayer:
 
     def last_config(self):
         return moe_last_config(self.ctx)
+
+    def router(self, x, wr, ids=None, w=None, stream=None):
+        """Fused router: (topk_ids int32 [T,k], topk_w fp32 [T,k]) from x bf16 [T,H] and wr bf16 [E,H]."""
+        import torch
+        T = x.shape[0]
+        if ids is None:
+            ids = torch.empty((T, self.k), dtype=torch.int32, device=x.device)
+        if w is None:
+            w = torch.empty((T, self.k), dtype=torch.float32, device=x.device)
+        for t in (x, wr, ids, w):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("MoeLayer.router needs contiguous CUDA tensors")
+        _check(moe_router_topk(self.ctx, T, _ptr(x), _ptr(wr), _ptr(ids), _ptr(w), _stream_handle(stream)),
+               "moe_router_topk")
+        return ids, w
 
     def set_green_ctx(self, dispatch_sms):
         """Green-Context partition: dispatch kernels on >= dispatch_sms SMs, GEMMs on the rest (0 = off)."""

@@ -157,6 +157,28 @@ moe_status moe_last_config(moe_ctx* ctx, int* tile_n, int* grid);
  * it off; the context stays usable.  Nothing faults, traps or hangs. */
 moe_status moe_set_fault_injection(moe_ctx* ctx, int mode);
 
+/* moe_router_topk -- fused router ("Mega Gate", DeepGEMM 26/09 news page:
+ * the router GEMM and the MoE routing operations in one kernel), producing
+ * the inputs of moe_forward():
+ *   logits[t, e] = sum_h x[t, h] * wr[e, h]  (bf16 inputs, fp32 accumulation)
+ *   topk_ids[t, :] = the k largest logits of token t, in descending order,
+ *                    ties to the lower expert index
+ *   topk_w[t, j]   = softmax over the k chosen logits
+ * (the page names the fusion but no formula; this is the plainest reading).
+ *   x        device bf16 [T, H] row-major (16-byte aligned)
+ *   wr       device bf16 [E, H] row-major router weights (16-byte aligned)
+ *   topk_ids device int32 [T, k] (output), topk_w device fp32 [T, k] (output)
+ * H, E, k and the largest T are the context's.  One kernel launch on
+ * `stream`, asynchronous, no host synchronisation; the context's router
+ * workspace is left zeroed for the next call, so calls on one context must be
+ * stream-ordered.  The fp32 partial logits of the K splits are added with
+ * atomic reductions, so a logit can differ from call to call in its last bits
+ * and a near-tie between the k-th and (k+1)-th expert can resolve either way.
+ * Returns MOE_ERR_UNSUPPORTED when E > 256 or E is not a multiple of 4,
+ * MOE_ERR_INVALID_ARG for null or misaligned pointers or T > max_T. */
+moe_status moe_router_topk(moe_ctx* ctx, int T, const void* x, const void* wr, int32_t* topk_ids, float* topk_w,
+                           void* stream);
+
 /* moe_set_green_ctx -- optional Green-Context partition of the GPU, the
  * single-GPU form of the GC-MoE abstract's split into a small dispatch
  * partition and a large compute partition (CUDA Green Contexts).
