@@ -352,35 +352,83 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     bool ok = true;
     int eit = 0;  // pipeline iteration
     griddep_wait();  // activation scales / combine buffer come from earlier kernels
-    for (int u = blockIdx.x; u < total; u += gridDim.x) {
-      const int rt = C::TILE_MAJOR ? u % NRT : u / num_tiles, ti = C::TILE_MAJOR ? u / NRT : u % num_tiles;
-      const int4 tile = p.tiles[ti];
-      const int e = tile.x, p0 = tile.y, nv = tile.z;
-      for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
-        const int kb = i / BN, j = i % BN;
-        asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
+    // Per-unit inputs of the epilogue: the activation scales of the tile's
+    // columns [KB][BN], the weight block scales [NA][KB] and (GEMM2) the
+    // combine target of every column.  In GEMM1 with tiles of up to 32 tokens
+    // the next unit's tile record and scales are loaded into registers during
+    // the current unit's K loop (record at K block 0, scales at K block 1), so
+    // a unit starts without waiting on memory.  (Doing the same in GEMM2,
+    // routing slot and combine weight included, made it slower.)
+    constexpr bool PREF = BN <= 32 && KIND == 1;
+    constexpr int NPA = PREF ? (BN * KB_MAX + C::EPI_THREADS - 1) / C::EPI_THREADS : 1;
+    auto unit_rt = [&](int uu) { return C::TILE_MAJOR ? uu % NRT : uu / num_tiles; };
+    auto unit_ti = [&](int uu) { return C::TILE_MAJOR ? uu / NRT : uu % num_tiles; };
+    int4 tile_n = make_int4(0, 0, 0, 0);
+    float pa[NPA];
+    float pw = 0.0f;
+    bool have_next = false;
+    auto pref_tile = [&](int un) {
+      have_next = PREF && un < total;
+      if (have_next) tile_n = p.tiles[unit_ti(un)];
+    };
+    auto pref_scales = [&](int un) {
+      if (!have_next) return;
+      const int rtn = unit_rt(un);
+#pragma unroll
+      for (int r = 0; r < NPA; ++r) {
+        const int i = etid + r * C::EPI_THREADS;
+        pa[r] = (i < BN * KB) ? p.ascale[(size_t)(i / BN) * p.scale_ld + tile_n.y + (i % BN)] : 0.0f;
       }
       if constexpr (WFMT == 0) {
-        for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
-          const int a = i / KB, kb = i % KB;
-          const int rb = (a == 0) ? rt : p.I / 128 + rt;
-          wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + rb) * KB + kb];
+        if (etid < NA * KB) {
+          const int a = etid / KB, kb = etid % KB;
+          const int rb = (a == 0) ? rtn : p.I / 128 + rtn;
+          pw = p.wscale[((size_t)tile_n.x * RB + rb) * KB + kb];
         }
       }
-      if constexpr (KIND == 2) {
-        for (int j = etid; j < BN; j += C::EPI_THREADS) {
-          int tok = 0;
-          float w = 0.0f;
-          if (j < nv) {
-            const int slot = p.perm[p0 + j];
-            tok = (slot < S) ? slot / p.k : slot - S;
-            w = (slot < S) ? p.topk_w[slot] : 1.0f;
+    };
+    bool from_regs = false;
+    for (int u = blockIdx.x; u < total; u += gridDim.x) {
+      const int rt = unit_rt(u), ti = unit_ti(u);
+      const int4 tile = from_regs ? tile_n : p.tiles[ti];
+      const int e = tile.x, p0 = tile.y, nv = tile.z;
+      if (from_regs) {
+#pragma unroll
+        for (int r = 0; r < NPA; ++r) {
+          const int i = etid + r * C::EPI_THREADS;
+          if (i < BN * KB) asc[i] = pa[r];
+        }
+        if constexpr (WFMT == 0) {
+          if (etid < NA * KB) wsc[(etid / KB) * KB_MAX + etid % KB] = pw;
+        }
+      } else {
+        for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
+          const int kb = i / BN, j = i % BN;
+          asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
+        }
+        if constexpr (WFMT == 0) {
+          for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
+            const int a = i / KB, kb = i % KB;
+            const int rb = (a == 0) ? rt : p.I / 128 + rt;
+            wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + rb) * KB + kb];
           }
-          slot_tok[j] = tok;
-          slot_w[j] = w;
+        }
+        if constexpr (KIND == 2) {
+          for (int j = etid; j < BN; j += C::EPI_THREADS) {
+            int tok = 0;
+            float w = 0.0f;
+            if (j < nv) {
+              const int slot = p.perm[p0 + j];
+              tok = (slot < S) ? slot / p.k : slot - S;
+              w = (slot < S) ? p.topk_w[slot] : 1.0f;
+            }
+            slot_tok[j] = tok;
+            slot_w[j] = w;
+          }
         }
       }
       named_sync(1, C::EPI_THREADS);
+      const int un = u + gridDim.x;
 
       float acc0[CPT], acc1[CPT];
 #pragma unroll
@@ -403,6 +451,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       named_sync(1, C::EPI_THREADS);
       for (int kb = 0; kb < KB; ++kb, ++eit) {
         if (kb + 1 < KB) fill_cs(kb + 1);
+        if (kb == 0) pref_tile(un);
+        if (kb == (KB > 1 ? 1 : 0)) pref_scales(un);
         if (ok) ok = mbar_wait(&mdone[eit % NMD], (uint32_t)(eit / NMD) & 1u, abort);
         ok = __all_sync(0xFFFFFFFFu, ok);
         if (ok) {
@@ -509,6 +559,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         }
       }
       named_sync(1, C::EPI_THREADS);
+      from_regs = have_next;
     }
   }
 
