@@ -26,7 +26,14 @@ Zipf(s=1.2) popularity over a seeded permutation of the experts); combine
 weights = softmax over the k chosen of N(0,1) logits (fp32); expert weights
 ~ N(0, 0.02), stored as FP8 E4M3 with one fp32 scale amax/448 per 128x128
 block, or as MXFP4 (E2M1 nibbles, element 2c in the low nibble, one E8M0
-scale per 32 elements along K with exponent floor(log2 amax) - 2).
+scale per 32 elements along K with exponent floor(log2 amax) - 2), or as
+NVFP4 (the same nibbles, one E4M3 scale per 16 elements along K and one fp32
+global scale per expert matrix: g = amax / (448 * 6), block scale
+e4m3(amax16 / 6 / g), element e2m1(w / (block scale * g))).
+
+The NVFP4 decode workload (not one of the table's rows) is row 2's shape
+with NVFP4 weights: ``decode_T128_H7168_E256_k8_I2048_nvfp4`` in
+``EXTRA_CONFIGS``.
 """
 from __future__ import annotations
 
@@ -38,6 +45,7 @@ import torch
 
 WFMT_FP8 = 0
 WFMT_MXFP4 = 1
+WFMT_NVFP4 = 2
 
 CONFIGS = [
     dict(name="tiny_T4_H256_E8_k2_I128_fp8", T=4, H=256, E=8, k=2, I=128,
@@ -50,6 +58,15 @@ CONFIGS = [
          wfmt=WFMT_FP8, routing="zipf1.2", n_shared=1),
     dict(name="prefill_T4096_H7168_E256_k8_I2048_fp8", T=4096, H=7168, E=256, k=8, I=2048,
          wfmt=WFMT_FP8, routing="uniform", n_shared=0),
+]
+
+
+# Workloads beyond the five above: the NVFP4 weight format on the decode shapes.
+EXTRA_CONFIGS = [
+    dict(name="decode_T128_H7168_E256_k8_I2048_nvfp4", T=128, H=7168, E=256, k=8, I=2048,
+         wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
+    dict(name="decode_T32_H7168_E256_k8_I2048_nvfp4", T=32, H=7168, E=256, k=8, I=2048,
+         wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
 ]
 
 
@@ -119,6 +136,32 @@ def _mxfp4_group(w: torch.Tensor):
     return packed.contiguous(), (e + 127).to(torch.uint8)
 
 
+def _nvfp4_matrix(w: torch.Tensor):
+    """w f32 [R, K] -> (packed uint8 [R, K/2], E4M3 block codes uint8 [R, K/16], g f32 scalar)."""
+    R, K = w.shape
+    g = w.abs().amax() / 2688.0                       # 2688 = E4M3 max 448 x E2M1 max 6
+    blk = w.reshape(R, K // 16, 16)
+    amax16 = blk.abs().amax(dim=2)
+    sc = ((amax16 / 6.0) / g).clamp(max=448.0).to(torch.float8_e4m3fn)
+    d = sc.float() * g
+    safe = torch.where(d == 0, torch.ones_like(d), d)
+    codes = _e2m1_round(blk / safe[:, :, None])
+    codes = torch.where((d == 0)[:, :, None], torch.zeros_like(codes), codes).reshape(R, K)
+    packed = codes[:, 0::2] | (codes[:, 1::2] << 4)
+    return packed.contiguous(), sc.view(torch.uint8), g.to(torch.float32)
+
+
+def make_weights_nvfp4(NE: int, rows: int, K: int, gen: torch.Generator, device, std: float = 0.02):
+    """NVFP4 expert weights: (packed [NE, rows, K/2], block codes [NE, rows, K/16], g [NE])."""
+    w = torch.empty(NE, rows, K // 2, dtype=torch.uint8, device=device)
+    s = torch.empty(NE, rows, K // 16, dtype=torch.uint8, device=device)
+    g = torch.empty(NE, dtype=torch.float32, device=device)
+    for e in range(NE):
+        dense = torch.randn(rows, K, generator=gen, device=device, dtype=torch.float32) * std
+        w[e], s[e], g[e] = _nvfp4_matrix(dense)
+    return w, s, g
+
+
 def make_weights(NE: int, rows: int, K: int, wfmt: int, gen: torch.Generator, device,
                  std: float = 0.02):
     """Expert weights [NE, rows, K] in the layer's storage format."""
@@ -153,14 +196,18 @@ class Layer:
     s13: torch.Tensor
     w2: torch.Tensor
     s2: torch.Tensor
+    g13: Optional[torch.Tensor] = None   # NVFP4: fp32 [NE] global scales of w13
+    g2: Optional[torch.Tensor] = None    # NVFP4: fp32 [NE] global scales of w2
 
     @property
     def S(self) -> int:
         return self.T * self.k
 
     def host(self) -> "Layer":
-        return dataclasses.replace(self, **{f: getattr(self, f).cpu() for f in
-                                            ("x", "ids", "topk_w", "w13", "s13", "w2", "s2")})
+        fields = ["x", "ids", "topk_w", "w13", "s13", "w2", "s2"]
+        if self.g13 is not None:
+            fields += ["g13", "g2"]
+        return dataclasses.replace(self, **{f: getattr(self, f).cpu() for f in fields})
 
 
 def make_layer(cfg: dict, seed: int, device="cpu", T: Optional[int] = None,
@@ -173,10 +220,15 @@ def make_layer(cfg: dict, seed: int, device="cpu", T: Optional[int] = None,
     gen.manual_seed(seed)
     x = make_x(T, H, gen, device)
     ids, w = make_routing(T, E, k, routing or cfg.get("routing", "uniform"), seed)
-    w13, s13 = make_weights(E + nsh, 2 * I, H, wfmt, gen, device)
-    w2, s2 = make_weights(E + nsh, H, I, wfmt, gen, device)
+    g13 = g2 = None
+    if wfmt == WFMT_NVFP4:
+        w13, s13, g13 = make_weights_nvfp4(E + nsh, 2 * I, H, gen, device)
+        w2, s2, g2 = make_weights_nvfp4(E + nsh, H, I, gen, device)
+    else:
+        w13, s13 = make_weights(E + nsh, 2 * I, H, wfmt, gen, device)
+        w2, s2 = make_weights(E + nsh, H, I, wfmt, gen, device)
     return Layer(T, H, I, E, k, wfmt, nsh, x, torch.from_numpy(ids).to(device),
-                 torch.from_numpy(w).to(device), w13, s13, w2, s2)
+                 torch.from_numpy(w).to(device), w13, s13, w2, s2, g13, g2)
 
 
 def bf16_bits(x: torch.Tensor) -> np.ndarray:

@@ -26,6 +26,7 @@ _lib = None
 
 WFMT_FP8 = 0
 WFMT_MXFP4 = 1
+WFMT_NVFP4 = 2
 
 
 def build(force: bool = False) -> str:
@@ -66,7 +67,9 @@ def lib() -> ctypes.CDLL:
             L.orc_bf16_decode.argtypes = [ctypes.c_uint16]
             L.orc_bf16_encode.restype = ctypes.c_uint16
             L.orc_bf16_encode.argtypes = [ctypes.c_float]
-            for name in ("orc_e4m3_decode_n", "orc_e4m3_encode_n", "orc_e2m1_decode_n"):
+            L.orc_e2m1_encode.restype = ctypes.c_uint8
+            L.orc_e2m1_encode.argtypes = [ctypes.c_float]
+            for name in ("orc_e4m3_decode_n", "orc_e4m3_encode_n", "orc_e2m1_decode_n", "orc_e2m1_encode_n"):
                 getattr(L, name).restype = None
                 getattr(L, name).argtypes = [vp, vp, ctypes.c_int64]
             L.orc_route.restype = ctypes.c_int
@@ -75,8 +78,14 @@ def lib() -> ctypes.CDLL:
             L.orc_quant_act.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
             L.orc_quant_row_f32.restype = None
             L.orc_quant_row_f32.argtypes = [ctypes.c_int, vp, vp, vp]
+            L.orc_quant_row_nvfp4.restype = None
+            L.orc_quant_row_nvfp4.argtypes = [ctypes.c_int, vp, vp, vp, vp]
+            L.orc_quant_act_nvfp4.restype = None
+            L.orc_quant_act_nvfp4.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
             L.orc_forward.restype = ctypes.c_int
             L.orc_forward.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 13
+            L.orc_forward_ex.restype = ctypes.c_int
+            L.orc_forward_ex.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 17
             L.orc_router.restype = ctypes.c_int
             L.orc_router.argtypes = [ctypes.c_int] * 4 + [vp] * 5
             L.orc_num_threads.restype = ctypes.c_int
@@ -118,6 +127,14 @@ def e2m1_decode(nibbles) -> np.ndarray:
     c = _c(np.asarray(nibbles, dtype=np.uint8), np.uint8)
     out = np.empty(c.shape, np.float32)
     lib().orc_e2m1_decode_n(_p(c), _p(out), c.size)
+    return out
+
+
+def e2m1_encode(values) -> np.ndarray:
+    """fp32 values -> E2M1 codes (one per byte, low nibble)."""
+    v = _c(np.asarray(values, dtype=np.float32), np.float32)
+    out = np.empty(v.shape, np.uint8)
+    lib().orc_e2m1_encode_n(_p(v), _p(out), v.size)
     return out
 
 
@@ -168,13 +185,37 @@ def quant_row_f32(v: np.ndarray):
     return q, s
 
 
+def quant_row_nvfp4(v: np.ndarray):
+    """fp32 row [K] -> (q packed uint8 [K/2], block codes uint8 [K/16], s float32 [K/128])."""
+    v = _c(v, np.float32)
+    (K,) = v.shape
+    q = np.empty(K // 2, np.uint8)
+    sc = np.empty(K // 16, np.uint8)
+    s = np.empty(K // 128, np.float32)
+    lib().orc_quant_row_nvfp4(K, _p(v), _p(q), _p(sc), _p(s))
+    return q, sc, s
+
+
+def quant_act_nvfp4(x_bf16_bits: np.ndarray):
+    """x as bf16 bits [T,H] -> (xq packed [T,H/2], xsc [T,H/16], xs [T,H/128])."""
+    x = _c(x_bf16_bits, np.uint16)
+    T, H = x.shape
+    xq = np.empty((T, H // 2), np.uint8)
+    xsc = np.empty((T, H // 16), np.uint8)
+    xs = np.empty((T, H // 128), np.float32)
+    lib().orc_quant_act_nvfp4(T, H, _p(x), _p(xq), _p(xsc), _p(xs))
+    return xq, xsc, xs
+
+
 def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
-            n_shared=0, token_mask=None, debug=False):
+            n_shared=0, token_mask=None, debug=False, g13=None, g2=None):
     """Whole layer on the CPU.
 
     Returns a dict with ``out_f32`` [T,H], ``out_bf16`` (uint16 bits) [T,H],
     ``dropped`` and, with ``debug``, ``xq``/``xs`` per token and ``hq``/``hs``
-    per routed position.  Rows of unselected tokens are NaN / 0.
+    per routed position (NVFP4: packed codes, plus ``xsc``/``hsc`` block
+    codes).  ``g13``/``g2`` are the NVFP4 per-expert global scales.  Rows of
+    unselected tokens are NaN / 0.
     """
     x = _c(x_bf16_bits, np.uint16)
     ids = _c(ids, np.int32)
@@ -192,23 +233,34 @@ def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
     if token_mask is not None:
         mask = _c(np.asarray(token_mask, dtype=np.uint8), np.uint8)
         assert mask.shape == (T,)
+    nv = wfmt == WFMT_NVFP4
+    if nv:
+        g13 = _c(np.asarray(g13, dtype=np.float32), np.float32)
+        g2 = _c(np.asarray(g2, dtype=np.float32), np.float32)
+        assert g13.shape == (E + n_shared,) and g2.shape == (E + n_shared,)
+    else:
+        g13 = g2 = None
     out_f32 = np.full((T, H), np.nan, np.float32)
     out_bf16 = np.zeros((T, H), np.uint16)
     dbg = {}
     if debug:
-        dbg = dict(xq=np.zeros((T, H), np.uint8), xs=np.zeros((T, H // 128), np.float32),
-                   hq=np.zeros((max(P, 1), I), np.uint8),
+        cw = 2 if nv else 1
+        dbg = dict(xq=np.zeros((T, H // cw), np.uint8), xs=np.zeros((T, H // 128), np.float32),
+                   hq=np.zeros((max(P, 1), I // cw), np.uint8),
                    hs=np.zeros((max(P, 1), I // 128), np.float32))
-    rc = lib().orc_forward(ctypes.byref(d), _p(x), _p(ids), _p(topk_w), _p(w13), _p(s13),
-                           _p(w2), _p(s2), _p(mask), _p(out_f32), _p(out_bf16),
-                           _p(dbg.get("xq")), _p(dbg.get("xs")), _p(dbg.get("hq")),
-                           _p(dbg.get("hs")))
+        if nv:
+            dbg.update(xsc=np.zeros((T, H // 16), np.uint8), hsc=np.zeros((max(P, 1), I // 16), np.uint8))
+    rc = lib().orc_forward_ex(ctypes.byref(d), _p(x), _p(ids), _p(topk_w), _p(w13), _p(s13), _p(g13),
+                              _p(w2), _p(s2), _p(g2), _p(mask), _p(out_f32), _p(out_bf16),
+                              _p(dbg.get("xq")), _p(dbg.get("xsc")), _p(dbg.get("xs")),
+                              _p(dbg.get("hq")), _p(dbg.get("hsc")), _p(dbg.get("hs")))
     if rc < 0:
         raise ValueError("oracle rejected the arguments")
     res = dict(out_f32=out_f32, out_bf16=out_bf16, dropped=rc)
     if debug:
-        dbg["hq"] = dbg["hq"][:P]
-        dbg["hs"] = dbg["hs"][:P]
+        for key in ("hq", "hs", "hsc"):
+            if key in dbg:
+                dbg[key] = dbg[key][:P]
         res.update(dbg)
     return res
 

@@ -77,6 +77,33 @@ float orc_e2m1_decode(uint8_t nibble) {
   return sign ? -mag : mag;
 }
 
+/* Round-to-nearest, ties to the even code (the one with mantissa bit 0),
+ * saturating at 6 (code 0x7).  The sign bit is kept, also when the magnitude
+ * rounds to zero (code 0x8 = -0), as for E4M3 above.  NaN is never produced
+ * by the layer; it maps to +6. */
+uint8_t orc_e2m1_encode(float v) {
+  uint8_t sign;
+  float a;
+  int lo;
+  if (isnan(v)) return 0x7;
+  sign = signbit(v) ? 0x8 : 0x0;
+  a = fabsf(v);
+  if (a >= 6.0f) return sign | 0x7;
+  lo = 0; /* largest code whose value is <= a (codes 0..7 increase in value) */
+  while (lo < 7 && orc_e2m1_decode((uint8_t)(lo + 1)) <= a) ++lo;
+  if (orc_e2m1_decode((uint8_t)lo) == a) return sign | (uint8_t)lo;
+  {
+    int up = lo + 1; /* <= 7 because a < 6 */
+    double d_lo = (double)a - (double)orc_e2m1_decode((uint8_t)lo);
+    double d_up = (double)orc_e2m1_decode((uint8_t)up) - (double)a;
+    int c;
+    if (d_lo < d_up) c = lo;
+    else if (d_up < d_lo) c = up;
+    else c = (lo & 1) ? up : lo;
+    return sign | (uint8_t)c;
+  }
+}
+
 float orc_e8m0_decode(uint8_t code) {
   if (code == 0xFF) return NAN;
   return ldexpf(1.0f, (int)code - 127);
@@ -105,6 +132,9 @@ void orc_e4m3_encode_n(const float* in, uint8_t* out, int64_t n) {
 }
 void orc_e2m1_decode_n(const uint8_t* in, float* out, int64_t n) {
   for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_decode(in[i]);
+}
+void orc_e2m1_encode_n(const float* in, uint8_t* out, int64_t n) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_e2m1_encode(in[i]);
 }
 
 int orc_num_threads(void) {
@@ -191,6 +221,66 @@ void orc_quant_act(int T, int H, const uint16_t* x, uint8_t* xq, float* xs) {
   free(row);
 }
 
+/* NVFP4 (NVIDIA's definition; the onnxruntime QMoE page lists the layout and
+ * a global scale but no rule) with the second-level scale taken per 128
+ * columns, the layer's activation group.  Readings: S = amax128 / 2688 in
+ * fp32 (2688 = E4M3 max 448 x E2M1 max 6, so the largest block scale code
+ * is ~448), S = 1 for an all-zero group; block code c = e4m3((amax16 / 6) /
+ * S) with two fp32 divisions; element code q = e2m1(v / d) with d =
+ * e4m3_value(c) * S; a block whose code underflows to 0 stores q = 0. */
+void orc_quant_row_nvfp4(int K, const float* v, uint8_t* q, uint8_t* sc, float* s) {
+  for (int c = 0; c < K / 2; ++c) q[c] = 0;
+  for (int g = 0; g < K / 128; ++g) {
+    const float* vg = v + (size_t)g * 128;
+    float amax = 0.0f;
+    float S;
+    for (int c = 0; c < 128; ++c) {
+      float a = fabsf(vg[c]);
+      if (a > amax) amax = a;
+    }
+    S = amax / 2688.0f;
+    if (amax == 0.0f) S = 1.0f;
+    s[g] = S;
+    for (int b = 0; b < 8; ++b) {
+      const float* vb = vg + b * 16;
+      float amax16 = 0.0f;
+      uint8_t code;
+      float d;
+      for (int c = 0; c < 16; ++c) {
+        float a = fabsf(vb[c]);
+        if (a > amax16) amax16 = a;
+      }
+      code = orc_e4m3_encode((amax16 / 6.0f) / S);
+      sc[g * 8 + b] = code;
+      d = orc_e4m3_decode(code) * S;
+      for (int c = 0; c < 16; ++c) {
+        const int col = g * 128 + b * 16 + c;
+        uint8_t nib = (code == 0) ? 0 : orc_e2m1_encode(vb[c] / d);
+        q[col / 2] |= (uint8_t)((col % 2 == 0) ? nib : (nib << 4));
+      }
+    }
+  }
+}
+
+void orc_quant_act_nvfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc, float* xs) {
+  float* row = (float*)malloc(sizeof(float) * (size_t)H);
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < H; ++c) row[c] = orc_bf16_decode(x[(size_t)t * H + c]);
+    orc_quant_row_nvfp4(H, row, xq + (size_t)t * (H / 2), xsc + (size_t)t * (H / 16), xs + (size_t)t * (H / 128));
+  }
+  free(row);
+}
+
+/* One NVFP4 row (packed E2M1 + E4M3 block codes) -> element x block scale
+ * values (exact in fp32: 2 x 4 significant bits); the second-level scale is
+ * applied per K block by the caller. */
+static void decode_nvfp4_row(const uint8_t* q, const uint8_t* sc, int K, float* out) {
+  for (int c = 0; c < K; ++c) {
+    uint8_t nib = (c % 2 == 0) ? (q[c / 2] & 0xF) : (q[c / 2] >> 4);
+    out[c] = orc_e2m1_decode(nib) * orc_e4m3_decode(sc[c / 16]);
+  }
+}
+
 /* ----------------------------------------------------------------------- */
 /* One weight row, decoded to fp32 without its FP8 block scale (FP8 path) or
  * with its E8M0 per-32 scale folded in (MXFP4 path: OCP MX element value =
@@ -199,6 +289,8 @@ static void decode_row(int wfmt, const uint8_t* wrow, const uint8_t* srow_e8m0, 
                        const float* e4m3_tab, float* out) {
   if (wfmt == ORC_WFMT_FP8) {
     for (int c = 0; c < K; ++c) out[c] = e4m3_tab[wrow[c]];
+  } else if (wfmt == ORC_WFMT_NVFP4) {
+    decode_nvfp4_row(wrow, srow_e8m0 /* E4M3 block codes here */, K, out);
   } else {
     for (int c = 0; c < K; ++c) {
       uint8_t byte = wrow[c / 2];
@@ -213,7 +305,9 @@ static void decode_row(int wfmt, const uint8_t* wrow, const uint8_t* srow_e8m0, 
  * per-token scale.  With 128-wide K blocks carrying their own scales, each
  * block's partial sum is scaled and added in ascending block order.
  *   FP8:   acc = sum_kb ( sum_{c in kb} a[c] * w[c] ) * (as[kb] * ws[kb])
- *   MXFP4: acc = sum_kb ( sum_{c in kb} a[c] * w[c] ) * as[kb]  (w carries its E8M0 scale) */
+ *   MXFP4: acc = sum_kb ( sum_{c in kb} a[c] * w[c] ) * as[kb]  (w carries its E8M0 scale)
+ *   NVFP4: as FP8 with ws[kb] = the expert's global scale, a and w carrying
+ *          their E4M3 block scales */
 static float row_dot(int K, const float* a, const float* as, const float* w,
                      const float* ws /* NULL for MXFP4 */) {
   float acc = 0.0f;
@@ -233,29 +327,35 @@ static float swiglu(float g, float u) {
   return g * sig * u;
 }
 
-int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
-                const float* topk_w, const void* w13v, const void* s13v,
-                const void* w2v, const void* s2v, const uint8_t* token_mask,
-                float* out_f32, uint16_t* out_bf16,
-                uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs) {
+int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
+                   const float* topk_w, const void* w13v, const void* s13v, const float* g13,
+                   const void* w2v, const void* s2v, const float* g2, const uint8_t* token_mask,
+                   float* out_f32, uint16_t* out_bf16,
+                   uint8_t* dbg_xq, uint8_t* dbg_xsc, float* dbg_xs,
+                   uint8_t* dbg_hq, uint8_t* dbg_hsc, float* dbg_hs) {
   const int T = d->T, H = d->H, I = d->I, E = d->E, k = d->k;
   const int wfmt = d->wfmt, nsh = d->n_shared;
   const int S = T * k, NG = E + nsh, P = S + nsh * T;
   const int HB = H / 128, IB = I / 128;
+  const int nv = (wfmt == ORC_WFMT_NVFP4);
   const uint8_t* w13 = (const uint8_t*)w13v;
   const uint8_t* w2 = (const uint8_t*)w2v;
-  /* per-expert strides in bytes (weights) and elements (scales) */
+  /* per-expert strides in bytes (weights) */
   const size_t w13_e = (wfmt == ORC_WFMT_FP8) ? (size_t)2 * I * H : (size_t)2 * I * H / 2;
   const size_t w2_e = (wfmt == ORC_WFMT_FP8) ? (size_t)H * I : (size_t)H * I / 2;
   const size_t w13_r = (wfmt == ORC_WFMT_FP8) ? (size_t)H : (size_t)H / 2;
   const size_t w2_r = (wfmt == ORC_WFMT_FP8) ? (size_t)I : (size_t)I / 2;
+  /* activation codes per row: E4M3 bytes, or packed E2M1 + E4M3 block codes */
+  const size_t xq_r = nv ? (size_t)H / 2 : (size_t)H;
+  const size_t hq_r = nv ? (size_t)I / 2 : (size_t)I;
   int32_t *counts, *offsets, *perm, *inv, *cidx;
-  uint8_t* xq;
+  uint8_t *xq, *xsc = NULL;
   float *xs, *xd, *Y, e4m3_tab[256];
   int dropped, ncomp = 0;
 
   if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || H % 128 || I % 128 ||
-      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4) || nsh < 0 || nsh > 1)
+      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4 && wfmt != ORC_WFMT_NVFP4) || nsh < 0 || nsh > 1 ||
+      (nv && (!g13 || !g2)))
     return -1;
   if (T == 0) return 0;
   for (int c = 0; c < 256; ++c) e4m3_tab[c] = orc_e4m3_decode((uint8_t)c);
@@ -267,13 +367,22 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   cidx = (int32_t*)malloc(sizeof(int32_t) * (size_t)P);
   dropped = orc_route(T, k, E, nsh, ids, counts, offsets, perm, inv);
 
-  /* step 2 for every token (cheap), then code values without their scale */
-  xq = (uint8_t*)malloc((size_t)T * H);
+  /* step 2 for every token (cheap), then code values without their
+   * per-128 scale (NVFP4: element x E4M3 block scale) */
+  xq = (uint8_t*)malloc((size_t)T * xq_r);
   xs = (float*)malloc(sizeof(float) * (size_t)T * HB);
   xd = (float*)malloc(sizeof(float) * (size_t)T * H);
-  orc_quant_act(T, H, x, xq, xs);
-  for (size_t i = 0; i < (size_t)T * H; ++i) xd[i] = e4m3_tab[xq[i]];
-  if (dbg_xq) memcpy(dbg_xq, xq, (size_t)T * H);
+  if (nv) {
+    xsc = (uint8_t*)malloc((size_t)T * (H / 16));
+    orc_quant_act_nvfp4(T, H, x, xq, xsc, xs);
+    for (int t = 0; t < T; ++t)
+      decode_nvfp4_row(xq + (size_t)t * xq_r, xsc + (size_t)t * (H / 16), H, xd + (size_t)t * H);
+    if (dbg_xsc) memcpy(dbg_xsc, xsc, (size_t)T * (H / 16));
+  } else {
+    orc_quant_act(T, H, x, xq, xs);
+    for (size_t i = 0; i < (size_t)T * H; ++i) xd[i] = e4m3_tab[xq[i]];
+  }
+  if (dbg_xq) memcpy(dbg_xq, xq, (size_t)T * xq_r);
   if (dbg_xs) memcpy(dbg_xs, xs, sizeof(float) * (size_t)T * HB);
 
   /* compact index of the positions whose token is selected */
@@ -291,7 +400,7 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     int n = 0;
     int *pos, *tok;
     float *G, *hd, *hs;
-    uint8_t* hq;
+    uint8_t *hq, *hsc;
     for (int p = p0; p < p1; ++p) n += (cidx[p] >= 0);
     if (n == 0) continue;
     pos = (int*)malloc(sizeof(int) * (size_t)n);
@@ -306,7 +415,8 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     G = (float*)malloc(sizeof(float) * (size_t)n * 2 * I);
     hd = (float*)malloc(sizeof(float) * (size_t)n * I);
     hs = (float*)malloc(sizeof(float) * (size_t)n * IB);
-    hq = (uint8_t*)malloc((size_t)n * I);
+    hq = (uint8_t*)malloc((size_t)n * hq_r);
+    hsc = (uint8_t*)malloc((size_t)n * (I / 16));
 
     /* step 3: GEMM1, G[i][r] for gate rows r < I and up rows r >= I */
 #pragma omp parallel
@@ -321,13 +431,16 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
           const float* s13 = (const float*)s13v;
           for (int kb = 0; kb < HB; ++kb)
             ws[kb] = s13[((size_t)g * (2 * I / 128) + (size_t)(r / 128)) * HB + kb];
+        } else if (nv) {
+          sr = (const uint8_t*)s13v + ((size_t)g * 2 * I + (size_t)r) * (H / 16);
+          for (int kb = 0; kb < HB; ++kb) ws[kb] = g13[g];
         } else {
           sr = (const uint8_t*)s13v + ((size_t)g * 2 * I + (size_t)r) * (H / 32);
         }
         decode_row(wfmt, wr, sr, H, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           G[(size_t)i * 2 * I + r] = row_dot(H, xd + (size_t)tok[i] * H, xs + (size_t)tok[i] * HB,
-                                             wrow, wfmt == ORC_WFMT_FP8 ? ws : NULL);
+                                             wrow, wfmt == ORC_WFMT_MXFP4 ? NULL : ws);
       }
       free(wrow);
       free(ws);
@@ -337,11 +450,18 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     {
       float* h = (float*)malloc(sizeof(float) * (size_t)I);
       for (int i = 0; i < n; ++i) {
+        uint8_t* hqi = hq + (size_t)i * hq_r;
         for (int c = 0; c < I; ++c)
           h[c] = swiglu(G[(size_t)i * 2 * I + c], G[(size_t)i * 2 * I + I + c]);
-        orc_quant_row_f32(I, h, hq + (size_t)i * I, hs + (size_t)i * IB);
-        for (int c = 0; c < I; ++c) hd[(size_t)i * I + c] = e4m3_tab[hq[(size_t)i * I + c]];
-        if (dbg_hq) memcpy(dbg_hq + (size_t)pos[i] * I, hq + (size_t)i * I, (size_t)I);
+        if (nv) {
+          orc_quant_row_nvfp4(I, h, hqi, hsc + (size_t)i * (I / 16), hs + (size_t)i * IB);
+          decode_nvfp4_row(hqi, hsc + (size_t)i * (I / 16), I, hd + (size_t)i * I);
+          if (dbg_hsc) memcpy(dbg_hsc + (size_t)pos[i] * (I / 16), hsc + (size_t)i * (I / 16), (size_t)(I / 16));
+        } else {
+          orc_quant_row_f32(I, h, hqi, hs + (size_t)i * IB);
+          for (int c = 0; c < I; ++c) hd[(size_t)i * I + c] = e4m3_tab[hqi[c]];
+        }
+        if (dbg_hq) memcpy(dbg_hq + (size_t)pos[i] * hq_r, hqi, hq_r);
         if (dbg_hs) memcpy(dbg_hs + (size_t)pos[i] * IB, hs + (size_t)i * IB, sizeof(float) * IB);
       }
       free(h);
@@ -360,18 +480,21 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
           const float* s2 = (const float*)s2v;
           for (int kb = 0; kb < IB; ++kb)
             ws[kb] = s2[((size_t)g * (H / 128) + (size_t)(r / 128)) * IB + kb];
+        } else if (nv) {
+          sr = (const uint8_t*)s2v + ((size_t)g * H + (size_t)r) * (I / 16);
+          for (int kb = 0; kb < IB; ++kb) ws[kb] = g2[g];
         } else {
           sr = (const uint8_t*)s2v + ((size_t)g * H + (size_t)r) * (I / 32);
         }
         decode_row(wfmt, wr, sr, I, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           Y[(size_t)cidx[pos[i]] * H + r] = row_dot(I, hd + (size_t)i * I, hs + (size_t)i * IB,
-                                                    wrow, wfmt == ORC_WFMT_FP8 ? ws : NULL);
+                                                    wrow, wfmt == ORC_WFMT_MXFP4 ? NULL : ws);
       }
       free(wrow);
       free(ws);
     }
-    free(pos); free(tok); free(G); free(hd); free(hs); free(hq);
+    free(pos); free(tok); free(G); free(hd); free(hs); free(hq); free(hsc);
   }
 
   /* step 7: top-k weighted combine (FusedDeepMoE ReducePermute: accumulate the
@@ -393,8 +516,18 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   }
 
   free(counts); free(offsets); free(perm); free(inv); free(cidx);
-  free(xq); free(xs); free(xd); free(Y);
+  free(xq); free(xsc); free(xs); free(xd); free(Y);
   return dropped;
+}
+
+int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
+                const float* topk_w, const void* w13, const void* s13,
+                const void* w2, const void* s2, const uint8_t* token_mask,
+                float* out_f32, uint16_t* out_bf16,
+                uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs) {
+  if (d && d->wfmt == ORC_WFMT_NVFP4) return -1; /* needs the global scales: orc_forward_ex */
+  return orc_forward_ex(d, x, ids, topk_w, w13, s13, NULL, w2, s2, NULL, token_mask, out_f32, out_bf16,
+                        dbg_xq, NULL, dbg_xs, dbg_hq, NULL, dbg_hs);
 }
 
 /* ----------------------------------------------------------------------- */

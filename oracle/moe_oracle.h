@@ -22,6 +22,12 @@
  *    floating point spec (E4M3, "e4m3fn": bias 7, no infinities, S.1111.111 is
  *    NaN, max 448) and OCP Microscaling (MX) v1.0 (E2M1 elements, E8M0 shared
  *    scale per 32 elements, 0xFF = NaN).
+ *  - NVFP4, named among the 4-bit expert layouts of the onnxruntime QMoE
+ *    offload PR page (with a per-tensor global scale folded into its FP4
+ *    lookup table) but not defined there; the definition taken is NVIDIA's
+ *    public one: E2M1 elements, one E4M3 scale per 16 consecutive elements,
+ *    and an fp32 second-level scale.  See orc_quant_row_nvfp4 for the
+ *    encoding rule and orc_forward_ex for where each scale applies.
  *
  * Precision: fp32 arithmetic throughout (the layer's own accumulate and
  * scale precision), partial sums of one 128-wide K block in ascending k,
@@ -30,7 +36,10 @@
  * Parity pins live in tests/test_oracle_pins.py (codec tables against torch's
  * float8 dtype and the OCP tables, routing against numpy's stable argsort,
  * the one-expert/dense-FFN reduction, fp64 brute force on tiny shapes,
- * linearity in the combine weights, zero input).
+ * linearity in the combine weights, zero input) and, for NVFP4, in
+ * tests/test_oracle_nvfp4.py (E2M1 rounding against the OCP table by brute
+ * force, exact round trips of representable groups, error bounds, the fp64
+ * restatement of the layer).
  */
 #ifndef MOE_ORACLE_H
 #define MOE_ORACLE_H
@@ -41,12 +50,13 @@
 extern "C" {
 #endif
 
-enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1 };
+enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1, ORC_WFMT_NVFP4 = 2 };
 
 /* ---- codecs (OCP FP8 / OCP MX v1.0) ---------------------------------- */
 float   orc_e4m3_decode(uint8_t code);          /* exact value, NaN for S.1111.111 */
 uint8_t orc_e4m3_encode(float v);               /* round-to-nearest-even, saturate to +-448 */
 float   orc_e2m1_decode(uint8_t nibble);        /* low 4 bits used */
+uint8_t orc_e2m1_encode(float v);               /* round-to-nearest-even, saturate to +-6, sign kept */
 float   orc_e8m0_decode(uint8_t code);          /* 2^(code-127), NaN for 0xFF */
 float   orc_bf16_decode(uint16_t bits);
 uint16_t orc_bf16_encode(float v);              /* round-to-nearest-even */
@@ -55,6 +65,7 @@ uint16_t orc_bf16_encode(float v);              /* round-to-nearest-even */
 void orc_e4m3_decode_n(const uint8_t* in, float* out, int64_t n);
 void orc_e4m3_encode_n(const float* in, uint8_t* out, int64_t n);
 void orc_e2m1_decode_n(const uint8_t* in, float* out, int64_t n);
+void orc_e2m1_encode_n(const float* in, uint8_t* out, int64_t n);
 
 /* ---- step 1: routing (counting sort of slots by expert) -------------- */
 /* ids [T*k] expert ids, slot s = t*k + j.  With n_shared == 1 the shared
@@ -74,10 +85,20 @@ void orc_quant_act(int T, int H, const uint16_t* x, uint8_t* xq, float* xs);
 /* Same rule on an fp32 row (used for the SwiGLU output requantisation). */
 void orc_quant_row_f32(int K, const float* v, uint8_t* q, float* s);
 
+/* NVFP4 form of steps 2 and 5 (activations meet NVFP4 weights as FP4 x FP4).
+ * One fp32 row of K (multiple of 128) values -> q packed E2M1 [K/2] (element
+ * 2c in the low nibble of byte c), sc E4M3 block codes [K/16], s fp32 [K/128]:
+ *   per 128-group:  S = amax128 / 2688  (2688 = 448 * 6; S = 1 if all zero)
+ *   per 16-block:   c = e4m3(amax16 / 6 / S),  d = e4m3_value(c) * S
+ *   per element:    q = e2m1(v / d)  (q = 0 when c == 0)
+ * so that v ~ e2m1_value(q) * e4m3_value(c) * S. */
+void orc_quant_row_nvfp4(int K, const float* v, uint8_t* q, uint8_t* sc, float* s);
+void orc_quant_act_nvfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc, float* xs);
+
 /* ---- steps 1-8: the whole layer -------------------------------------- */
 typedef struct {
   int T, H, I, E, k;
-  int wfmt;       /* ORC_WFMT_FP8 or ORC_WFMT_MXFP4 */
+  int wfmt;       /* ORC_WFMT_FP8, ORC_WFMT_MXFP4 or ORC_WFMT_NVFP4 */
   int n_shared;   /* 0 or 1: shared expert stored as expert index E */
 } orc_dims;
 
@@ -98,6 +119,22 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
                 const void* w2, const void* s2, const uint8_t* token_mask,
                 float* out_f32, uint16_t* out_bf16,
                 uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs);
+
+/* All three formats.  For ORC_WFMT_NVFP4 (g13, g2 required; ignored otherwise):
+ *   w13 u8 [NE, 2I, H/2] packed E2M1, s13 u8 E4M3 [NE, 2I, H/16], g13 f32 [NE]
+ *   w2  u8 [NE, H, I/2],              s2  u8 E4M3 [NE, H, I/16],  g2  f32 [NE]
+ * weight value = e2m1(q) * e4m3(s) * g[expert].  Activations are quantised
+ * with orc_quant_row_nvfp4; each 128-wide K block's partial sum of
+ * (element x block scale) products is scaled by S_act[kb] * g[expert] and
+ * added in ascending block order.  NVFP4 debug outputs: xq [T, H/2],
+ * xsc [T, H/16], xs [T, H/128]; hq [P, I/2], hsc [P, I/16], hs [P, I/128]
+ * (dbg_xsc / dbg_hsc are unused for the other formats). */
+int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
+                   const float* topk_w, const void* w13, const void* s13, const float* g13,
+                   const void* w2, const void* s2, const float* g2, const uint8_t* token_mask,
+                   float* out_f32, uint16_t* out_bf16,
+                   uint8_t* dbg_xq, uint8_t* dbg_xsc, float* dbg_xs,
+                   uint8_t* dbg_hq, uint8_t* dbg_hsc, float* dbg_hs);
 
 /* ---- fused router (a "Mega Gate": routing GEMM + top-k in one step) ----
  * DeepGEMM 26/09 news page: the router GEMM and the MoE routing ops fused

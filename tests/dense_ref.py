@@ -2,8 +2,9 @@
 
 Used only by tests on tiny shapes.  It shares no code with the oracle: the
 FP8 encode/decode steps go through torch's ``float8_e4m3fn`` dtype, E2M1
-decoding through the OCP MX table in ``tests/golden``, matrix products through
-numpy ``einsum`` in float64, and tokens are processed densely per expert.
+decoding through the OCP MX table in ``tests/golden`` (and E2M1 encoding by
+brute-force nearest search over that table), matrix products through numpy
+``einsum`` in float64, and tokens are processed densely per expert.
 """
 from __future__ import annotations
 
@@ -49,23 +50,63 @@ def quant128(v: np.ndarray):
     return q.to(torch.float64).reshape(t.shape).numpy(), s.numpy()
 
 
+def e2m1_nearest(v: np.ndarray) -> np.ndarray:
+    """E2M1 codes by brute force over the OCP table: the nearest value, ties to
+    the code with mantissa bit 0, magnitudes beyond 6 to 6, sign bit kept."""
+    vals = _E2M1_ARR[:8]
+    a = np.minimum(np.abs(np.asarray(v, dtype=np.float64)), 6.0)
+    dist = np.abs(a[..., None] - vals)
+    cand = dist == dist.min(axis=-1, keepdims=True)
+    even = cand & (np.arange(8) % 2 == 0)
+    code = np.where(even.any(axis=-1), even.argmax(axis=-1), cand.argmax(axis=-1)).astype(np.uint8)
+    return np.where(np.signbit(v), code | 8, code).astype(np.uint8)
+
+
+def unpack_e2m1(w: np.ndarray, K: int) -> np.ndarray:
+    codes = np.empty(w.shape[:-1] + (K,), dtype=np.uint8)
+    codes[..., 0::2] = w & 0xF
+    codes[..., 1::2] = w >> 4
+    return codes
+
+
+def quant_nvfp4(v: np.ndarray):
+    """fp32 rows [..., K] -> (element x block-scale values float64 [..., K],
+    per-128 scales float32 [..., K/128], E2M1 codes [..., K], E4M3 block codes
+    [..., K/16]).  S = amax128/2688 (1 if zero), block code from torch's RNE
+    cast of amax16/6/S, element codes by brute-force nearest of v/d."""
+    t = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32))
+    K = t.shape[-1]
+    g = t.reshape(*t.shape[:-1], K // 128, 128)
+    amax = g.abs().amax(dim=-1)
+    S = torch.where(amax == 0, torch.ones_like(amax), amax / 2688.0)
+    b = t.reshape(*t.shape[:-1], K // 16, 16)
+    S16 = S.repeat_interleave(8, dim=-1)
+    c = ((b.abs().amax(dim=-1) / 6.0) / S16).to(torch.float8_e4m3fn)
+    d = c.float() * S16
+    ratio = (b / torch.where(d == 0, torch.ones_like(d), d)[..., None]).numpy()
+    q = e2m1_nearest(ratio)
+    q = np.where((d == 0).numpy()[..., None], 0, q).astype(np.uint8)
+    vals = _E2M1_ARR[q] * c.to(torch.float64).numpy()[..., None]
+    shape = t.shape
+    return vals.reshape(shape), S.numpy(), q.reshape(shape), c.view(torch.uint8).numpy()
+
+
 def dequant_weights(w: np.ndarray, s: np.ndarray, wfmt: int, K: int) -> np.ndarray:
     """One expert's weights [R, K] as float64 code values, with the MXFP4 E8M0
-    scale folded in.  FP8 block scales are applied separately per K block."""
+    scale (NVFP4: the E4M3 block scale) folded in.  FP8 block scales and the
+    NVFP4 global scale are applied separately."""
     if wfmt == 0:
         return e4m3_values(w)
-    lo = w & 0xF
-    hi = w >> 4
-    codes = np.empty((w.shape[0], K), dtype=np.uint8)
-    codes[:, 0::2] = lo
-    codes[:, 1::2] = hi
-    vals = _E2M1_ARR[codes]
+    vals = _E2M1_ARR[unpack_e2m1(w, K)]
+    if wfmt == 2:
+        return vals * np.repeat(e4m3_values(s), 16, axis=1)
     scale = np.exp2(s.astype(np.float64) - 127.0)
     return vals * np.repeat(scale, 32, axis=1)
 
 
-def grouped_gemm(ad: np.ndarray, as_: np.ndarray, wd: np.ndarray, ws, wfmt: int) -> np.ndarray:
-    """ad [n,K] code values, as_ [n,K/128]; wd [R,K]; ws [R/128,K/128] (FP8) -> [n,R] fp64."""
+def grouped_gemm(ad: np.ndarray, as_: np.ndarray, wd: np.ndarray, ws, wfmt: int, wg=None) -> np.ndarray:
+    """ad [n,K] code values, as_ [n,K/128]; wd [R,K]; ws [R/128,K/128] (FP8);
+    wg the NVFP4 global scale -> [n,R] fp64."""
     n, K = ad.shape
     R = wd.shape[0]
     KB = K // 128
@@ -73,33 +114,44 @@ def grouped_gemm(ad: np.ndarray, as_: np.ndarray, wd: np.ndarray, ws, wfmt: int)
     part = part * as_.astype(np.float64)[:, None, :]
     if wfmt == 0:
         part = part * np.repeat(ws.astype(np.float64), 128, axis=0)[None, :, :]
+    if wfmt == 2:
+        part = part * float(wg)
     return part.sum(axis=2)
 
 
-def expert_ffn(xd, xs, w13, s13, w2, s2, wfmt, H, I):
+def expert_ffn(xd, xs, w13, s13, w2, s2, wfmt, H, I, g13=None, g2=None):
     """Tokens of one expert: quantised activations -> fp64 expert output [n,H]."""
-    G = grouped_gemm(xd, xs, dequant_weights(w13, s13, wfmt, H), s13, wfmt)
+    G = grouped_gemm(xd, xs, dequant_weights(w13, s13, wfmt, H), s13, wfmt, g13)
     g, u = G[:, :I], G[:, I:]
     h = g / (1.0 + np.exp(-g)) * u
-    hd, hs = quant128(h.astype(np.float32))
-    return grouped_gemm(hd, hs, dequant_weights(w2, s2, wfmt, I), s2, wfmt)
+    if wfmt == 2:
+        hd, hs = quant_nvfp4(h.astype(np.float32))[:2]
+    else:
+        hd, hs = quant128(h.astype(np.float32))
+    return grouped_gemm(hd, hs, dequant_weights(w2, s2, wfmt, I), s2, wfmt, g2)
 
 
-def moe_layer(x_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt, n_shared=0):
+def moe_layer(x_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt, n_shared=0, g13=None, g2=None):
     """Whole layer, token by token and slot by slot, in fp64."""
     x = (x_bits.astype(np.uint32) << 16).view(np.float32)
-    xd, xs = quant128(x)
+    xd, xs = quant_nvfp4(x)[:2] if wfmt == 2 else quant128(x)
     T, k = ids.shape
     out = np.zeros((T, H), dtype=np.float64)
+
+    def gs(g, e):
+        return None if g is None else g[e]
+
     for t in range(T):
         for j in range(k):
             e = int(ids[t, j])
             if not 0 <= e < E:
                 continue
-            y = expert_ffn(xd[t:t + 1], xs[t:t + 1], w13[e], s13[e], w2[e], s2[e], wfmt, H, I)
+            y = expert_ffn(xd[t:t + 1], xs[t:t + 1], w13[e], s13[e], w2[e], s2[e], wfmt, H, I,
+                           gs(g13, e), gs(g2, e))
             out[t] += float(topk_w[t, j]) * y[0]
         if n_shared:
-            y = expert_ffn(xd[t:t + 1], xs[t:t + 1], w13[E], s13[E], w2[E], s2[E], wfmt, H, I)
+            y = expert_ffn(xd[t:t + 1], xs[t:t + 1], w13[E], s13[E], w2[E], s2[E], wfmt, H, I,
+                           gs(g13, E), gs(g2, E))
             out[t] += y[0]
     return out
 

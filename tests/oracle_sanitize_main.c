@@ -2,7 +2,7 @@
  * (built by tests/test_oracle_sanitizers.py with -fsanitize=address,undefined
  * -fno-sanitize-recover=all, single-threaded).  Every entry point runs on
  * small seeded inputs that include ragged shapes, the shared expert, dropped
- * ids, both weight formats and the router; any out-of-bounds access, leak or
+ * ids, all three weight formats and the router; any out-of-bounds access, leak or
  * undefined operation aborts with a non-zero exit status. */
 #include <math.h>
 #include <stdint.h>
@@ -46,6 +46,11 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
     s13_bytes = sizeof(float) * NE * (2 * I / 128) * (H / 128);
     w2_bytes = (size_t)NE * H * I;
     s2_bytes = sizeof(float) * NE * (H / 128) * (I / 128);
+  } else if (wfmt == ORC_WFMT_NVFP4) {
+    w13_bytes = (size_t)NE * 2 * I * H / 2;
+    s13_bytes = (size_t)NE * 2 * I * (H / 16);
+    w2_bytes = (size_t)NE * H * I / 2;
+    s2_bytes = (size_t)NE * H * (I / 16);
   } else {
     w13_bytes = (size_t)NE * 2 * I * H / 2;
     s13_bytes = (size_t)NE * 2 * I * (H / 32);
@@ -63,19 +68,32 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
     float* f2 = (float*)s2;
     for (size_t i = 0; i < s13_bytes / sizeof(float); ++i) f13[i] = 0.001f + 0.01f * (unit() + 0.5f);
     for (size_t i = 0; i < s2_bytes / sizeof(float); ++i) f2[i] = 0.001f + 0.01f * (unit() + 0.5f);
+  } else if (wfmt == ORC_WFMT_NVFP4) {
+    for (size_t i = 0; i < s13_bytes; ++i) s13[i] = (uint8_t)(0x30 + rnd() % 0x40); /* E4M3 0.25 .. 240 */
+    for (size_t i = 0; i < s2_bytes; ++i) s2[i] = (uint8_t)(0x30 + rnd() % 0x40);
   } else {
     for (size_t i = 0; i < s13_bytes; ++i) s13[i] = (uint8_t)(118 + rnd() % 8);
     for (size_t i = 0; i < s2_bytes; ++i) s2[i] = (uint8_t)(118 + rnd() % 8);
+  }
+  float* g13 = malloc(sizeof(float) * NE);
+  float* g2 = malloc(sizeof(float) * NE);
+  for (int e = 0; e < NE; ++e) {
+    g13[e] = 1e-4f * (1.0f + unit());
+    g2[e] = 1e-4f * (1.0f + unit());
   }
   const size_t P = S + (size_t)n_shared * T;
   float* out = malloc(sizeof(float) * T * H);
   uint16_t* outb = malloc(sizeof(uint16_t) * T * H);
   uint8_t* xq = malloc((size_t)T * H);
+  uint8_t* xsc = malloc((size_t)T * (H / 16));
   float* xs = malloc(sizeof(float) * T * (H / 128));
   uint8_t* hq = malloc(P * I + 1);
+  uint8_t* hsc = malloc(P * (I / 16) + 1);
   float* hs = malloc(sizeof(float) * (P * (I / 128) + 1));
   orc_dims d = {T, H, I, E, k, wfmt, n_shared};
-  const int dropped = orc_forward(&d, x, ids, w, w13, s13, w2, s2, NULL, out, outb, xq, xs, hq, hs);
+  const int dropped = (wfmt == ORC_WFMT_NVFP4)
+      ? orc_forward_ex(&d, x, ids, w, w13, s13, g13, w2, s2, g2, NULL, out, outb, xq, xsc, xs, hq, hsc, hs)
+      : orc_forward(&d, x, ids, w, w13, s13, w2, s2, NULL, out, outb, xq, xs, hq, hs);
   int ok = dropped == (bad_ids && S > 2 ? 2 : 0) && check_finite(out, (size_t)T * H);
   int32_t* counts = malloc(sizeof(int32_t) * (NE + 1));
   int32_t* offsets = malloc(sizeof(int32_t) * (NE + 2));
@@ -84,6 +102,7 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
   ok = ok && orc_route(T, k, E, n_shared, ids, counts, offsets, perm, inv) == dropped;
   free(x); free(ids); free(w); free(w13); free(w2); free(s13); free(s2); free(out); free(outb);
   free(xq); free(xs); free(hq); free(hs); free(counts); free(offsets); free(perm); free(inv);
+  free(g13); free(g2); free(xsc); free(hsc);
   return ok;
 }
 
@@ -107,6 +126,8 @@ int main(void) {
   ok &= run_layer(7, 384, 256, 5, 3, ORC_WFMT_FP8, 1, 1);
   ok &= run_layer(3, 256, 128, 4, 2, ORC_WFMT_MXFP4, 1, 0);
   ok &= run_layer(1, 128, 128, 1, 1, ORC_WFMT_MXFP4, 0, 0);
+  ok &= run_layer(5, 256, 128, 6, 2, ORC_WFMT_NVFP4, 1, 1);
+  ok &= run_layer(2, 384, 256, 3, 3, ORC_WFMT_NVFP4, 0, 0);
   ok &= run_router(9, 256, 16, 4);
   ok &= run_router(2, 128, 8, 8);
   uint8_t codes[256];
@@ -116,6 +137,12 @@ int main(void) {
   uint8_t back[256];
   for (int i = 0; i < 256; ++i) vals[i] = isfinite(vals[i]) ? vals[i] : 0.0f;
   orc_e4m3_encode_n(vals, back, 256);
+  {
+    float v16[16];
+    uint8_t c16[16];
+    for (int i = 0; i < 16; ++i) v16[i] = 8.0f * unit();
+    orc_e2m1_encode_n(v16, c16, 16);
+  }
   printf(ok ? "sanitized oracle run ok\n" : "sanitized oracle run FAILED\n");
   return ok ? 0 : 1;
 }
