@@ -25,6 +25,11 @@ struct moe_ctx {
   int4* tiles;
   uint8_t *xq, *hq;
   float *xs, *hs, *out_acc;
+  // NVFP4: E4M3 block codes of the activations, [K/64][S_pad][16] bytes
+  // (per 64-column MMA step and position: four codes, then zeros), and their
+  // TMA maps (boxes of 16 bytes x 32 rows = one block-scale atom)
+  uint8_t *xsc, *hsc;
+  CUtensorMap tm_xsc, tm_hsc;
   // tensor-map cache
   const void* c_w13;
   const void* c_w2;
@@ -116,9 +121,10 @@ const GreenFns& green_fns() {
 }
 
 // 2-D map over a row-major matrix [rows, inner] (inner contiguous), box
-// {box_inner elements, box_rows}, 128-byte swizzle.
+// {box_inner elements, box_rows}, 128-byte swizzle unless given.
 bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
-              uint64_t row_bytes, uint32_t box_rows, CUtensorMapL2promotion l2, uint32_t box_inner = 128) {
+              uint64_t row_bytes, uint32_t box_rows, CUtensorMapL2promotion l2, uint32_t box_inner = 128,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   EncodeTiledFn fn = encode_fn();
   if (!fn) return false;
   cuuint64_t gdim[2] = {inner, rows};
@@ -126,7 +132,7 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
   cuuint32_t box[2] = {box_inner, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), gdim, gstride, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swz, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -139,6 +145,7 @@ int pick_tile_n(const moe_ctx* c, int T) {
   int bn = avg <= 8 ? 16 : avg <= 20 ? 32 : avg <= 48 ? 64 : 128;
   if (c->tile_n_override) bn = c->tile_n_override;
   if (c->wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 && bn > 64) bn = 64;
+  if (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 && bn > 32) bn = 32;  // token scale atom: 32 tokens
   return bn;
 }
 
@@ -169,7 +176,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || max_T <= 0 || n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128 || H > 8192 || I > 8192 || E > 1024 || k > moe::kMaxK || n_shared > 1)
     return MOE_ERR_UNSUPPORTED;
-  if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32) return MOE_ERR_UNSUPPORTED;
+  if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16)
+    return MOE_ERR_UNSUPPORTED;
   if ((long long)max_T * (k + n_shared) > (1LL << 26)) return MOE_ERR_UNSUPPORTED;
 
   int dev = 0;
@@ -199,7 +207,9 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   if (const char* env = getenv("MOE_GREEN_CTX")) c->gc_sms = atoi(env);  // applied below, once created
   if (const char* env = getenv("MOE_TILE_N")) {
     const int v = atoi(env);
-    if (v == 16 || v == 32 || v == 64 || (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128)) c->tile_n_override = v;
+    if (v == 16 || v == 32 || (v == 64 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) ||
+        (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128))
+      c->tile_n_override = v;
   }
 
   const size_t HB = H / 128, IB = I / 128;
@@ -221,6 +231,9 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_xs = take(sizeof(float) * (size_t)c->S_pad * HB);
   const size_t o_hs = take(sizeof(float) * (size_t)c->S_pad * IB);
   const size_t o_acc = take(sizeof(float) * (size_t)max_T * H);
+  const bool nvfp4 = wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16;
+  const size_t o_xsc = nvfp4 ? take((size_t)(H / 64) * c->S_pad * 16) : 0;
+  const size_t o_hsc = nvfp4 ? take((size_t)(I / 64) * c->S_pad * 16) : 0;
   const bool want_rows = c->combine_mode == 2;
   const size_t o_rows = want_rows ? take(sizeof(float) * (size_t)c->S_pad * H) : 0;
   // fused router workspace (E <= 256, E % 4 == 0): logits of every token tile + a counter per tile
@@ -253,6 +266,16 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->xs = reinterpret_cast<float*>(b + o_xs);
   c->hs = reinterpret_cast<float*>(b + o_hs);
   c->out_acc = reinterpret_cast<float*>(b + o_acc);
+  c->xsc = nvfp4 ? reinterpret_cast<uint8_t*>(b + o_xsc) : nullptr;
+  c->hsc = nvfp4 ? reinterpret_cast<uint8_t*>(b + o_hsc) : nullptr;
+  if (nvfp4 && (!make_map(&c->tm_xsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xsc, 16, (uint64_t)(H / 64) * c->S_pad, 16,
+                          32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+                !make_map(&c->tm_hsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hsc, 16, (uint64_t)(I / 64) * c->S_pad, 16,
+                          32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16, CU_TENSOR_MAP_SWIZZLE_NONE))) {
+    cudaFree(base);
+    delete c;
+    return MOE_ERR_CUDA;
+  }
   c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
   c->rt_logits = want_router ? reinterpret_cast<float*>(b + o_rt_logits) : nullptr;
   c->rt_counters = want_router ? reinterpret_cast<int32_t*>(b + o_rt_counters) : nullptr;
@@ -348,14 +371,19 @@ void moe_destroy(moe_ctx* c) {
   delete c;
 }
 
-moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w, const void* w13,
-                       const void* s13, const void* w2, const void* s2, void* out, void* stream) {
+// The launch sequence of one layer for every weight format; g13 / g2 are the
+// NVFP4 global scales (null for the other formats).
+static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,
+                               const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
+                               const float* g2, void* out, void* stream) {
   if (!c || T < 0 || T > c->max_T) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
   if (!x || !ids || !topk_w || !w13 || !s13 || !w2 || !s2 || !out) return MOE_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(out, 16) || !aligned(w13, 128) || !aligned(w2, 128) || !aligned(s13, 16) ||
       !aligned(s2, 16) || !aligned(ids, 4) || !aligned(topk_w, 4))
     return MOE_ERR_INVALID_ARG;
+  const bool nvfp4 = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16);
+  if (nvfp4 && (!g13 || !g2 || !aligned(g13, 4) || !aligned(g2, 4))) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = c->H, I = c->I, NE = c->NG;
   const int S = T * c->k;
@@ -371,9 +399,14 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
 
   // weight maps (re-encoded only when the caller's pointers change)
   const CUtensorMapL2promotion wpromo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+  // NVFP4: packed bytes [rows, K/2], boxes of 64 bytes (one 128-wide K
+  // block) x 128 rows with 64-byte swizzle
+  constexpr CUtensorMapSwizzle sw64 = CU_TENSOR_MAP_SWIZZLE_64B;
   if (w13 != c->c_w13) {
     const bool ok = fp8 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H, (uint64_t)NE * 2 * I, H, 128,
                                    wpromo)
+                    : nvfp4 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H / 2, (uint64_t)NE * 2 * I,
+                                       H / 2, 128, wpromo, 64, sw64)
                         : make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13, H, (uint64_t)NE * 2 * I,
                                    H / 2, 128, wpromo);
     if (!ok) {
@@ -385,6 +418,8 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   if (w2 != c->c_w2) {
     const bool ok = fp8 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I, (uint64_t)NE * H, I, 128,
                                    wpromo)
+                    : nvfp4 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I / 2, (uint64_t)NE * H, I / 2,
+                                       128, wpromo, 64, sw64)
                         : make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2, I, (uint64_t)NE * H, I / 2,
                                    128, wpromo);
     if (!ok) {
@@ -394,10 +429,16 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
     c->c_w2 = w2;
   }
   if (BN != c->c_bn) {
-    if (!make_map(&c->tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H, c->S_pad, H, BN,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
-        !make_map(&c->tm_hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hq, I, c->S_pad, I, BN,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
+    const bool ok = nvfp4
+        ? make_map(&c->tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H / 2, c->S_pad, H / 2, BN,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 64, sw64) &&
+              make_map(&c->tm_hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hq, I / 2, c->S_pad, I / 2, BN,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 64, sw64)
+        : make_map(&c->tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H, c->S_pad, H, BN,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
+              make_map(&c->tm_hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hq, I, c->S_pad, I, BN,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+    if (!ok) {
       c->c_bn = 0;
       return MOE_ERR_CUDA;
     }
@@ -430,8 +471,10 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs;
   qp.xs_ld = c->S_pad;
   qp.out_acc = rows ? nullptr : c->out_acc;
+  qp.xsc = c->xsc;
   mark(MOE_STAGE_QUANT);
-  if (moe::launch_quant(qp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
+  if ((nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp) : moe::launch_quant(qp, s_disp)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   if (green) {
     if (cudaEventRecord(c->gev_disp, s_disp) != cudaSuccess || cudaStreamWaitEvent(s_gemm, c->gev_disp, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -448,15 +491,21 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
   g.y_rows = nullptr;
   g.inject = c->inject;
+  g.wglobal = g13;
+  g.hsc = c->hsc;
+  // the token block-code maps exist for NVFP4 only; the other formats ignore the argument
+  const CUtensorMap& tsx = nvfp4 ? c->tm_xsc : c->tm_xq;
+  const CUtensorMap& tsh = nvfp4 ? c->tm_hsc : c->tm_hq;
   mark(MOE_STAGE_GEMM1);
-  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
   g.kblocks = I / 128;
   g.wscale = static_cast<const float*>(s2);
+  g.wglobal = g2;
   g.ascale = c->hs;
   mark(MOE_STAGE_GEMM2);
   g.y_rows = rows ? c->y_rows : nullptr;
-  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, tsh, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
   mark(MOE_STAGE_FINALIZE);
   if (rows) {
@@ -476,6 +525,19 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
   c->last_bn = BN;
   c->last_grid = grid;
   return MOE_OK;
+}
+
+moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w, const void* w13,
+                       const void* s13, const void* w2, const void* s2, void* out, void* stream) {
+  if (c && c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_INVALID_ARG;  // needs moe_forward_nvfp4
+  return forward_impl(c, T, x, ids, topk_w, w13, s13, nullptr, w2, s2, nullptr, out, stream);
+}
+
+moe_status moe_forward_nvfp4(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,
+                             const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
+                             const float* g2, void* out, void* stream) {
+  if (!c || c->wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_INVALID_ARG;
+  return forward_impl(c, T, x, ids, topk_w, w13, s13, g13, w2, s2, g2, out, stream);
 }
 
 moe_status moe_router_topk(moe_ctx* c, int T, const void* x, const void* wr, int32_t* topk_ids, float* topk_w,
@@ -526,6 +588,13 @@ moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
   return MOE_OK;
 }
 
+moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream) {
+  if (!src || !dst || src == dst || rows <= 0 || K <= 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
+  if (moe::launch_pack_e8m0(src, dst, rows, K / 16, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
+}
+
 moe_status moe_get_routing(moe_ctx* c, int32_t* counts, int32_t* offsets, int32_t* perm, int32_t* inv,
                            void* stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
@@ -545,8 +614,9 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
   cudaError_t e = cudaSuccess;
-  if (xq && P && e == cudaSuccess) e = cudaMemcpy(xq, c->xq, P * c->H, cudaMemcpyDefault);
-  if (hq && P && e == cudaSuccess) e = cudaMemcpy(hq, c->hq, P * c->I, cudaMemcpyDefault);
+  const size_t cw = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) ? 2 : 1;  // codes per byte
+  if (xq && P && e == cudaSuccess) e = cudaMemcpy(xq, c->xq, P * c->H / cw, cudaMemcpyDefault);
+  if (hq && P && e == cudaSuccess) e = cudaMemcpy(hq, c->hq, P * c->I / cw, cudaMemcpyDefault);
   // The scales are stored K-block major on the device ([K/128][S_pad]); the
   // caller gets them position major ([P][K/128]).
   auto scales = [&](float* dst, const float* src, int kb) {
@@ -573,6 +643,37 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
   };
   scales(xs, c->xs, c->H / 128);
   scales(hs, c->hs, c->I / 128);
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+moe_status moe_get_block_scales(moe_ctx* c, uint8_t* xsc, uint8_t* hsc, void* stream) {
+  if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_UNSUPPORTED;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
+  cudaError_t e = cudaSuccess;
+  // device [K/64][S_pad][16] (four codes per step and position) -> caller [P][K/16]
+  auto gather = [&](uint8_t* dst, const uint8_t* src, int K) {
+    if (!dst || !P || e != cudaSuccess) return;
+    const size_t steps = (size_t)K / 64;
+    uint8_t* tmp = new (std::nothrow) uint8_t[steps * P * 4];
+    uint8_t* out = new (std::nothrow) uint8_t[steps * P * 4];
+    if (!tmp || !out) {
+      e = cudaErrorMemoryAllocation;
+    } else {
+      for (size_t st = 0; st < steps && e == cudaSuccess; ++st)
+        e = cudaMemcpy2D(tmp + st * P * 4, 4, src + st * c->S_pad * 16, 16, 4, P, cudaMemcpyDeviceToHost);
+      if (e == cudaSuccess) {
+        for (size_t i = 0; i < P; ++i)
+          for (size_t st = 0; st < steps; ++st) memcpy(out + (i * steps + st) * 4, tmp + (st * P + i) * 4, 4);
+        e = cudaMemcpy(dst, out, steps * P * 4, cudaMemcpyDefault);
+      }
+    }
+    delete[] tmp;
+    delete[] out;
+  };
+  gather(xsc, c->xsc, c->H);
+  gather(hsc, c->hsc, c->I);
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 

@@ -48,9 +48,17 @@ namespace moe {
 template <int KIND, int BN, int WFMT>
 struct GemmCfg {
   static constexpr int NA = (KIND == 1) ? 2 : 1;          // weight tiles per stage (gate + up)
-  static constexpr int A_BYTES = 128 * 128;               // 128 rows x 128 K bytes (E2M1 padded to 8 bits)
-  static constexpr int B_BYTES = BN * 128;
-  static constexpr int SF_BYTES = (WFMT == 1) ? NA * 512 : 0;
+  // NVFP4 (WFMT 2): both operands packed E2M1, 64 bytes per row per 128-wide
+  // K block, 64-byte swizzle; the block scales of a K block travel with the
+  // stage as 512-byte atoms, two per weight tile and two for the token tile
+  // (one per K = 64 MMA step each).
+  static constexpr bool NV = WFMT == 2;
+  static constexpr int KBYTES = NV ? 64 : 128;            // smem bytes per row per K block
+  static constexpr int A_BYTES = 128 * KBYTES;            // FP8 / E2M1 padded to 8 bits: 128 B rows
+  static constexpr int B_BYTES = BN * KBYTES;
+  static constexpr int SFA_BYTES = (WFMT == 1) ? 512 : NV ? 1024 : 0;  // per weight tile
+  static constexpr int SFB_BYTES = NV ? 1024 : 0;
+  static constexpr int SF_BYTES = NA * SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int KB_MAX = 64;                       // K <= 8192
   static constexpr int CG = (BN <= 64) ? 1 : BN / 64;     // epilogue column groups
@@ -76,7 +84,7 @@ struct GemmCfg {
   static constexpr int MMA_WARP = NPROD;  // first MMA warp; allocates TMEM
   static constexpr int EPI_WARP0 = NPROD + NMMA;
   static constexpr int THREADS = 32 * EPI_WARP0 + EPI_THREADS;
-  static constexpr int MAX_STAGES = 12;
+  static constexpr int MAX_STAGES = NV ? 24 : 12;
   // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
   // the promoting epilogue (short K steps would otherwise be latency bound).
   static constexpr int NBUF_RAW = 256 / (NA * BN);
@@ -89,9 +97,14 @@ struct GemmCfg {
   static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
   static constexpr int ACC_COLS = NBUF * NA * BN;         // NBUF accumulators
-  static constexpr int SFA_COL = ACC_COLS;                // MXFP4: NBUF x NA x 4 columns
-  static constexpr int SFB_COL = SFA_COL + NBUF * NA * 4; // MXFP4: 4 columns of unit scales
-  static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : ACC_COLS;
+  // Scale-factor columns per accumulator buffer: MXFP4 one 4-column atom per
+  // weight tile (B: 4 shared columns of unit scales); NVFP4 two atoms per
+  // weight tile and two for the token tile.  An MMA's scale operand starts
+  // at a 4-column atom boundary.
+  static constexpr int SFA_PER_BUF = NV ? NA * 8 : NA * 4;
+  static constexpr int SFA_COL = ACC_COLS;
+  static constexpr int SFB_COL = SFA_COL + NBUF * SFA_PER_BUF;
+  static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : NV ? SFB_COL + NBUF * 8 : ACC_COLS;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                  : USED_COLS <= 256 ? 256 : 512;
   // Transaction bytes per stage: a packed-E2M1 weight tile moves 64 bytes per
@@ -101,6 +114,9 @@ struct GemmCfg {
   static_assert(STAGES >= 2, "shared memory too small");
   static_assert(USED_COLS <= 512, "TMEM too small");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 64, "BN");
+  // NVFP4 token scales: an atom is one box of 32 positions, token n of the
+  // tile in row n (TMEM lane n, the atom's first column).
+  static_assert(!NV || BN <= 32, "NVFP4 tiles hold at most 32 tokens");
 };
 
 // Bounded wait that ignores the abort word (used to drain in-flight copies
@@ -115,16 +131,17 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 template <int KIND, int BN, int WFMT>
 __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmS, const GemmParams p) {
   using C = GemmCfg<KIND, BN, WFMT>;
   constexpr int NA = C::NA, STAGES = C::STAGES, KB_MAX = C::KB_MAX, CPT = C::CPT;
+  constexpr bool NV = C::NV;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = sA + STAGES * NA * C::A_BYTES;
   uint8_t* sSF = sB + STAGES * C::B_BYTES;
   float* asc = reinterpret_cast<float*>(sSF + STAGES * C::SF_BYTES);  // [KB_MAX][BN] activation scales
-  float* wsc = asc + BN * KB_MAX;                                     // [NA][KB_MAX] FP8 weight scales
+  float* wsc = asc + BN * KB_MAX;                                     // [NA][KB_MAX] FP8 weight scales (NVFP4: [0] global)
   float* red = wsc + NA * KB_MAX;                                     // [4][BN] per-quarter amax
   int* slot_tok = reinterpret_cast<int*>(red + 4 * BN);               // [BN] GEMM2: token of column
   float* slot_w = reinterpret_cast<float*>(slot_tok + BN);            // [BN] GEMM2: combine weight
@@ -165,6 +182,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA);
     tma_prefetch_map(&tmB);
+    if constexpr (NV) tma_prefetch_map(&tmS);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -215,7 +233,17 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     bool waited = false;
     constexpr int NPEND = (STAGES + C::NPROD - 1) / C::NPROD;
     int npend = 0;
-    int pend_c0[NPEND], pend_p0[NPEND], pend_st[NPEND];
+    int pend_kb[NPEND], pend_p0[NPEND], pend_st[NPEND];
+    // token tile of K block kb at positions p0.. (NVFP4: plus the block-code
+    // atoms of its two MMA steps, rows ks * scale_ld + p0 .. + 31)
+    auto load_tokens = [&](int st, int kb, int p0) {
+      tma_load_2d(&tmB, &full[st], sB + st * C::B_BYTES, kb * C::KBYTES, p0, pol_a);
+      if constexpr (NV) {
+        uint8_t* dst = sSF + st * C::SF_BYTES + NA * C::SFA_BYTES;
+        tma_load_2d(&tmS, &full[st], dst, 0, (2 * kb) * p.scale_ld + p0, pol_a);
+        tma_load_2d(&tmS, &full[st], dst + 512, 0, (2 * kb + 1) * p.scale_ld + p0, pol_a);
+      }
+    };
     int it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const int rt = C::TILE_MAJOR ? u % NRT : u / num_tiles, ti = C::TILE_MAJOR ? u / NRT : u % num_tiles;
@@ -229,8 +257,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
         if (tok_lane && !waited && it >= STAGES) {
           griddep_wait();
-          for (int i = 0; i < npend; ++i)
-            tma_load_2d(&tmB, &full[pend_st[i]], sB + pend_st[i] * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
+          for (int i = 0; i < npend; ++i) load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
           waited = true;
         }
         if (lane == 0 && ok && it >= STAGES) {  // the stage's previous iteration has been consumed
@@ -250,17 +277,18 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
           }
           __syncwarp();
           if (lane < NJ - 1) {
-            tma_load_2d(&tmA, &full[stage], sA + (stage * NA + lane) * C::A_BYTES, kb * 128, row, pol_w);
-            if constexpr (WFMT == 1) {
+            tma_load_2d(&tmA, &full[stage], sA + (stage * NA + lane) * C::A_BYTES, kb * C::KBYTES, row, pol_w);
+            if constexpr (WFMT == 1 || NV) {
+              // the K block's block-scale atoms of these 128 rows (packed layout)
               const uint8_t* sf = reinterpret_cast<const uint8_t*>(p.wscale);
-              bulk_load(sSF + stage * C::SF_BYTES + lane * 512, sf + ((size_t)(row / 128) * KB + kb) * 512, 512,
-                        &full[stage], pol_w);
+              bulk_load(sSF + stage * C::SF_BYTES + lane * C::SFA_BYTES,
+                        sf + ((size_t)(row / 128) * KB + kb) * C::SFA_BYTES, C::SFA_BYTES, &full[stage], pol_w);
             }
           } else if (tok_lane) {
             if (waited) {
-              tma_load_2d(&tmB, &full[stage], sB + stage * C::B_BYTES, kb * 128, p0, pol_a);
+              load_tokens(stage, kb, p0);
             } else {
-              pend_c0[npend] = kb * 128;
+              pend_kb[npend] = kb;
               pend_p0[npend] = p0;
               pend_st[npend] = stage;
               ++npend;
@@ -271,8 +299,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     }
     if (tok_lane && !waited) {
       griddep_wait();
-      for (int i = 0; i < npend; ++i)
-        tma_load_2d(&tmB, &full[pend_st[i]], sB + pend_st[i] * C::B_BYTES, pend_c0[i], pend_p0[i], pol_a);
+      for (int i = 0; i < npend; ++i) load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
     }
     // Without an abort every issued load was consumed by the MMA warps.  After
     // one, wait (bounded) for this warp's last loads into each stage; a later
@@ -299,9 +326,40 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
           tc_fence_after();
           if (lane == 0) {
             const uint32_t d0 = tmem + buf * (NA * BN);
-            const uint64_t ad = sdesc_k_sw128(smem_u32(sA + stage * NA * C::A_BYTES));
-            const uint64_t bd = sdesc_k_sw128(smem_u32(sB + stage * C::B_BYTES));
-            if constexpr (WFMT == 0) {
+            const uint64_t ad = NV ? sdesc_k_sw64(smem_u32(sA + stage * NA * C::A_BYTES))
+                                   : sdesc_k_sw128(smem_u32(sA + stage * NA * C::A_BYTES));
+            const uint64_t bd = NV ? sdesc_k_sw64(smem_u32(sB + stage * C::B_BYTES))
+                                   : sdesc_k_sw128(smem_u32(sB + stage * C::B_BYTES));
+            if constexpr (NV) {
+              // Scale atoms of this K block, smem -> TMEM (columns of buffer
+              // buf): per weight tile a, atoms of K steps 0 and 1 at sfa + 8a
+              // and sfa + 8a + 4; the token atoms at sfb and sfb + 4.
+              const uint32_t sfa = tmem + C::SFA_COL + buf * C::SFA_PER_BUF;
+              const uint32_t sfb = tmem + C::SFB_COL + buf * 8;
+              uint8_t* sfs = sSF + stage * C::SF_BYTES;
+              auto cp_atom = [&](uint32_t taddr, const uint8_t* src) {
+                uint64_t sd = 0;
+                sd |= static_cast<uint64_t>((smem_u32(src) & 0x3FFFFu) >> 4);
+                sd |= static_cast<uint64_t>(128 >> 4) << 32;  // 8 rows x 16 bytes per core group
+                sd |= static_cast<uint64_t>(1) << 46;
+                tmem_cp_32x128b_warpx4(taddr, sd);
+              };
+#pragma unroll
+              for (int a = 0; a < NA; ++a) {
+                cp_atom(sfa + a * 8, sfs + a * 1024);
+                cp_atom(sfa + a * 8 + 4, sfs + a * 1024 + 512);
+              }
+              cp_atom(sfb, sfs + NA * 1024);
+              cp_atom(sfb + 4, sfs + NA * 1024 + 512);
+              constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                mma_mxf4nvf4(d0, ad + 2 * ks, bd + 2 * ks, idesc, sfa + ks * 4, sfb + ks * 4, ks > 0);
+                if constexpr (KIND == 1)
+                  mma_mxf4nvf4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * ks, bd + 2 * ks, idesc, sfa + 8 + ks * 4,
+                               sfb + ks * 4, ks > 0);
+              }
+            } else if constexpr (WFMT == 0) {
               constexpr uint32_t idesc = idesc_f8f6f4(128, BN, AF, 0);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
@@ -386,6 +444,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
           pw = p.wscale[((size_t)tile_n.x * RB + rb) * KB + kb];
         }
       }
+      if constexpr (NV) {
+        if (etid == 0) pw = p.wglobal[tile_n.x];
+      }
     };
     bool from_regs = false;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
@@ -401,6 +462,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         if constexpr (WFMT == 0) {
           if (etid < NA * KB) wsc[(etid / KB) * KB_MAX + etid % KB] = pw;
         }
+        if constexpr (NV) {
+          if (etid == 0) wsc[0] = pw;
+        }
       } else {
         for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
           const int kb = i / BN, j = i % BN;
@@ -412,6 +476,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
             const int rb = (a == 0) ? rt : p.I / 128 + rt;
             wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + rb) * KB + kb];
           }
+        }
+        if constexpr (NV) {
+          if (etid == 0) wsc[0] = p.wglobal[e];
         }
         if constexpr (KIND == 2) {
           for (int j = etid; j < BN; j += C::EPI_THREADS) {
@@ -438,13 +505,16 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       }
       // Combined scale of K block kb per tile column, shared by all 128 rows:
       // cs[kb & 1][a][j] = activation scale (column j, kb) x weight block
-      // scale (tile a, kb) (MXFP4: the activation scale alone).  Filled one K
-      // block ahead by the epilogue threads, one named barrier per K block.
+      // scale (tile a, kb) (MXFP4: the activation scale alone; NVFP4: x the
+      // expert's global scale).  Filled one K block ahead by the epilogue
+      // threads, one named barrier per K block.
       auto fill_cs = [&](int kb) {
         float* dst = cs + (kb & 1) * (NA * BN);
         for (int i = etid; i < NA * BN; i += C::EPI_THREADS) {
           const int a = i / BN, j = i - (i / BN) * BN;
-          dst[i] = (WFMT == 0) ? asc[kb * BN + j] * wsc[a * KB_MAX + kb] : asc[kb * BN + j];
+          dst[i] = (WFMT == 0) ? asc[kb * BN + j] * wsc[a * KB_MAX + kb]
+                   : NV        ? asc[kb * BN + j] * wsc[0]
+                               : asc[kb * BN + j];
         }
       };
       fill_cs(0);
@@ -510,7 +580,49 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         }
       }
 
-      if constexpr (KIND == 1) {
+      if constexpr (KIND == 1 && NV) {
+        // SwiGLU, then NVFP4 requantisation of each token's 128 channels
+        // (the rule of quant_nvfp4_kernel): lanes 16i .. 16i+15 of a warp
+        // hold one 16-channel block, the tile's four warps one 128 group.
+        float* h = acc0;
+        float a16[CPT];
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) {
+          const float g = acc0[c];
+          const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+          h[c] = g * sig * acc1[c];
+          float m = fabsf(h[c]);
+#pragma unroll
+          for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+          a16[c] = m;
+          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+          if (lane == 0) red[q * BN + cg * CPT + c] = m;
+        }
+        named_sync(1, C::EPI_THREADS);
+        if (ok) {
+          const int ch = rt * 128 + row;
+#pragma unroll
+          for (int c = 0; c < CPT; ++c) {
+            const int j = cg * CPT + c;
+            const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
+            const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+            const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16[c], 6.0f), sg));
+            const float d = __fmul_rn(e4m3_code_value(code), sg);
+            const uint32_t nib = code ? f32_to_e2m1(__fdiv_rn(h[c], d)) : 0u;
+            // eight neighbouring channels -> one 32-bit word of packed codes
+            uint32_t word = nib << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+            if (j < nv) {
+              if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
+              if ((lane & 15) == 0)
+                p.hsc[((size_t)(ch / 64) * p.scale_ld + p0 + j) * 16 + (ch / 16) % 4] = static_cast<uint8_t>(code);
+              if (row == 0) p.hs[(size_t)rt * p.scale_ld + p0 + j] = sg;
+            }
+          }
+        }
+      } else if constexpr (KIND == 1) {
         // SwiGLU (gate rows 0..I-1 of W13, up rows I..2I-1: same channel),
         // then FP8 requantisation per token over the tile's 128 channels.
         float* h = acc0;  // h overwrites the gate accumulator in place
@@ -581,8 +693,8 @@ static cudaError_t set_attr() {
 }
 
 template <int KIND, int BN, int WFMT>
-static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const GemmParams& p,
-                          cudaStream_t s) {
+static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
+                          const GemmParams& p, cudaStream_t s) {
   using C = GemmCfg<KIND, BN, WFMT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
@@ -594,7 +706,7 @@ static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT>, ta, tb, p);
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT>, ta, tb, ts, p);
 }
 
 cudaError_t gemm_setup(int wfmt) {
@@ -605,47 +717,60 @@ cudaError_t gemm_setup(int wfmt) {
     MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0)
     MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0)
     if (e == cudaSuccess) e = gemm_tm_setup();
-  } else {
+  } else if (wfmt == 1) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
     MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
+  } else {
+    MOE_SET(1, 16, 2) MOE_SET(1, 32, 2)
+    MOE_SET(2, 16, 2) MOE_SET(2, 32, 2)
   }
 #undef MOE_SET
   return e;
 }
 
 cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& tx,
-                         const GemmParams& p, cudaStream_t s) {
+                         const CUtensorMap& tsf, const GemmParams& p, cudaStream_t s) {
   if (wfmt == 0) {
     switch (BN) {
-      case 16: return launch<1, 16, 0>(grid, tw, tx, p, s);
-      case 32: return launch<1, 32, 0>(grid, tw, tx, p, s);
-      case 64: return launch<1, 64, 0>(grid, tw, tx, p, s);
+      case 16: return launch<1, 16, 0>(grid, tw, tx, tsf, p, s);
+      case 32: return launch<1, 32, 0>(grid, tw, tx, tsf, p, s);
+      case 64: return launch<1, 64, 0>(grid, tw, tx, tsf, p, s);
       case 128: return launch_gemm1_tm(grid, tw, tx, p, s);
+    }
+  } else if (wfmt == 1) {
+    switch (BN) {
+      case 16: return launch<1, 16, 1>(grid, tw, tx, tsf, p, s);
+      case 32: return launch<1, 32, 1>(grid, tw, tx, tsf, p, s);
+      case 64: return launch<1, 64, 1>(grid, tw, tx, tsf, p, s);
     }
   } else {
     switch (BN) {
-      case 16: return launch<1, 16, 1>(grid, tw, tx, p, s);
-      case 32: return launch<1, 32, 1>(grid, tw, tx, p, s);
-      case 64: return launch<1, 64, 1>(grid, tw, tx, p, s);
+      case 16: return launch<1, 16, 2>(grid, tw, tx, tsf, p, s);
+      case 32: return launch<1, 32, 2>(grid, tw, tx, tsf, p, s);
     }
   }
   return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
-                         const GemmParams& p, cudaStream_t s) {
+                         const CUtensorMap& tsf, const GemmParams& p, cudaStream_t s) {
   if (wfmt == 0) {
     switch (BN) {
-      case 16: return launch<2, 16, 0>(grid, tw, th, p, s);
-      case 32: return launch<2, 32, 0>(grid, tw, th, p, s);
-      case 64: return launch<2, 64, 0>(grid, tw, th, p, s);
+      case 16: return launch<2, 16, 0>(grid, tw, th, tsf, p, s);
+      case 32: return launch<2, 32, 0>(grid, tw, th, tsf, p, s);
+      case 64: return launch<2, 64, 0>(grid, tw, th, tsf, p, s);
       case 128: return launch_gemm2_tm(grid, tw, th, p, s);
+    }
+  } else if (wfmt == 1) {
+    switch (BN) {
+      case 16: return launch<2, 16, 1>(grid, tw, th, tsf, p, s);
+      case 32: return launch<2, 32, 1>(grid, tw, th, tsf, p, s);
+      case 64: return launch<2, 64, 1>(grid, tw, th, tsf, p, s);
     }
   } else {
     switch (BN) {
-      case 16: return launch<2, 16, 1>(grid, tw, th, p, s);
-      case 32: return launch<2, 32, 1>(grid, tw, th, p, s);
-      case 64: return launch<2, 64, 1>(grid, tw, th, p, s);
+      case 16: return launch<2, 16, 2>(grid, tw, th, tsf, p, s);
+      case 32: return launch<2, 32, 2>(grid, tw, th, tsf, p, s);
     }
   }
   return cudaErrorInvalidValue;

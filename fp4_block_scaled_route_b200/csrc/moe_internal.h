@@ -32,6 +32,12 @@ struct QuantParams {
   float* xs;              // [H/128, xs_ld]    K-block major: one row of position scales per K block
   int xs_ld;              // = S_pad
   float* out_acc;         // [T, H] zeroed here (null: not needed)
+  // NVFP4 activations (quant_nvfp4_kernel): xq holds packed E2M1 [S_pad, H/2]
+  // and xsc the E4M3 block codes as [H/64][xs_ld][16] bytes: per 64-column
+  // MMA step and position, the step's four codes in bytes 0..3 (bytes 4..15
+  // stay zero), so that 32 consecutive positions of one step form a
+  // block-scale atom of the MMA's B operand.
+  uint8_t* xsc;
 };
 
 struct GemmParams {
@@ -50,6 +56,10 @@ struct GemmParams {
   int32_t* status;
   float* y_rows;          // GEMM2: non-null = store fp32 rows [S_pad, H] instead of the fused combine
   int inject;             // failure-injection test hook (0 in normal use), see moe_set_fault_injection
+  // NVFP4: wscale = packed E4M3 block-scale atoms; wglobal = fp32 [NE] global
+  // scales; GEMM1 writes hq as packed E2M1 [S_pad, I/2] plus hsc block codes.
+  const float* wglobal;
+  uint8_t* hsc;           // GEMM1: E4M3 block codes [I/64][scale_ld][16] (layout of QuantParams::xsc)
 };
 
 struct CombineParams {
@@ -81,13 +91,16 @@ cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, const Ro
 size_t route_smem_bytes(int n_groups);
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);
+cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s);
 cudaError_t gemm_setup(int wfmt);  // raise shared-memory limits once per process
 // tw: weight tiles; tx / th: token tiles.
+// tsf: NVFP4 token block-scale codes, map over [K/64 * S_pad rows, 16 bytes]
+// with boxes of 32 rows; unused otherwise.
 cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& tx,
-                         const GemmParams& p, cudaStream_t s);
+                         const CUtensorMap& tsf, const GemmParams& p, cudaStream_t s);
 cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
-                         const GemmParams& p, cudaStream_t s);
+                         const CUtensorMap& tsf, const GemmParams& p, cudaStream_t s);
 // Token-major kernels for 128-token tiles (FP8 weights), moe_gemm_tm.cu.
 cudaError_t gemm_tm_setup();
 cudaError_t launch_gemm1_tm(int grid, const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,

@@ -188,11 +188,12 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   g.tiles = rp.tiles; g.num_tiles = rp.num_tiles; g.status = status;
   g.y_rows = nullptr;  // fused combine into the fp32 accumulator
   g.inject = 0;
-  if (moe::launch_gemm1(wfmt, BN, g_num_sms[dev], tw13, txq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  g.wglobal = nullptr; g.hsc = nullptr;
+  if (moe::launch_gemm1(wfmt, BN, g_num_sms[dev], tw13, txq, txq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
   g.kblocks = I / 128;
   g.wscale = static_cast<const float*>(s2);
   g.ascale = hs;
-  if (moe::launch_gemm2(wfmt, BN, g_num_sms[dev], tw2, thq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::launch_gemm2(wfmt, BN, g_num_sms[dev], tw2, thq, thq, g, s) != cudaSuccess) return MOE_ERR_CUDA;
   if (moe::launch_finalize(acc, static_cast<uint16_t*>(out), (long long)T * H, s) != cudaSuccess)
     return MOE_ERR_CUDA;
   return MOE_OK;

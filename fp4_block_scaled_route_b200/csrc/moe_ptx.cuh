@@ -140,6 +140,18 @@ __device__ __forceinline__ uint64_t sdesc_k_sw128(uint32_t saddr) {
   return d;
 }
 
+// The same for a K-major tile written by TMA with 64-byte swizzle: rows of
+// 64 bytes, 8-row core groups 512 bytes apart, tile base 512-byte aligned.
+__device__ __forceinline__ uint64_t sdesc_k_sw64(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);  // start address
+  d |= static_cast<uint64_t>(1) << 16;                  // leading byte offset (unused: K fits one row)
+  d |= static_cast<uint64_t>(512 >> 4) << 32;           // stride byte offset
+  d |= static_cast<uint64_t>(1) << 46;                  // descriptor version for sm_100
+  d |= static_cast<uint64_t>(4) << 61;                  // layout: 64-byte swizzle
+  return d;
+}
+
 // Instruction descriptor, kind::f8f6f4, fp32 accumulate, both operands
 // K-major.  fmt: 0 = E4M3, 5 = E2M1 (unpacked in shared memory).
 __host__ __device__ constexpr uint32_t idesc_f8f6f4(int M, int N, int a_fmt, int b_fmt) {
@@ -159,6 +171,18 @@ __host__ __device__ constexpr uint32_t idesc_mxf8f6f4(int M, int N, int a_fmt, i
          | (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(a_sf_id) << 29);
 }
 
+// Instruction descriptor, kind::mxf4nvf4.block_scale with E4M3 (UE4M3)
+// scales per 16 elements: both operands packed E2M1 (format 1), K-major,
+// dense K = 64, fp32 accumulate, scale-factor ids 0 (all four bytes of a
+// scale column are used).
+__host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
+  return (1u << 7)                                   // A format E2M1
+         | (1u << 10)                                // B format E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (0u << 23)                                // scale format UE4M3
+         | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
+}
+
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                            uint32_t accumulate) {
   asm volatile(
@@ -175,6 +199,20 @@ __device__ __forceinline__ void mma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, ui
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// One K = 64 step of packed-E2M1 operands with E4M3 scales per 16 elements:
+// the scale column of A row m holds its four block scales (byte i = K
+// elements 16i .. 16i+15 of the step), likewise for B column n.
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
@@ -271,6 +309,37 @@ __device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Value of a non-negative E4M3 code (OCP FP8: bias 7, 3 mantissa bits;
+// exponent field 0 is subnormal, m * 2^-9).  Exact; NaN (0x7F) never occurs
+// for the codes produced here (the conversions saturate at 448).
+__device__ __forceinline__ float e4m3_code_value(uint32_t code) {
+  const uint32_t e = (code >> 3) & 0xFu, m = code & 7u;
+  return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+}
+
+// fp32 -> E2M1 code (low nibble), round-to-nearest-even, saturating to +-6;
+// the sign bit is kept also when the magnitude rounds to zero.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(0.0f), "f"(v));
+  return r & 0xFu;
+}
+
+// Four fp32 values -> four E2M1 codes, value i in bits 4i .. 4i+3.
+__device__ __forceinline__ uint32_t f32x4_to_e2m1x4(float v0, float v1, float v2, float v3) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t0, t1;\n\t.reg .b16 h;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t1, %4, %3;\n\t"
+      "mov.b16 h, {t0, t1};\n\t"
+      "cvt.u32.u16 %0, h;\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
   return r;
 }
 

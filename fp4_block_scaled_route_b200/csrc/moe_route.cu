@@ -213,6 +213,77 @@ cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
+// NVFP4 form of step 2 (NVIDIA NVFP4: E2M1 elements, E4M3 scale per 16, fp32
+// second-level scale; the second level per token per 128 columns, the FP8
+// activation group of the FusedDeepMoE QuantToken step):
+//   S = amax128 / 2688 (1 for an all-zero group), block code
+//   c = e4m3((amax16 / 6) / S), element code q = e2m1(v / (e4m3_value(c) * S))
+//   (q = 0 when c = 0), every operation one IEEE fp32 operation.
+// Same grid as quant_kernel; a lane holds 4 consecutive columns, so a 16-
+// column block is 4 neighbouring lanes and a 64-column MMA step 16 lanes.
+// Outputs per routed position: packed codes (element 2c in the low nibble of
+// byte c), the four block codes of each step as one 32-bit word (layout of
+// QuantParams::xsc), S.
+__global__ void __launch_bounds__(kQuantThreads) quant_nvfp4_kernel(QuantParams p) {
+  griddep_launch_dependents();
+  const int t = blockIdx.x;
+  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  __shared__ int rows[kMaxK + 1];
+  __shared__ int nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int r = p.inv[t * p.k + j];
+      if (r >= 0) rows[n++] = r;
+    }
+    if (p.n_shared) rows[n++] = p.inv[S + t];
+    nrows = n;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xr = p.x + (size_t)t * H;
+  for (int g = warp; g < HB; g += kQuantThreads / 32) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    float f[4];
+    f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
+    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
+    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float a16 = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+    a16 = fmaxf(a16, __shfl_xor_sync(0xFFFFFFFFu, a16, 1));
+    a16 = fmaxf(a16, __shfl_xor_sync(0xFFFFFFFFu, a16, 2));
+    float amax = a16;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+    const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16, 6.0f), sg));
+    const float d = __fmul_rn(e4m3_code_value(code), sg);
+    uint32_t packed = 0;
+    if (code != 0)
+      packed = f32x4_to_e2m1x4(__fdiv_rn(f[0], d), __fdiv_rn(f[1], d), __fdiv_rn(f[2], d), __fdiv_rn(f[3], d));
+    // the step's four codes into one word (lanes 0 and 16 hold steps 2g, 2g+1)
+    uint32_t word = ((lane & 3) == 0) ? code << (8 * ((lane >> 2) & 3)) : 0u;
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
+    const size_t step = (size_t)(2 * g + (lane >> 4));
+    for (int r = 0; r < nrows; ++r) {
+      *reinterpret_cast<uint16_t*>(p.xq + (size_t)rows[r] * (H / 2) + g * 64 + lane * 2) = (uint16_t)packed;
+      if ((lane & 15) == 0) *reinterpret_cast<uint32_t*>(p.xsc + (step * p.xs_ld + rows[r]) * 16) = word;
+      if (lane == 0) p.xs[(size_t)g * p.xs_ld + rows[r]] = sg;
+    }
+  }
+  if (p.out_acc) {
+    float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
+    for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s) {
+  quant_nvfp4_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 __global__ void finalize_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, long long n4) {
   griddep_wait();  // the combine buffer is complete once GEMM2 has finished
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
@@ -305,10 +376,12 @@ cudaError_t launch_combine(const CombineParams& p, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
-// E8M0 scales, plain layout [rows, kgroups] (one byte per 32 K elements) ->
-// the block-scaled MMA layout: for each 128-row block and each 128-wide K
-// block, one 512-byte atom with row m's 4 scales at byte
-// (m % 32) * 16 + (m / 32) * 4 + (k-group within the K block).
+// Block scales, plain layout [rows, kgroups] (one byte per scale group along
+// K: E8M0 per 32 elements for MXFP4, E4M3 per 16 for NVFP4) -> the
+// block-scaled MMA layout: for each 128-row block and each run of four
+// groups (one 128-wide K block of MXFP4, one K = 64 MMA step of NVFP4), one
+// 512-byte atom with row m's 4 scales at byte
+// (m % 32) * 16 + (m / 32) * 4 + (group within the run).
 __global__ void pack_e8m0_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst, int rows, int kgroups) {
   const long long total = (long long)rows * kgroups;
   const int kblocks = kgroups / 4;

@@ -27,6 +27,7 @@ MOE_ERR_BAD_ROUTING = 6
 
 MOE_WFMT_FP8_E4M3_B128 = 0
 MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1
+MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2
 
 # Every entry point declared in include/moe.h: name -> (restype, argtypes)
 _vp = ctypes.c_void_p
@@ -36,9 +37,12 @@ SIGNATURES = {
     "moe_create_ex": (_i, [_i, _i, _i, _i, _i, _i, _i, ctypes.POINTER(_vp)]),
     "moe_destroy": (None, [_vp]),
     "moe_forward": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_forward_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_pack_mxfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
+    "moe_pack_nvfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
     "moe_get_routing": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_get_activations": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_get_block_scales": (_i, [_vp, _vp, _vp, _vp]),
     "moe_get_device_status": (_i, [_vp, _vp]),
     "moe_last_config": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "moe_set_fault_injection": (_i, [_vp, _i]),
@@ -106,6 +110,10 @@ def moe_forward(ctx, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, stream) -> i
     return lib().moe_forward(ctx, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, stream)
 
 
+def moe_forward_nvfp4(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out, stream) -> int:
+    return lib().moe_forward_nvfp4(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out, stream)
+
+
 def moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, d_status,
                         stream) -> int:
     return lib().moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13, s13, w2, s2, out,
@@ -114,6 +122,14 @@ def moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13,
 
 def moe_pack_mxfp4_scales(src, dst, rows, K, stream) -> int:
     return lib().moe_pack_mxfp4_scales(src, dst, rows, K, stream)
+
+
+def moe_pack_nvfp4_scales(src, dst, rows, K, stream) -> int:
+    return lib().moe_pack_nvfp4_scales(src, dst, rows, K, stream)
+
+
+def moe_get_block_scales(ctx, xsc, hsc, stream) -> int:
+    return lib().moe_get_block_scales(ctx, xsc, hsc, stream)
 
 
 def moe_get_routing(ctx, counts, offsets, perm, inv, stream) -> int:
@@ -198,16 +214,24 @@ class MoeLayer:
         except Exception:
             pass
 
-    def forward(self, x, topk_ids, topk_w, w13, s13, w2, s2, out=None, stream=None):
+    def forward(self, x, topk_ids, topk_w, w13, s13, w2, s2, out=None, stream=None, g13=None, g2=None):
+        """One layer; NVFP4 contexts also take the global scales g13 / g2 (moe_forward_nvfp4)."""
         import torch
         T = x.shape[0]
         if out is None:
             out = torch.empty((T, self.H), dtype=torch.bfloat16, device=x.device)
-        for t in (x, topk_ids, topk_w, w13, s13, w2, s2, out):
-            if not t.is_cuda or not t.is_contiguous():
+        nv = self.wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16
+        ts = (x, topk_ids, topk_w, w13, s13, w2, s2, out) + ((g13, g2) if nv else ())
+        for t in ts:
+            if t is None or not t.is_cuda or not t.is_contiguous():
                 raise ValueError("MoeLayer.forward needs contiguous CUDA tensors")
-        _check(moe_forward(self.ctx, T, _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(s13),
-                           _ptr(w2), _ptr(s2), _ptr(out), _stream_handle(stream)), "moe_forward")
+        if nv:
+            _check(moe_forward_nvfp4(self.ctx, T, _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(s13),
+                                     _ptr(g13), _ptr(w2), _ptr(s2), _ptr(g2), _ptr(out), _stream_handle(stream)),
+                   "moe_forward_nvfp4")
+        else:
+            _check(moe_forward(self.ctx, T, _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(s13),
+                               _ptr(w2), _ptr(s2), _ptr(out), _stream_handle(stream)), "moe_forward")
         return out
 
     def routing(self, T, stream=None):
@@ -224,16 +248,28 @@ class MoeLayer:
         return counts, offsets, perm[:P], inv[:P]
 
     def activations(self, T, stream=None):
-        """(xq, xs, hq, hs) of the last forward, host numpy arrays in routing-position order."""
+        """(xq, xs, hq, hs) of the last forward, host numpy arrays in routing-position order
+        (NVFP4: xq / hq packed, two codes per byte)."""
         import numpy as np
         P = T * self.k + self.n_shared * T
-        xq = np.zeros((max(P, 1), self.H), np.uint8)
+        cw = 2 if self.wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 else 1
+        xq = np.zeros((max(P, 1), self.H // cw), np.uint8)
         xs = np.zeros((max(P, 1), self.H // 128), np.float32)
-        hq = np.zeros((max(P, 1), self.I), np.uint8)
+        hq = np.zeros((max(P, 1), self.I // cw), np.uint8)
         hs = np.zeros((max(P, 1), self.I // 128), np.float32)
         _check(moe_get_activations(self.ctx, xq.ctypes.data, xs.ctypes.data, hq.ctypes.data, hs.ctypes.data,
                                    _stream_handle(stream)), "moe_get_activations")
         return xq[:P], xs[:P], hq[:P], hs[:P]
+
+    def block_scales(self, T, stream=None):
+        """NVFP4: (xsc [P, H/16], hsc [P, I/16]) E4M3 block codes of the last forward, host numpy."""
+        import numpy as np
+        P = T * self.k + self.n_shared * T
+        xsc = np.zeros((max(P, 1), self.H // 16), np.uint8)
+        hsc = np.zeros((max(P, 1), self.I // 16), np.uint8)
+        _check(moe_get_block_scales(self.ctx, xsc.ctypes.data, hsc.ctypes.data, _stream_handle(stream)),
+               "moe_get_block_scales")
+        return xsc[:P], hsc[:P]
 
     def device_status(self, stream=None) -> int:
         return moe_get_device_status(self.ctx, _stream_handle(stream))
@@ -260,6 +296,15 @@ class MoeLayer:
         """Green-Context partition: dispatch kernels on >= dispatch_sms SMs, GEMMs on the rest (0 = off)."""
         _check(moe_set_green_ctx(self.ctx, dispatch_sms), "moe_set_green_ctx")
         return moe_green_ctx_sms(self.ctx)
+
+
+def pack_nvfp4_scales(s, stream=None):
+    """Plain E4M3 block codes [NE, rows, K/16] (uint8 CUDA tensor) -> the layout moe_forward_nvfp4 reads."""
+    NE, rows, kg = s.shape
+    dst = __import__("torch").empty_like(s)
+    _check(moe_pack_nvfp4_scales(_ptr(s.contiguous()), _ptr(dst), NE * rows, kg * 16, _stream_handle(stream)),
+           "moe_pack_nvfp4_scales")
+    return dst
 
 
 def pack_mxfp4_scales(s, stream=None):

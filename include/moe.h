@@ -66,7 +66,16 @@ enum {
    * w2 u8 [NE, H, I/2]; scales are E8M0 (2^(e-127)) per 32 elements along K,
    * plain layout [NE, rows, K/32], converted once with moe_pack_mxfp4_scales()
    * into the layout moe_forward() reads. */
-  MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1
+  MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1,
+  /* NVFP4 (named among the 4-bit expert layouts of the onnxruntime QMoE
+   * offload PR page; NVIDIA's definition): w13 u8 [NE, 2I, H/2] and w2 u8
+   * [NE, H, I/2] E2M1 nibbles as for MXFP4; s13 / s2 E4M3 scale codes per 16
+   * elements along K, plain layout [NE, rows, K/16], converted once with
+   * moe_pack_nvfp4_scales(); g13 / g2 fp32 [NE] per-expert global scales.
+   * Weight value = e2m1 * e4m3(scale) * g.  The tensor cores take NVFP4 only
+   * with FP4 on both sides, so the activations are quantised to NVFP4 too
+   * (see moe_forward_nvfp4).  Used through moe_forward_nvfp4(). */
+  MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2
 };
 
 /* moe_create -- context for a layer with hidden size H, expert intermediate
@@ -115,12 +124,35 @@ moe_status moe_forward(moe_ctx* ctx, int T, const void* x, const int32_t* topk_i
                        const void* w13, const void* s13, const void* w2, const void* s2, void* out,
                        void* stream);
 
+/* moe_forward_nvfp4 -- one MoE layer with NVFP4 weights (a context created
+ * with MOE_WFMT_NVFP4_E2M1_E4M3_K16; other contexts: MOE_ERR_INVALID_ARG).
+ * Arguments as moe_forward(), plus the per-expert global scales g13, g2
+ * (device fp32 [NE], 4-byte aligned); s13 / s2 in the packed layout of
+ * moe_pack_nvfp4_scales().  Activations (x, and the SwiGLU output) are
+ * quantised to NVFP4 per token: for every 128 columns S = amax / 2688 (1 for
+ * an all-zero group), for every 16 columns an E4M3 code
+ * c = e4m3((amax16 / 6) / S), elements e2m1(v / (e4m3(c) * S)) (0 where
+ * c = 0).  Each 128-wide K block's MMA sum (E2M1 x E4M3 block scales of both
+ * operands, in the tensor cores) is scaled by S x g[expert] and accumulated
+ * in fp32.  Tiles hold at most 32 tokens. */
+moe_status moe_forward_nvfp4(moe_ctx* ctx, int T, const void* x, const int32_t* topk_ids, const float* topk_w,
+                             const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
+                             const float* g2, void* out, void* stream);
+
 /* moe_pack_mxfp4_scales -- converts E8M0 scales from the plain layout
  * [rows, K/32] (rows = NE*2I for s13, NE*H for s2) into the 128x128 atom
  * layout moe_forward() reads for MOE_WFMT_MXFP4_E2M1_E8M0_K32 (same byte
  * count).  src and dst are distinct device buffers; rows % 128 == 0 and
  * K % 128 == 0.  Weight-load-time step, asynchronous on `stream`. */
 moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream);
+
+/* moe_pack_nvfp4_scales -- converts NVFP4 E4M3 block-scale codes from the
+ * plain layout [rows, K/16] into the layout moe_forward_nvfp4() reads (same
+ * byte count): per 128 rows and per 64 elements along K one 512-byte atom,
+ * row m's four codes at bytes (m % 32) * 16 + (m / 32) * 4 + 0..3.  src and
+ * dst are distinct device buffers; rows % 128 == 0 and K % 128 == 0.
+ * Weight-load-time step, asynchronous on `stream`. */
+moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream);
 
 /* moe_get_routing -- copies the routing of the last moe_forward() (after a
  * stream synchronisation) into caller buffers (host or device):
@@ -136,8 +168,16 @@ moe_status moe_get_routing(moe_ctx* ctx, int32_t* counts, int32_t* offsets, int3
  * (after a stream synchronisation), rows in routing-position order:
  *   xq u8 E4M3 [P, H], xs fp32 [P, H/128]  (GEMM1 input, P = T*k + n_shared*T)
  *   hq u8 E4M3 [P, I], hs fp32 [P, I/128]  (GEMM2 input)
- * Rows of dropped positions are unspecified.  Any pointer may be NULL. */
+ * (NVFP4 contexts: xq [P, H/2] and hq [P, I/2] packed E2M1, xs / hs the
+ * per-128 scales S.)  Rows of dropped positions are unspecified.  Any
+ * pointer may be NULL. */
 moe_status moe_get_activations(moe_ctx* ctx, uint8_t* xq, float* xs, uint8_t* hq, float* hs, void* stream);
+
+/* moe_get_block_scales -- NVFP4 contexts only (else MOE_ERR_UNSUPPORTED):
+ * the E4M3 block codes of the last call's activations, after a stream
+ * synchronisation, rows in routing-position order: xsc u8 [P, H/16],
+ * hsc u8 [P, I/16].  Either pointer may be NULL.  Debug / test entry point. */
+moe_status moe_get_block_scales(moe_ctx* ctx, uint8_t* xsc, uint8_t* hsc, void* stream);
 
 /* moe_get_device_status -- synchronises `stream`, returns MOE_OK,
  * MOE_ERR_TIMEOUT or MOE_ERR_BAD_ROUTING (timeout wins) for all calls since
