@@ -48,9 +48,10 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", type=int, default=1, help="index into synth.CONFIGS")
+    ap.add_argument("--workload", type=int, default=1,
+                    help="index into synth.CONFIGS (0-4), then synth.EXTRA_CONFIGS (5: NVFP4 T=128, 6: NVFP4 T=32)")
     ap.add_argument("--shape", default=None,
-                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4) instead of --workload")
+                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4|nvfp4) instead of --workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -174,10 +175,16 @@ def gpu_uuid(dev):
 
 
 # ---------------------------------------------------------------------------
+WFMT_NAMES = ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32", "nvfp4_e2m1_e4m3_k16"]
+DTYPES = ["fp8_e4m3", "mxfp4_e2m1 x fp8_e4m3", "nvfp4_e2m1 x nvfp4_e2m1"]
+
+
 def weight_bytes_per_expert(L) -> int:
     H, I = L.H, L.I
     if L.wfmt == 0:
         return 2 * I * H + (2 * I // 128) * (H // 128) * 4 + H * I + (H // 128) * (I // 128) * 4
+    if L.wfmt == 2:  # E2M1 nibbles, one E4M3 code per 16, one fp32 global scale per matrix
+        return 2 * I * H // 2 + 2 * I * H // 16 + 4 + H * I // 2 + H * I // 16 + 4
     return 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
 
 
@@ -185,6 +192,8 @@ def gemm1_weight_bytes_per_expert(L) -> int:
     H, I = L.H, L.I
     if L.wfmt == 0:
         return 2 * I * H + (2 * I // 128) * (H // 128) * 4
+    if L.wfmt == 2:
+        return 2 * I * H // 2 + 2 * I * H // 16 + 4
     return 2 * I * H // 2 + 2 * I * H // 32
 
 
@@ -198,7 +207,11 @@ def workload_stats(L, ids_np):
     P = L.T * L.k + L.n_shared * L.T
     wbytes = n_exp * weight_bytes_per_expert(L)
     flops = 2.0 * P * 3 * L.I * L.H
-    g1 = n_exp * gemm1_weight_bytes_per_expert(L) + P * L.H + P * (L.H // 128) * 4 + P * L.I + P * (L.I // 128) * 4
+    if L.wfmt == 2:  # activations in and out as NVFP4: nibbles, block codes, per-128 scales
+        act = P * (L.H // 2 + L.H // 16 + (L.H // 128) * 4 + L.I // 2 + L.I // 16 + (L.I // 128) * 4)
+    else:
+        act = P * L.H + P * (L.H // 128) * 4 + P * L.I + P * (L.I // 128) * 4
+    g1 = n_exp * gemm1_weight_bytes_per_expert(L) + act
     return dict(experts_touched=n_exp, weight_bytes=wbytes, flops=flops, gemm1_bytes=g1, positions=P)
 
 
@@ -207,12 +220,13 @@ def build_layer(args, device):
     if args.shape:
         f = args.shape.split(",")
         T, H, E, k, I = (int(v) for v in f[:5])
-        wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4}[f[5]]
+        wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4, "nvfp4": synth.WFMT_NVFP4}[f[5]]
         nsh = int(f[6]) if len(f) > 6 else 0
         cfg = dict(name=f"custom_T{T}_H{H}_E{E}_k{k}_I{I}_{f[5]}" + ("_shared" if nsh else ""), T=T, H=H, E=E,
                    k=k, I=I, wfmt=wfmt, routing="uniform", n_shared=nsh)
         return cfg, synth.make_layer(cfg, 2000, device=device)
-    cfg = synth.CONFIGS[args.workload]
+    allc = synth.CONFIGS + synth.EXTRA_CONFIGS
+    cfg = allc[args.workload]
     L = synth.make_layer(cfg, synth.config_seed(args.workload), device=device)
     return cfg, L
 
@@ -269,6 +283,7 @@ def cpu_baseline_sample(L, n_slots: int):
     idx = torch.tensor(experts, device=L.w13.device)
     pick = lambda a: a.index_select(0, idx).cpu().numpy()
     w13, s13, w2, s2 = pick(L.w13), pick(L.s13), pick(L.w2), pick(L.s2)
+    gs = dict(g13=pick(L.g13), g2=pick(L.g2)) if L.g13 is not None else {}
     remap = {e: i for i, e in enumerate(experts)}
     toks = sorted({t for (t, _) in slots})
     x = synth.bf16_bits(L.x[toks])
@@ -278,7 +293,7 @@ def cpu_baseline_sample(L, n_slots: int):
         ids_s[toks.index(t), j] = remap[int(ids[t, j])]
         w_s[toks.index(t), j] = w[t, j]
     t0 = time.perf_counter()
-    oracle.forward(x, ids_s, w_s, w13, s13, w2, s2, H=L.H, I=L.I, E=len(experts), wfmt=L.wfmt, n_shared=0)
+    oracle.forward(x, ids_s, w_s, w13, s13, w2, s2, H=L.H, I=L.I, E=len(experts), wfmt=L.wfmt, n_shared=0, **gs)
     dt = time.perf_counter() - t0
     nbytes = len(experts) * weight_bytes_per_expert(L)
     return dt, nbytes, len(experts), oracle.num_threads()
@@ -308,7 +323,7 @@ def run_reference(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
         "data": "synthetic (seeded)",
         "config": {"workload": cfg["name"], "T": cfg["T"], "H": cfg["H"], "E": cfg["E"], "k": cfg["k"],
-                   "I": cfg["I"], "wfmt": ["fp8", "mxfp4"][cfg["wfmt"]], "parallelism": "replicas"},
+                   "I": cfg["I"], "wfmt": WFMT_NAMES[cfg["wfmt"]], "parallelism": "replicas"},
         "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle",
                          "sample": "per step one (token, expert) slot of the workload: one expert FFN on one token"},
         "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -379,13 +394,16 @@ def main():
     green = layer.set_green_ctx(args.green_ctx) if args.green_ctx else None
     if L.wfmt == synth.WFMT_MXFP4:
         w13, s13, w2, s2 = L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2)
+    elif L.wfmt == synth.WFMT_NVFP4:
+        w13, s13, w2, s2 = L.w13, moe.pack_nvfp4_scales(L.s13), L.w2, moe.pack_nvfp4_scales(L.s2)
     else:
         w13, s13, w2, s2 = L.w13, L.s13, L.w2, L.s2
+    gsc = dict(g13=L.g13, g2=L.g2) if L.wfmt == synth.WFMT_NVFP4 else {}
     out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step():
-        layer.forward(L.x, L.ids, L.topk_w, w13, s13, w2, s2, out=out, stream=stream)
+        layer.forward(L.x, L.ids, L.topk_w, w13, s13, w2, s2, out=out, stream=stream, **gsc)
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -444,7 +462,7 @@ def main():
             x_d.copy_(x_h, non_blocking=True)
             ids_d.copy_(ids_h, non_blocking=True)
             w_d.copy_(w_h, non_blocking=True)
-            layer.forward(x_d, ids_d, w_d, w13, s13, w2, s2, out=out, stream=stream)
+            layer.forward(x_d, ids_d, w_d, w13, s13, w2, s2, out=out, stream=stream, **gsc)
             out_h.copy_(out, non_blocking=True)
 
         for _ in range(3):
@@ -467,11 +485,14 @@ def main():
     hbm_peak, bf16_peak, peak_src = peaks()
     g1_ms = stage_ms[2]
     g1_gbs = st["gemm1_bytes"] / (g1_ms * 1e-3) / 1e9 if g1_ms > 0 else None
-    # the same launch against the FP8 dense tensor peak (measured bf16 x the nominal FP8/bf16 ratio 2)
+    # the same launch against the dense tensor peak of its operand type (measured
+    # bf16 x the nominal ratio: 2 for FP8, 4 for FP4 x FP4)
     g1_flops = 2.0 * st["positions"] * 2 * L.I * L.H
     g1_tflops = g1_flops / (g1_ms * 1e-3) / 1e12 if g1_ms > 0 else None
-    fp8_peak = 2.0 * bf16_peak
-    roofline = {"kernel": "GEMM1 (grouped GEMM1 + SwiGLU + FP8 requant)", "bound": "hbm",
+    ratio = 4.0 if L.wfmt == synth.WFMT_NVFP4 else 2.0
+    fp8_peak = ratio * bf16_peak
+    req = "NVFP4" if L.wfmt == synth.WFMT_NVFP4 else "FP8"
+    roofline = {"kernel": f"GEMM1 (grouped GEMM1 + SwiGLU + {req} requant)", "bound": "hbm",
                 "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": (g1_gbs / hbm_peak) if g1_gbs else None,
                 "traffic": recorded_traffic(cfg["name"]),
@@ -479,7 +500,8 @@ def main():
                 "peak_source": f"{peak_src} hbm_gbs (copy bandwidth)",
                 "tensor_tflops": g1_tflops, "tensor_peak_tflops": fp8_peak,
                 "tensor_frac": (g1_tflops / fp8_peak) if g1_tflops else None,
-                "tensor_peak_source": f"{peak_src} bf16_tflops x 2 (FP8/bf16 nominal ratio)",
+                "tensor_peak_source": f"{peak_src} bf16_tflops x {ratio:g} ({'FP4' if ratio == 4 else 'FP8'}/bf16 "
+                                      f"nominal ratio)",
                 "launches_timed": ncalls}
 
     if dist:
@@ -499,10 +521,10 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8_e4m3" if L.wfmt == 0 else "mxfp4_e2m1 x fp8_e4m3",
+        "vs_baseline": None, "dtype": DTYPES[L.wfmt],
         "data": "synthetic (seeded: x~N(0,1) bf16, uniform/zipf top-k, weights N(0,0.02) quantised)",
         "config": {"workload": cfg["name"], "T": L.T, "H": L.H, "E": L.E, "k": L.k, "I": L.I,
-                   "wfmt": ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32"][L.wfmt], "n_shared": L.n_shared,
+                   "wfmt": WFMT_NAMES[L.wfmt], "n_shared": L.n_shared,
                    "experts_touched": st["experts_touched"], "weight_bytes_per_step": st["weight_bytes"],
                    "l2": "inputs larger than L2 (weights streamed per step exceed the 126 MB L2); no flush",
                    "parallelism": "replicas" if world > 1 else "single GPU",

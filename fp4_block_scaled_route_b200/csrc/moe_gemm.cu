@@ -45,9 +45,14 @@
 
 namespace moe {
 
-template <int KIND, int BN, int WFMT>
+// NT: 128-row weight tiles per stage and unit.  GEMM1: pairs of a gate and
+// an up tile of the same channels (NT = 2: one 128-channel tile, NT = 4: two
+// neighbouring ones); GEMM2: NT neighbouring 128-row tiles of W2.  More tiles
+// per stage share one token tile, its block-scale copies and one commit.
+template <int KIND, int BN, int WFMT, int NT = (KIND == 1 ? 2 : 1)>
 struct GemmCfg {
-  static constexpr int NA = (KIND == 1) ? 2 : 1;          // weight tiles per stage (gate + up)
+  static constexpr int NA = NT;                           // weight tiles per stage
+  static_assert(KIND != 1 || NT % 2 == 0, "GEMM1 tiles come in gate/up pairs");
   // NVFP4 (WFMT 2): both operands packed E2M1, 64 bytes per row per 128-wide
   // K block, 64-byte swizzle; the block scales of a K block travel with the
   // stage as 512-byte atoms, two per weight tile and two for the token tile
@@ -61,7 +66,10 @@ struct GemmCfg {
   static constexpr int SF_BYTES = NA * SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int KB_MAX = 64;                       // K <= 8192
-  static constexpr int CG = (BN <= 64) ? 1 : BN / 64;     // epilogue column groups
+  // Epilogue column groups (warpgroups, each taking CPT of the BN columns):
+  // two for NVFP4 stages of four tiles, whose per-unit SwiGLU + requant tail
+  // would otherwise stall the MMAs (only NBUF K blocks fit ahead of it).
+  static constexpr int CG = (BN > 64) ? BN / 64 : (NV && NT == 4) ? 2 : 1;
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
   // Warpgroup 0: NPROD TMA producer warps (warp p issues all loads of the
@@ -114,6 +122,7 @@ struct GemmCfg {
   static_assert(STAGES >= 2, "shared memory too small");
   static_assert(USED_COLS <= 512, "TMEM too small");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 64, "BN");
+  static_assert(CPT % 8 == 0, "columns per epilogue thread");
   // NVFP4 token scales: an atom is one box of 32 positions, token n of the
   // tile in row n (TMEM lane n, the atom's first column).
   static_assert(!NV || BN <= 32, "NVFP4 tiles hold at most 32 tokens");
@@ -128,11 +137,11 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int KIND, int BN, int WFMT>
-__global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
+template <int KIND, int BN, int WFMT, int NT>
+__global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmS, const GemmParams p) {
-  using C = GemmCfg<KIND, BN, WFMT>;
+  using C = GemmCfg<KIND, BN, WFMT, NT>;
   constexpr int NA = C::NA, STAGES = C::STAGES, KB_MAX = C::KB_MAX, CPT = C::CPT;
   constexpr bool NV = C::NV;
   extern __shared__ uint8_t smem_raw[];
@@ -167,9 +176,15 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
   const int KB = p.kblocks;
   const int num_tiles = *p.num_tiles;
   const int rows_e = (KIND == 1) ? 2 * p.I : p.H;      // weight rows per expert
-  const int NRT = ((KIND == 1) ? p.I : p.H) / 128;     // row tiles per expert
+  constexpr int CT = (KIND == 1) ? NA / 2 : NA;        // 128-channel output tiles per unit
+  const int NRT = ((KIND == 1) ? p.I : p.H) / 128 / CT;  // units per expert and token tile
   const int RB = rows_e / 128;                          // 128-row scale blocks per expert
   const int total = num_tiles * NRT;
+  // 128-row block (within the expert) of weight tile a of unit row index rt:
+  // GEMM1 tile 2c = gate, 2c + 1 = up of output tile rt * CT + c.
+  auto tile_rb = [&](int rt, int a) {
+    return (KIND == 1) ? (a & 1) * (p.I / 128) + rt * CT + (a >> 1) : rt * CT + a;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) mbar_init(&full[s], 1);
@@ -219,7 +234,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
     // only) weight tile [+ its E8M0 atom], lane 1 the GEMM1 up tile [+ atom],
     // lane NJ-1 the token tile.  Lane 0 waits for the stage and posts the
     // transaction bytes before any lane issues.
-    constexpr int NJ = (KIND == 1) ? 3 : 2;
+    constexpr int NJ = NA + 1;
     const int pr = warp;
     const uint64_t pol_w = policy_evict_first();
     const uint64_t pol_a = policy_evict_last();
@@ -249,8 +264,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       const int rt = C::TILE_MAJOR ? u % NRT : u / num_tiles, ti = C::TILE_MAJOR ? u / NRT : u % num_tiles;
       const int4 tile = p.tiles[ti];
       const int e = tile.x, p0 = tile.y;
-      const int row0 = e * rows_e + rt * 128;
-      const int row = (KIND == 1 && lane == 1) ? row0 + p.I : row0;  // gate / up / GEMM2 weight rows
+      const int row = e * rows_e + tile_rb(rt, lane < NA ? lane : 0) * 128;  // this lane's weight tile
       for (int kb = 0; kb < KB; ++kb, ++it) {
         if (it % C::NPROD != pr) continue;
         const int stage = it % STAGES;
@@ -330,6 +344,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
                                    : sdesc_k_sw128(smem_u32(sA + stage * NA * C::A_BYTES));
             const uint64_t bd = NV ? sdesc_k_sw64(smem_u32(sB + stage * C::B_BYTES))
                                    : sdesc_k_sw128(smem_u32(sB + stage * C::B_BYTES));
+            constexpr uint32_t ATILE = C::A_BYTES >> 4;  // descriptor step between weight tiles
             if constexpr (NV) {
               // Scale atoms of this K block, smem -> TMEM (columns of buffer
               // buf): per weight tile a, atoms of K steps 0 and 1 at sfa + 8a
@@ -353,20 +368,17 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
               cp_atom(sfb + 4, sfs + NA * 1024 + 512);
               constexpr uint32_t idesc = idesc_mxf4nvf4(128, BN);
 #pragma unroll
-              for (int ks = 0; ks < 2; ++ks) {
-                mma_mxf4nvf4(d0, ad + 2 * ks, bd + 2 * ks, idesc, sfa + ks * 4, sfb + ks * 4, ks > 0);
-                if constexpr (KIND == 1)
-                  mma_mxf4nvf4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * ks, bd + 2 * ks, idesc, sfa + 8 + ks * 4,
+              for (int ks = 0; ks < 2; ++ks)
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+                  mma_mxf4nvf4(d0 + a * BN, ad + a * ATILE + 2 * ks, bd + 2 * ks, idesc, sfa + a * 8 + ks * 4,
                                sfb + ks * 4, ks > 0);
-              }
             } else if constexpr (WFMT == 0) {
               constexpr uint32_t idesc = idesc_f8f6f4(128, BN, AF, 0);
 #pragma unroll
-              for (int kk = 0; kk < 4; ++kk) {
-                mma_f8f6f4(d0, ad + 2 * kk, bd + 2 * kk, idesc, kk > 0);
-                if constexpr (KIND == 1)
-                  mma_f8f6f4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * kk, bd + 2 * kk, idesc, kk > 0);
-              }
+              for (int kk = 0; kk < 4; ++kk)
+#pragma unroll
+                for (int a = 0; a < NA; ++a) mma_f8f6f4(d0 + a * BN, ad + a * ATILE + 2 * kk, bd + 2 * kk, idesc, kk > 0);
             } else {
               // scale factors of this K block: smem atoms -> TMEM (parity buf)
               const uint32_t sfa = tmem + C::SFA_COL + buf * (NA * 4);  // per accumulator buffer
@@ -383,9 +395,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint32_t idesc = idesc_mxf8f6f4(128, BN, AF, 0, kk, 0);
-                mma_mxf8f6f4(d0, ad + 2 * kk, bd + 2 * kk, idesc, sfa, sfb, kk > 0);
-                if constexpr (KIND == 1)
-                  mma_mxf8f6f4(d0 + BN, ad + (C::A_BYTES >> 4) + 2 * kk, bd + 2 * kk, idesc, sfa + 4, sfb, kk > 0);
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+                  mma_mxf8f6f4(d0 + a * BN, ad + a * ATILE + 2 * kk, bd + 2 * kk, idesc, sfa + a * 4, sfb, kk > 0);
               }
             }
             mma_commit(&mdone[mit % NMD]);
@@ -440,8 +452,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       if constexpr (WFMT == 0) {
         if (etid < NA * KB) {
           const int a = etid / KB, kb = etid % KB;
-          const int rb = (a == 0) ? rtn : p.I / 128 + rtn;
-          pw = p.wscale[((size_t)tile_n.x * RB + rb) * KB + kb];
+          pw = p.wscale[((size_t)tile_n.x * RB + tile_rb(rtn, a)) * KB + kb];
         }
       }
       if constexpr (NV) {
@@ -473,8 +484,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         if constexpr (WFMT == 0) {
           for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
             const int a = i / KB, kb = i % KB;
-            const int rb = (a == 0) ? rt : p.I / 128 + rt;
-            wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + rb) * KB + kb];
+            wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + tile_rb(rt, a)) * KB + kb];
           }
         }
         if constexpr (NV) {
@@ -497,12 +507,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
       named_sync(1, C::EPI_THREADS);
       const int un = u + gridDim.x;
 
-      float acc0[CPT], acc1[CPT];
+      float acc[NA][CPT];  // one fp32 accumulator row per weight tile
 #pragma unroll
-      for (int c = 0; c < CPT; ++c) {
-        acc0[c] = 0.0f;
-        acc1[c] = 0.0f;
-      }
+      for (int a = 0; a < NA; ++a)
+#pragma unroll
+        for (int c = 0; c < CPT; ++c) acc[a][c] = 0.0f;
       // Combined scale of K block kb per tile column, shared by all 128 rows:
       // cs[kb & 1][a][j] = activation scale (column j, kb) x weight block
       // scale (tile a, kb) (MXFP4: the activation scale alone; NVFP4: x the
@@ -528,47 +537,51 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         if (ok) {
           tc_fence_after();
           const uint32_t tb = tmem + ((uint32_t)(q * 32) << 16) + buf * (NA * BN) + cg * CPT;
-          const float* csg = cs + (kb & 1) * (NA * BN) + cg * CPT;
-          const float* csu = csg + (NA - 1) * BN;
+          const float* csb = cs + (kb & 1) * (NA * BN) + cg * CPT;
           // acc += D_kb * combined scale, two columns per paired fp32 FMA
           if constexpr (KIND == 1 && CPT >= 64) {
-            // wide tiles: gate and up chunks one after the other, so only 16
-            // loaded values are live next to the 2 x CPT accumulators
+            // wide tiles (one gate/up pair): gate and up chunks one after the
+            // other, so only 16 loaded values are live next to the 2 x CPT
+            // accumulators
+            static_assert(NA == 2, "wide tiles use one gate/up pair");
 #pragma unroll
             for (int c0 = 0; c0 < 2 * CPT; c0 += 16) {
               float d[16];
-              const bool up = c0 >= CPT;
-              const int cc = up ? c0 - CPT : c0;
-              tmem_ld16(tb + (up ? BN : 0) + cc, d);
+              const int a = c0 >= CPT ? 1 : 0;
+              const int cc = c0 - a * CPT;
+              tmem_ld16(tb + a * BN + cc, d);
               tmem_wait_ld();
               if (c0 + 16 >= 2 * CPT) {
                 tc_fence_before();
                 mbar_arrive(&tempty[buf]);
               }
-              const float2* s2 = reinterpret_cast<const float2*>((up ? csu : csg) + cc);
-              float2* a2 = reinterpret_cast<float2*>(up ? acc1 + cc : acc0 + cc);
+              const float2* s2 = reinterpret_cast<const float2*>(csb + a * BN + cc);
+              float2* a2 = reinterpret_cast<float2*>(&acc[a][cc]);
 #pragma unroll
               for (int i = 0; i < 8; ++i) a2[i] = __ffma2_rn(make_float2(d[2 * i], d[2 * i + 1]), s2[i], a2[i]);
             }
           } else {
+            constexpr int LD = CPT >= 16 ? 16 : 8;  // columns per TMEM load
 #pragma unroll
-            for (int c0 = 0; c0 < CPT; c0 += 16) {
-              float d0[16], d1[16];
-              tmem_ld16(tb + c0, d0);
-              if constexpr (KIND == 1) tmem_ld16(tb + BN + c0, d1);
+            for (int c0 = 0; c0 < CPT; c0 += LD) {
+              float d[NA][LD];
+#pragma unroll
+              for (int a = 0; a < NA; ++a) {
+                if constexpr (LD == 16) tmem_ld16(tb + a * BN + c0, d[a]);
+                else tmem_ld8(tb + a * BN + c0, d[a]);
+              }
               tmem_wait_ld();
-              if (c0 + 16 >= CPT) {
+              if (c0 + LD >= CPT) {
                 tc_fence_before();
                 mbar_arrive(&tempty[buf]);
               }
-              const float2* sg = reinterpret_cast<const float2*>(csg + c0);
-              const float2* su = reinterpret_cast<const float2*>(csu + c0);
-              float2* g2 = reinterpret_cast<float2*>(acc0 + c0);
-              float2* u2 = reinterpret_cast<float2*>(acc1 + c0);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                g2[i] = __ffma2_rn(make_float2(d0[2 * i], d0[2 * i + 1]), sg[i], g2[i]);
-                if constexpr (KIND == 1) u2[i] = __ffma2_rn(make_float2(d1[2 * i], d1[2 * i + 1]), su[i], u2[i]);
+              for (int a = 0; a < NA; ++a) {
+                const float2* s2 = reinterpret_cast<const float2*>(csb + a * BN + c0);
+                float2* a2 = reinterpret_cast<float2*>(&acc[a][c0]);
+#pragma unroll
+                for (int i = 0; i < LD / 2; ++i)
+                  a2[i] = __ffma2_rn(make_float2(d[a][2 * i], d[a][2 * i + 1]), s2[i], a2[i]);
               }
             }
           }
@@ -580,92 +593,85 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
         }
       }
 
-      if constexpr (KIND == 1 && NV) {
-        // SwiGLU, then NVFP4 requantisation of each token's 128 channels
-        // (the rule of quant_nvfp4_kernel): lanes 16i .. 16i+15 of a warp
-        // hold one 16-channel block, the tile's four warps one 128 group.
-        float* h = acc0;
-        float a16[CPT];
+      if constexpr (KIND == 1) {
+        // Per gate/up pair (gate rows 0..I-1 of W13, up rows I..2I-1: same
+        // channels): SwiGLU, then requantisation per token over the output
+        // tile's 128 channels -- NVFP4 (the rule of quant_nvfp4_kernel: lanes
+        // 16i .. 16i+15 of a warp hold one 16-channel block, the four warps
+        // one 128 group) or FP8.  h overwrites the gate accumulator in place.
 #pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          const float g = acc0[c];
-          const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
-          h[c] = g * sig * acc1[c];
-          float m = fabsf(h[c]);
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-          a16[c] = m;
-          m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-          if (lane == 0) red[q * BN + cg * CPT + c] = m;
-        }
-        named_sync(1, C::EPI_THREADS);
-        if (ok) {
-          const int ch = rt * 128 + row;
+        for (int pr = 0; pr < NA / 2; ++pr) {
+          float* h = acc[2 * pr];
+          const float* up = acc[2 * pr + 1];
+          const int ct = rt * CT + pr;  // output channel tile
+          const int ch = ct * 128 + row;
+          float a16[NV ? CPT : 1];
 #pragma unroll
           for (int c = 0; c < CPT; ++c) {
-            const int j = cg * CPT + c;
-            const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
-            const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-            const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16[c], 6.0f), sg));
-            const float d = __fmul_rn(e4m3_code_value(code), sg);
-            const uint32_t nib = code ? f32_to_e2m1(__fdiv_rn(h[c], d)) : 0u;
-            // eight neighbouring channels -> one 32-bit word of packed codes
-            uint32_t word = nib << (4 * (lane & 7));
-            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
-            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-            word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-            if (j < nv) {
-              if ((lane & 7) == 0) *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
-              if ((lane & 15) == 0)
-                p.hsc[((size_t)(ch / 64) * p.scale_ld + p0 + j) * 16 + (ch / 16) % 4] = static_cast<uint8_t>(code);
-              if (row == 0) p.hs[(size_t)rt * p.scale_ld + p0 + j] = sg;
+            const float g = h[c];
+            const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+            h[c] = g * sig * up[c];
+            float m = fabsf(h[c]);
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+            if constexpr (NV) a16[c] = m;
+            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+            if (lane == 0) red[q * BN + cg * CPT + c] = m;
+          }
+          named_sync(1, C::EPI_THREADS);
+          if (ok) {
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+              const int j = cg * CPT + c;
+              const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
+              if constexpr (NV) {
+                const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16[c], 6.0f), sg));
+                const float d = __fmul_rn(e4m3_code_value(code), sg);
+                const uint32_t nib = code ? f32_to_e2m1(__fdiv_rn(h[c], d)) : 0u;
+                // eight neighbouring channels -> one 32-bit word of packed codes
+                uint32_t word = nib << (4 * (lane & 7));
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+                if (j < nv) {
+                  if ((lane & 7) == 0)
+                    *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
+                  if ((lane & 15) == 0)
+                    p.hsc[((size_t)(ch / 64) * p.scale_ld + p0 + j) * 16 + (ch / 16) % 4] =
+                        static_cast<uint8_t>(code);
+                  if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sg;
+                }
+              } else {
+                const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+                if (j < nv) {
+                  p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[c], sc)));
+                  if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sc;
+                }
+              }
             }
           }
-        }
-      } else if constexpr (KIND == 1) {
-        // SwiGLU (gate rows 0..I-1 of W13, up rows I..2I-1: same channel),
-        // then FP8 requantisation per token over the tile's 128 channels.
-        float* h = acc0;  // h overwrites the gate accumulator in place
-#pragma unroll
-        for (int c = 0; c < CPT; ++c) {
-          const float g = acc0[c];
-          const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
-          h[c] = g * sig * acc1[c];
-          float m = fabsf(h[c]);
-#pragma unroll
-          for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-          if (lane == 0) red[q * BN + cg * CPT + c] = m;
-        }
-        named_sync(1, C::EPI_THREADS);
-        if (ok) {
-          const int ch = rt * 128 + row;
-#pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            const int j = cg * CPT + c;
-            const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
-            const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-            if (j < nv) {
-              p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[c], sc)));
-              if (row == 0) p.hs[(size_t)rt * p.scale_ld + p0 + j] = sc;
-            }
-          }
+          if (pr + 1 < NA / 2) named_sync(1, C::EPI_THREADS);  // red is reused by the next pair
         }
       } else {
         if (ok) {
-          const int ch = rt * 128 + row;
-          if (p.y_rows) {
-            // unfused combine: keep this position's expert output row
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-              const int j = cg * CPT + c;
-              if (j < nv) p.y_rows[(size_t)(p0 + j) * p.H + ch] = acc0[c];
-            }
-          } else {
-            // fused combine: out_acc[token] += w * y (fp32 reductions in L2)
+          for (int a = 0; a < NA; ++a) {
+            const int ch = (rt * CT + a) * 128 + row;
+            if (p.y_rows) {
+              // unfused combine: keep this position's expert output row
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-              const int j = cg * CPT + c;
-              if (j < nv) atomicAdd(p.out_acc + (size_t)slot_tok[j] * p.H + ch, slot_w[j] * acc0[c]);
+              for (int c = 0; c < CPT; ++c) {
+                const int j = cg * CPT + c;
+                if (j < nv) p.y_rows[(size_t)(p0 + j) * p.H + ch] = acc[a][c];
+              }
+            } else {
+              // fused combine: out_acc[token] += w * y (fp32 reductions in L2)
+#pragma unroll
+              for (int c = 0; c < CPT; ++c) {
+                const int j = cg * CPT + c;
+                if (j < nv) atomicAdd(p.out_acc + (size_t)slot_tok[j] * p.H + ch, slot_w[j] * acc[a][c]);
+              }
             }
           }
         }
@@ -685,17 +691,17 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-template <int KIND, int BN, int WFMT>
+template <int KIND, int BN, int WFMT, int NT>
 static cudaError_t set_attr() {
-  using C = GemmCfg<KIND, BN, WFMT>;
-  return cudaFuncSetAttribute(moe_gemm_kernel<KIND, BN, WFMT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  using C = GemmCfg<KIND, BN, WFMT, NT>;
+  return cudaFuncSetAttribute(moe_gemm_kernel<KIND, BN, WFMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               C::SMEM_BYTES);
 }
 
-template <int KIND, int BN, int WFMT>
+template <int KIND, int BN, int WFMT, int NT = (KIND == 1 ? 2 : 1)>
 static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
                           const GemmParams& p, cudaStream_t s) {
-  using C = GemmCfg<KIND, BN, WFMT>;
+  using C = GemmCfg<KIND, BN, WFMT, NT>;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::THREADS);
@@ -706,13 +712,27 @@ static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT>, ta, tb, ts, p);
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT>, ta, tb, ts, p);
+}
+
+// NVFP4 weight tiles per stage: a stage of two packed 128-row tiles carries
+// only 16 KB of weights, and per stage the tensor pipe also copies the
+// block-scale atoms and commits, which at that size issues slower than HBM
+// delivers.  16-token tiles therefore take four tiles per stage (32 KB)
+// where the channel count divides: GEMM1 two gate/up pairs (I % 256 == 0),
+// GEMM2 four output tiles (H % 512 == 0), else two (H % 256 == 0), else one.
+static int nvfp4_tiles(int kind, int BN, const GemmParams& p) {
+  if (kind == 1) return (BN == 16 && p.I % 256 == 0) ? 4 : 2;
+  if (BN == 16 && p.H % 512 == 0) return 4;
+  return (p.H % 256 == 0) ? 2 : 1;
 }
 
 cudaError_t gemm_setup(int wfmt) {
   cudaError_t e = cudaSuccess;
 #define MOE_SET(K, B, W) \
-  if (e == cudaSuccess) e = set_attr<K, B, W>();
+  if (e == cudaSuccess) e = set_attr<K, B, W, (K == 1 ? 2 : 1)>();
+#define MOE_SET_NT(K, B, W, N) \
+  if (e == cudaSuccess) e = set_attr<K, B, W, N>();
   if (wfmt == 0) {
     MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0)
     MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0)
@@ -721,10 +741,12 @@ cudaError_t gemm_setup(int wfmt) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
     MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
   } else {
-    MOE_SET(1, 16, 2) MOE_SET(1, 32, 2)
-    MOE_SET(2, 16, 2) MOE_SET(2, 32, 2)
+    MOE_SET_NT(1, 16, 2, 4) MOE_SET_NT(1, 16, 2, 2) MOE_SET_NT(1, 32, 2, 2)
+    MOE_SET_NT(2, 16, 2, 4) MOE_SET_NT(2, 16, 2, 2) MOE_SET_NT(2, 16, 2, 1)
+    MOE_SET_NT(2, 32, 2, 2) MOE_SET_NT(2, 32, 2, 1)
   }
 #undef MOE_SET
+#undef MOE_SET_NT
   return e;
 }
 
@@ -744,10 +766,9 @@ cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 64: return launch<1, 64, 1>(grid, tw, tx, tsf, p, s);
     }
   } else {
-    switch (BN) {
-      case 16: return launch<1, 16, 2>(grid, tw, tx, tsf, p, s);
-      case 32: return launch<1, 32, 2>(grid, tw, tx, tsf, p, s);
-    }
+    const int nt = nvfp4_tiles(1, BN, p);
+    if (BN == 16) return nt == 4 ? launch<1, 16, 2, 4>(grid, tw, tx, tsf, p, s) : launch<1, 16, 2, 2>(grid, tw, tx, tsf, p, s);
+    if (BN == 32) return launch<1, 32, 2, 2>(grid, tw, tx, tsf, p, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -768,10 +789,13 @@ cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 64: return launch<2, 64, 1>(grid, tw, th, tsf, p, s);
     }
   } else {
-    switch (BN) {
-      case 16: return launch<2, 16, 2>(grid, tw, th, tsf, p, s);
-      case 32: return launch<2, 32, 2>(grid, tw, th, tsf, p, s);
+    const int nt = nvfp4_tiles(2, BN, p);
+    if (BN == 16) {
+      if (nt == 4) return launch<2, 16, 2, 4>(grid, tw, th, tsf, p, s);
+      if (nt == 2) return launch<2, 16, 2, 2>(grid, tw, th, tsf, p, s);
+      return launch<2, 16, 2, 1>(grid, tw, th, tsf, p, s);
     }
+    if (BN == 32) return nt == 2 ? launch<2, 32, 2, 2>(grid, tw, th, tsf, p, s) : launch<2, 32, 2, 1>(grid, tw, th, tsf, p, s);
   }
   return cudaErrorInvalidValue;
 }
