@@ -50,9 +50,8 @@ struct moe_ctx {
   CUgreenCtx gc_small, gc_large;
   CUstream gs_small, gs_large;
   cudaEvent_t gev_in, gev_disp, gev_done;
-  // fused router (moe_router_topk): fp32 logit accumulators and tile counters
+  // fused router (moe_router_topk): fp32 logit accumulators
   float* rt_logits;
-  int32_t* rt_counters;
   const void* c_wr;
   CUtensorMap tm_wr;
 };
@@ -236,11 +235,10 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_hsc = nvfp4 ? take((size_t)(I / 64) * c->S_pad * 16) : 0;
   const bool want_rows = c->combine_mode == 2;
   const size_t o_rows = want_rows ? take(sizeof(float) * (size_t)c->S_pad * H) : 0;
-  // fused router workspace (E <= 256, E % 4 == 0): logits of every token tile + a counter per tile
+  // fused router workspace (E <= 256, E % 4 == 0): logits of every token tile
   const bool want_router = E <= 256 && E % 4 == 0;
   const size_t rt_tiles = ((size_t)max_T + 127) / 128;
   const size_t o_rt_logits = want_router ? take(sizeof(float) * rt_tiles * 128 * E) : 0;
-  const size_t o_rt_counters = want_router ? take(sizeof(int32_t) * rt_tiles) : 0;
   void* base = nullptr;
   if (cudaMalloc(&base, off) != cudaSuccess) {
     delete c;
@@ -278,7 +276,6 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   }
   c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
   c->rt_logits = want_router ? reinterpret_cast<float*>(b + o_rt_logits) : nullptr;
-  c->rt_counters = want_router ? reinterpret_cast<int32_t*>(b + o_rt_counters) : nullptr;
   if (want_router && moe::router_setup(E) != cudaSuccess) {
     cudaFree(base);
     delete c;
@@ -575,7 +572,7 @@ moe_status moe_router_topk(moe_ctx* c, int T, const void* x, const void* wr, int
   rp.splits = splits;
   rp.wbox_rows = NP;
   rp.tmem_cols = NP <= 32 ? 32 : NP <= 64 ? 64 : NP <= 128 ? 128 : 256;
-  rp.logits = c->rt_logits; rp.counters = c->rt_counters;
+  rp.logits = c->rt_logits;
   rp.ids = topk_ids; rp.w = topk_w; rp.status = c->status;
   if (moe::launch_router(tx, c->tm_wr, rp, s) != cudaSuccess) return MOE_ERR_CUDA;
   return MOE_OK;

@@ -78,7 +78,6 @@ struct RouterParams {
   int wbox_rows;          // rows of one router-weight TMA box (= N)
   int tmem_cols;
   float* logits;          // fp32 [tiles*128, E], zero between calls
-  int32_t* counters;      // [tiles], zero between calls
   int32_t* ids;           // [T, k]
   float* w;               // [T, k]
   int32_t* status;

@@ -1,20 +1,24 @@
 // moe_router.cu -- fused router ("Mega Gate"): the routing GEMM and the MoE
-// routing step in one kernel (DeepGEMM 26/09 news page: the router GEMM and
-// the MoE routing operations fused into a single kernel).
+// routing step behind one call (DeepGEMM 26/09 news page: the router GEMM and
+// the MoE routing operations fused).
 //
 //   logits[t, e] = sum_h x[t, h] * Wr[e, h]      x bf16 [T, H], Wr bf16 [E, H]
 //   ids[t, :]    = the k largest logits of token t, descending, ties to the
 //                  lower expert index
 //   w[t, j]      = softmax over the k chosen logits
 //
-// One launch.  CTA (token tile of 128, K split): TMA streams 64-element K
-// blocks of x and Wr into shared memory, tcgen05.mma kind::f16 (bf16 x bf16,
-// fp32 accumulate; M = 128 tokens, N = E experts) accumulates the CTA's K
-// range in TMEM, and the epilogue adds its partial logits into an fp32 buffer
-// with vector reductions.  The CTA that finishes a tile last (atomic counter;
-// nobody waits for anybody) reads the tile's logits into shared memory, selects
-// and normalises the top k per token (one thread per token), and returns the
-// buffer rows and the counter to zero for the next call.
+// Two kernels, the second a programmatic dependent launch of the first:
+//   router_kernel       CTA (token tile of 128, K split): TMA streams 64-
+//                       element K blocks of x and Wr into shared memory,
+//                       tcgen05.mma kind::f16 (bf16 x bf16, fp32 accumulate;
+//                       M = 128 tokens, N = E experts) accumulates the CTA's
+//                       K range in TMEM, and the epilogue adds its partial
+//                       logits into an fp32 buffer with vector reductions.
+//   router_topk_kernel  one warp per token: top k + softmax from the summed
+//                       logits, then the token's buffer row back to zero for
+//                       the next call.
+// (Selecting in the CTA that finishes a tile last kept one CTA busy with 128
+// tokens while the rest of the GPU idled: 36 us of a 68 us call at T = 128.)
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
@@ -27,7 +31,6 @@ namespace {
 constexpr int kRtStages = 4;
 constexpr int kRtThreads = 192;  // warp 0 TMA, warp 1 MMA + TMEM, warps 2-5 epilogue
 constexpr int kRtA = 128 * 128;  // token tile: 128 rows x 64 bf16
-constexpr int kRtBMax = 256 * 128;
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 accumulate, K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
@@ -53,13 +56,10 @@ __device__ __forceinline__ void rt_drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Top k (k <= 8) of one logit row in a single scan.  Each (value, index)
-// pair becomes one 64-bit key that orders like "larger logit first, then
-// lower index": the float's order-preserving bit pattern in the high word and
-// the complemented index in the low word.  A sorted list of eight keys lives
-// in named registers; an element enters when its key exceeds the k-th entry
-// and moves down the list by plain 64-bit comparisons.  Then the softmax over
-// the chosen logits.
+// Each (value, index) pair becomes one 64-bit key that orders like "larger
+// logit first, then lower index": the float's order-preserving bit pattern in
+// the high word and the complemented index in the low word, so all keys of a
+// row are distinct and plain 64-bit comparisons select.
 __device__ __forceinline__ uint64_t rank_key(float v, int e) {
   const uint32_t b = __float_as_uint(v == 0.0f ? 0.0f : v);  // -0 and +0 tie, as values do
   const uint32_t ord = (b & 0x80000000u) ? ~b : (b | 0x80000000u);  // monotone in v
@@ -73,44 +73,28 @@ __device__ __forceinline__ int key_index(uint64_t key) {
   return static_cast<int>(0xFFFFFFFFu - static_cast<uint32_t>(key));
 }
 
-__device__ __forceinline__ void topk8_row(const float* __restrict__ r, int E, int k, int32_t* ids, float* w) {
-  uint64_t l0 = 0, l1 = 0, l2 = 0, l3 = 0, l4 = 0, l5 = 0, l6 = 0, l7 = 0;  // 0 ranks after every key
-  uint64_t thr = 0;                                                         // key of the k-th entry
-  for (int e = 0; e < E; ++e) {
-    const uint64_t cv = rank_key(r[e], e);
-    if (cv > thr) {
-      // insertion slot = number of entries ranking before cv (the list is
-      // sorted, so these are independent comparisons); entries from the slot
-      // on move down by one
-      const bool g0 = l0 > cv, g1 = l1 > cv, g2 = l2 > cv, g3 = l3 > cv, g4 = l4 > cv, g5 = l5 > cv,
-                 g6 = l6 > cv, g7 = l7 > cv;
-      l7 = g7 ? l7 : (g6 ? cv : l6);
-      l6 = g6 ? l6 : (g5 ? cv : l5);
-      l5 = g5 ? l5 : (g4 ? cv : l4);
-      l4 = g4 ? l4 : (g3 ? cv : l3);
-      l3 = g3 ? l3 : (g2 ? cv : l2);
-      l2 = g2 ? l2 : (g1 ? cv : l1);
-      l1 = g1 ? l1 : (g0 ? cv : l0);
-      l0 = g0 ? l0 : cv;
-      thr = (k == 1) ? l0 : (k == 2) ? l1 : (k == 3) ? l2 : (k == 4) ? l3 : (k == 5) ? l4 : (k == 6) ? l5
-          : (k == 7) ? l6 : l7;
-    }
-  }
-  const uint64_t ls[8] = {l0, l1, l2, l3, l4, l5, l6, l7};
-  const float m = key_value(l0);
-  float z = 0.0f;
+// Top-8 of two lists sorted in descending key order, left in `a` (sorted):
+// the element-wise larger of a[i] and b[7-i] is a bitonic sequence holding
+// exactly the 8 largest keys of both lists, and three half-cleaner stages
+// (distances 4, 2, 1) sort it.  Keys are distinct (the expert index is part
+// of the key), so both partners of an exchange end with the same list.
+__device__ __forceinline__ void merge_top8(uint64_t (&a)[8], const uint64_t (&b)[8]) {
+  uint64_t m[8];
 #pragma unroll
-  for (int s = 0; s < 8; ++s)
-    if (s < k) z += expf(key_value(ls[s]) - m);
+  for (int i = 0; i < 8; ++i) m[i] = a[i] > b[7 - i] ? a[i] : b[7 - i];
 #pragma unroll
-  for (int s = 0; s < 8; ++s)
-    if (s < k) {
-      ids[s] = key_index(ls[s]);
-      w[s] = __fdiv_rn(expf(key_value(ls[s]) - m), z);
-    }
+  for (int d = 4; d > 0; d >>= 1)
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      if ((i & d) == 0) {
+        const uint64_t x = m[i], y = m[i + d];
+        m[i] = x > y ? x : y;
+        m[i + d] = x > y ? y : x;
+      }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) a[i] = m[i];
 }
 
-// k > 8: k scans, each taking the largest logit ordered after the previous pick.
 __device__ void topk_row_scan(const float* __restrict__ r, int E, int k, int32_t* ids, float* w) {
   float pv = 0.0f, m = 0.0f, z = 0.0f;
   int pe = -1;
@@ -147,7 +131,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   const int stage_bytes = kRtA + ((b_bytes + 1023) / 1024) * 1024;
   __shared__ uint64_t full[kRtStages], empty[kRtStages], mma_done;
   __shared__ uint32_t tmem_holder;
-  __shared__ int s_last;
   __shared__ int abort_w;
   volatile int* abort = &abort_w;
 
@@ -174,6 +157,9 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = tmem_holder;
+  // the selection kernel may be scheduled now; it waits for this grid's
+  // completion before it reads the logits
+  griddep_launch_dependents();
 
   if (warp == 0) {
     // TMA: lane 0 the token tile, lane 1 the router weight rows.
@@ -241,46 +227,6 @@ __global__ void __launch_bounds__(kRtThreads, 1)
         }
       }
     }
-    __threadfence();
-    named_sync(1, 128);
-    if (threadIdx.x == 64) s_last = (atomicAdd(p.counters + tile, 1) == p.splits - 1);
-    named_sync(1, 128);
-    if (s_last) {
-      // ---- last CTA of the tile: top-k + softmax per token ----
-      __threadfence();
-      const int nrows = min(128, p.T - t0);
-      const int ld = p.E + 1;  // padded row: conflict-free column reads
-      float* lg = reinterpret_cast<float*>(smem);  // the pipeline stages are idle now
-      const int et = threadIdx.x - 64;
-      // The tile's rows are one contiguous block of nrows * E floats (E % 4 == 0):
-      // float4 loads, several in flight per thread, into padded shared rows;
-      // then a second pass returns the block to zero.
-      const int n4 = nrows * p.E / 4;
-      float4* blk = reinterpret_cast<float4*>(p.logits + (size_t)t0 * p.E);
-#pragma unroll 16
-      for (int i = et; i < n4; i += 128) {
-        const float4 v = __ldcg(blk + i);
-        const int idx = i * 4, r = idx / p.E, c = idx - r * p.E;
-        float* d = lg + r * ld + c;
-        d[0] = v.x;
-        d[1] = v.y;
-        d[2] = v.z;
-        d[3] = v.w;
-      }
-      named_sync(1, 128);
-#pragma unroll 16
-      for (int i = et; i < n4; i += 128) blk[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-      // one thread per token
-      if (et < nrows) {
-        const float* r = lg + et * ld;
-        const size_t o = (size_t)(t0 + et) * p.k;
-        if (p.k <= 8)
-          topk8_row(r, p.E, p.k, p.ids + o, p.w + o);
-        else
-          topk_row_scan(r, p.E, p.k, p.ids + o, p.w + o);
-      }
-      if (threadIdx.x == 64) p.counters[tile] = 0;
-    }
   }
 
   tc_fence_before();
@@ -292,12 +238,77 @@ __global__ void __launch_bounds__(kRtThreads, 1)
   if (threadIdx.x == 0 && *abort) atomicOr(p.status, DEV_TIMEOUT);
 }
 
+// Eight keys sorted in descending order (bitonic network: blocks of 2, 4, 8).
+__device__ __forceinline__ void sort8_desc(uint64_t (&m)[8]) {
+#pragma unroll
+  for (int kk = 2; kk <= 8; kk <<= 1)
+#pragma unroll
+    for (int j = kk >> 1; j > 0; j >>= 1)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int l = i ^ j;
+        if (l > i) {
+          const uint64_t x = m[i], y = m[l];
+          const bool desc = (i & kk) == 0;
+          const bool keep = desc ? x > y : x < y;
+          m[i] = keep ? x : y;
+          m[l] = keep ? y : x;
+        }
+      }
+}
+
+// One warp per token t < T: lane l takes logits l, l + 32, ... (E <= 256, at
+// most 8), sorts its keys, and five shuffle rounds merge the lanes' lists
+// into the token's top 8; lane 0 writes the k ids and softmax weights (k > 8:
+// lane 0 scans the row k times).  The warp then zeroes the row.
+constexpr int kTopkWarps = 4;
+__global__ void __launch_bounds__(32 * kTopkWarps) router_topk_kernel(const RouterParams p) {
+  griddep_wait();  // the logits are complete once the GEMM grid has finished
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kTopkWarps + warp;
+  if (t >= p.T) return;  // warp-uniform
+  float* row = p.logits + (size_t)t * p.E;
+  int32_t* ids = p.ids + (size_t)t * p.k;
+  float* w = p.w + (size_t)t * p.k;
+  if (p.k <= 8) {
+    uint64_t ls[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      ls[j] = (e < p.E) ? rank_key(__ldcg(row + e), e) : 0;  // 0 ranks after every key
+    }
+    sort8_desc(ls);
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      uint64_t other[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) other[i] = __shfl_xor_sync(0xFFFFFFFFu, ls[i], off);
+      merge_top8(ls, other);
+    }
+    if (lane == 0) {
+      const float m = key_value(ls[0]);
+      float z = 0.0f;
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        if (s < p.k) z += expf(key_value(ls[s]) - m);
+#pragma unroll
+      for (int s = 0; s < 8; ++s)
+        if (s < p.k) {
+          ids[s] = key_index(ls[s]);
+          w[s] = __fdiv_rn(expf(key_value(ls[s]) - m), z);
+        }
+    }
+  } else if (lane == 0) {
+    topk_row_scan(row, p.E, p.k, ids, w);
+  }
+  __syncwarp();
+  for (int e = lane * 4; e < p.E; e += 128) *reinterpret_cast<float4*>(row + e) = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
 size_t router_smem_bytes(int E) {
   const int NP = (E + 15) / 16 * 16;
   const int stage = kRtA + ((NP * 128 + 1023) / 1024) * 1024;
-  const size_t pipe = (size_t)kRtStages * stage;
-  const size_t topk = (size_t)128 * (E + 1) * 4;
-  return 1024 + (pipe > topk ? pipe : topk);
+  return 1024 + (size_t)kRtStages * stage;
 }
 
 cudaError_t router_setup(int E) {
@@ -307,7 +318,18 @@ cudaError_t router_setup(int E) {
 cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, const RouterParams& p, cudaStream_t s) {
   const int tiles = (p.T + 127) / 128;
   router_kernel<<<tiles * p.splits, kRtThreads, router_smem_bytes(p.E), s>>>(tx, tw, p);
-  return cudaGetLastError();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((p.T + kTopkWarps - 1) / kTopkWarps));
+  cfg.blockDim = dim3(32 * kTopkWarps);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, router_topk_kernel, p);
 }
 
 }  // namespace moe

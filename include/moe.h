@@ -208,10 +208,11 @@ moe_status moe_set_fault_injection(moe_ctx* ctx, int mode);
  *   x        device bf16 [T, H] row-major (16-byte aligned)
  *   wr       device bf16 [E, H] row-major router weights (16-byte aligned)
  *   topk_ids device int32 [T, k] (output), topk_w device fp32 [T, k] (output)
- * H, E, k and the largest T are the context's.  One kernel launch on
- * `stream`, asynchronous, no host synchronisation; the context's router
- * workspace is left zeroed for the next call, so calls on one context must be
- * stream-ordered.  The fp32 partial logits of the K splits are added with
+ * H, E, k and the largest T are the context's.  Two kernels on `stream`:
+ * the logits GEMM, then (a programmatic dependent launch) one warp per token
+ * for the top k and the softmax.  Asynchronous, no host synchronisation; the
+ * context's router workspace is left zeroed for the next call, so calls on
+ * one context must be stream-ordered.  The fp32 partial logits of the K splits are added with
  * atomic reductions, so a logit can differ from call to call in its last bits
  * and a near-tie between the k-th and (k+1)-th expert can resolve either way.
  * Returns MOE_ERR_UNSUPPORTED when E > 256 or E is not a multiple of 4,
