@@ -736,6 +736,7 @@ cudaError_t gemm_setup(int wfmt) {
   if (wfmt == 0) {
     MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0)
     MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0)
+    MOE_SET_NT(2, 16, 0, 2) MOE_SET_NT(2, 32, 0, 2)
     if (e == cudaSuccess) e = gemm_tm_setup();
   } else if (wfmt == 1) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
@@ -776,9 +777,12 @@ cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
 cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, const CUtensorMap& th,
                          const CUtensorMap& tsf, const GemmParams& p, cudaStream_t s) {
   if (wfmt == 0) {
+    // decode tiles: two 128-row W2 tiles per stage and unit (one token tile,
+    // one commit and one unit prologue / combine per 256 output channels)
+    const bool two = p.H % 256 == 0;
     switch (BN) {
-      case 16: return launch<2, 16, 0>(grid, tw, th, tsf, p, s);
-      case 32: return launch<2, 32, 0>(grid, tw, th, tsf, p, s);
+      case 16: return two ? launch<2, 16, 0, 2>(grid, tw, th, tsf, p, s) : launch<2, 16, 0>(grid, tw, th, tsf, p, s);
+      case 32: return two ? launch<2, 32, 0, 2>(grid, tw, th, tsf, p, s) : launch<2, 32, 0>(grid, tw, th, tsf, p, s);
       case 64: return launch<2, 64, 0>(grid, tw, th, tsf, p, s);
       case 128: return launch_gemm2_tm(grid, tw, th, p, s);
     }
