@@ -31,9 +31,8 @@ NVFP4 (the same nibbles, one E4M3 scale per 16 elements along K and one fp32
 global scale per expert matrix: g = amax / (448 * 6), block scale
 e4m3(amax16 / 6 / g), element e2m1(w / (block scale * g))).
 
-The NVFP4 decode workload (not one of the table's rows) is row 2's shape
-with NVFP4 weights: ``decode_T128_H7168_E256_k8_I2048_nvfp4`` in
-``EXTRA_CONFIGS``.
+The NVFP4 decode workloads and an MXFP4-weights-and-activations workload
+(not rows of the table) use the decode shapes, in ``EXTRA_CONFIGS``.
 """
 from __future__ import annotations
 
@@ -46,6 +45,7 @@ import torch
 WFMT_FP8 = 0
 WFMT_MXFP4 = 1
 WFMT_NVFP4 = 2
+WFMT_MXFP4_A4 = 3  # MXFP4 weights (the WFMT_MXFP4 bytes) with MXFP4 activations
 
 CONFIGS = [
     dict(name="tiny_T4_H256_E8_k2_I128_fp8", T=4, H=256, E=8, k=2, I=128,
@@ -67,6 +67,8 @@ EXTRA_CONFIGS = [
          wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
     dict(name="decode_T32_H7168_E256_k8_I2048_nvfp4", T=32, H=7168, E=256, k=8, I=2048,
          wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
+    dict(name="decode_T128_H7168_E256_k8_I2048_mxfp4_a4", T=128, H=7168, E=256, k=8, I=2048,
+         wfmt=WFMT_MXFP4_A4, routing="uniform", n_shared=0),
 ]
 
 
@@ -225,8 +227,9 @@ def make_layer(cfg: dict, seed: int, device="cpu", T: Optional[int] = None,
         w13, s13, g13 = make_weights_nvfp4(E + nsh, 2 * I, H, gen, device)
         w2, s2, g2 = make_weights_nvfp4(E + nsh, H, I, gen, device)
     else:
-        w13, s13 = make_weights(E + nsh, 2 * I, H, wfmt, gen, device)
-        w2, s2 = make_weights(E + nsh, H, I, wfmt, gen, device)
+        wf = WFMT_MXFP4 if wfmt == WFMT_MXFP4_A4 else wfmt  # the same MXFP4 weight bytes
+        w13, s13 = make_weights(E + nsh, 2 * I, H, wf, gen, device)
+        w2, s2 = make_weights(E + nsh, H, I, wf, gen, device)
     return Layer(T, H, I, E, k, wfmt, nsh, x, torch.from_numpy(ids).to(device),
                  torch.from_numpy(w).to(device), w13, s13, w2, s2, g13, g2)
 

@@ -27,6 +27,7 @@ _lib = None
 WFMT_FP8 = 0
 WFMT_MXFP4 = 1
 WFMT_NVFP4 = 2
+WFMT_MXFP4_A4 = 3
 
 
 def build(force: bool = False) -> str:
@@ -82,6 +83,10 @@ def lib() -> ctypes.CDLL:
             L.orc_quant_row_nvfp4.argtypes = [ctypes.c_int, vp, vp, vp, vp]
             L.orc_quant_act_nvfp4.restype = None
             L.orc_quant_act_nvfp4.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp, vp]
+            L.orc_quant_row_mxfp4.restype = None
+            L.orc_quant_row_mxfp4.argtypes = [ctypes.c_int, vp, vp, vp]
+            L.orc_quant_act_mxfp4.restype = None
+            L.orc_quant_act_mxfp4.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
             L.orc_forward.restype = ctypes.c_int
             L.orc_forward.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 13
             L.orc_forward_ex.restype = ctypes.c_int
@@ -207,6 +212,26 @@ def quant_act_nvfp4(x_bf16_bits: np.ndarray):
     return xq, xsc, xs
 
 
+def quant_row_mxfp4(v: np.ndarray):
+    """fp32 row [K] -> (q packed uint8 [K/2], E8M0 codes uint8 [K/32])."""
+    v = _c(v, np.float32)
+    (K,) = v.shape
+    q = np.empty(K // 2, np.uint8)
+    sc = np.empty(K // 32, np.uint8)
+    lib().orc_quant_row_mxfp4(K, _p(v), _p(q), _p(sc))
+    return q, sc
+
+
+def quant_act_mxfp4(x_bf16_bits: np.ndarray):
+    """x as bf16 bits [T,H] -> (xq packed [T,H/2], xsc E8M0 [T,H/32])."""
+    x = _c(x_bf16_bits, np.uint16)
+    T, H = x.shape
+    xq = np.empty((T, H // 2), np.uint8)
+    xsc = np.empty((T, H // 32), np.uint8)
+    lib().orc_quant_act_mxfp4(T, H, _p(x), _p(xq), _p(xsc))
+    return xq, xsc
+
+
 def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
             n_shared=0, token_mask=None, debug=False, g13=None, g2=None):
     """Whole layer on the CPU.
@@ -244,12 +269,14 @@ def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
     out_bf16 = np.zeros((T, H), np.uint16)
     dbg = {}
     if debug:
-        cw = 2 if nv else 1
+        a4 = wfmt in (WFMT_NVFP4, WFMT_MXFP4_A4)
+        cw = 2 if a4 else 1
         dbg = dict(xq=np.zeros((T, H // cw), np.uint8), xs=np.zeros((T, H // 128), np.float32),
                    hq=np.zeros((max(P, 1), I // cw), np.uint8),
                    hs=np.zeros((max(P, 1), I // 128), np.float32))
-        if nv:
-            dbg.update(xsc=np.zeros((T, H // 16), np.uint8), hsc=np.zeros((max(P, 1), I // 16), np.uint8))
+        if a4:
+            bs = 16 if nv else 32
+            dbg.update(xsc=np.zeros((T, H // bs), np.uint8), hsc=np.zeros((max(P, 1), I // bs), np.uint8))
     rc = lib().orc_forward_ex(ctypes.byref(d), _p(x), _p(ids), _p(topk_w), _p(w13), _p(s13), _p(g13),
                               _p(w2), _p(s2), _p(g2), _p(mask), _p(out_f32), _p(out_bf16),
                               _p(dbg.get("xq")), _p(dbg.get("xsc")), _p(dbg.get("xs")),

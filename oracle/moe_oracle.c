@@ -271,6 +271,67 @@ void orc_quant_act_nvfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* 
   free(row);
 }
 
+/* MXFP4 activations (OCP MX v1.0 conversion with E2M1 elements): shared
+ * exponent X = floor(log2(amax32)) - 2, clamped to the E8M0 range [-127, 127]
+ * (an all-zero block: X = -127); elements e2m1(v / 2^X).  floor(log2 a) of a
+ * positive float is read from its exponent field (normal) or its leading one
+ * (subnormal), so it is exact. */
+static int floor_log2f(float a) {
+  uint32_t u;
+  int e;
+  memcpy(&u, &a, 4);
+  e = (int)((u >> 23) & 0xFF);
+  if (e != 0) return e - 127;
+  {
+    uint32_t m = u & 0x7FFFFFu;
+    int p = 22;
+    while (p >= 0 && !(m & (1u << p))) --p;
+    return p - 149; /* subnormal: 2^-149 * m */
+  }
+}
+
+void orc_quant_row_mxfp4(int K, const float* v, uint8_t* q, uint8_t* sc) {
+  for (int c = 0; c < K / 2; ++c) q[c] = 0;
+  for (int g = 0; g < K / 32; ++g) {
+    const float* vg = v + (size_t)g * 32;
+    float amax = 0.0f;
+    int X;
+    float s;
+    for (int c = 0; c < 32; ++c) {
+      float a = fabsf(vg[c]);
+      if (a > amax) amax = a;
+    }
+    X = (amax == 0.0f) ? -127 : floor_log2f(amax) - 2;
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    sc[g] = (uint8_t)(X + 127);
+    s = ldexpf(1.0f, X); /* exact: 2^-127 is a subnormal float */
+    for (int c = 0; c < 32; ++c) {
+      const int col = g * 32 + c;
+      uint8_t nib = orc_e2m1_encode(vg[c] / s);
+      q[col / 2] |= (uint8_t)((col % 2 == 0) ? nib : (nib << 4));
+    }
+  }
+}
+
+void orc_quant_act_mxfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc) {
+  float* row = (float*)malloc(sizeof(float) * (size_t)H);
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < H; ++c) row[c] = orc_bf16_decode(x[(size_t)t * H + c]);
+    orc_quant_row_mxfp4(H, row, xq + (size_t)t * (H / 2), xsc + (size_t)t * (H / 32));
+  }
+  free(row);
+}
+
+/* One MXFP4 row (packed E2M1 + E8M0 codes per 32) -> element x 2^X values
+ * (exact in fp32). */
+static void decode_mxfp4_row(const uint8_t* q, const uint8_t* sc, int K, float* out) {
+  for (int c = 0; c < K; ++c) {
+    uint8_t nib = (c % 2 == 0) ? (q[c / 2] & 0xF) : (q[c / 2] >> 4);
+    out[c] = orc_e2m1_decode(nib) * orc_e8m0_decode(sc[c / 32]);
+  }
+}
+
 /* One NVFP4 row (packed E2M1 + E4M3 block codes) -> element x block scale
  * values (exact in fp32: 2 x 4 significant bits); the second-level scale is
  * applied per K block by the caller. */
@@ -338,6 +399,9 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   const int S = T * k, NG = E + nsh, P = S + nsh * T;
   const int HB = H / 128, IB = I / 128;
   const int nv = (wfmt == ORC_WFMT_NVFP4);
+  const int mx4 = (wfmt == ORC_WFMT_MXFP4_A4);      /* MXFP4 weights and MXFP4 activations */
+  const int a4 = nv || mx4;                          /* 4-bit activations */
+  const int wsc = mx4 ? ORC_WFMT_MXFP4 : wfmt;       /* weight decoding */
   const uint8_t* w13 = (const uint8_t*)w13v;
   const uint8_t* w2 = (const uint8_t*)w2v;
   /* per-expert strides in bytes (weights) */
@@ -345,16 +409,18 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   const size_t w2_e = (wfmt == ORC_WFMT_FP8) ? (size_t)H * I : (size_t)H * I / 2;
   const size_t w13_r = (wfmt == ORC_WFMT_FP8) ? (size_t)H : (size_t)H / 2;
   const size_t w2_r = (wfmt == ORC_WFMT_FP8) ? (size_t)I : (size_t)I / 2;
-  /* activation codes per row: E4M3 bytes, or packed E2M1 + E4M3 block codes */
-  const size_t xq_r = nv ? (size_t)H / 2 : (size_t)H;
-  const size_t hq_r = nv ? (size_t)I / 2 : (size_t)I;
+  /* activation codes per row: E4M3 bytes, or packed E2M1 (+ block codes) */
+  const size_t xq_r = a4 ? (size_t)H / 2 : (size_t)H;
+  const size_t hq_r = a4 ? (size_t)I / 2 : (size_t)I;
+  const int bs = mx4 ? 32 : 16;                      /* 4-bit activations: elements per block code */
   int32_t *counts, *offsets, *perm, *inv, *cidx;
   uint8_t *xq, *xsc = NULL;
   float *xs, *xd, *Y, e4m3_tab[256];
   int dropped, ncomp = 0;
 
   if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || H % 128 || I % 128 ||
-      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4 && wfmt != ORC_WFMT_NVFP4) || nsh < 0 || nsh > 1 ||
+      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4 && wfmt != ORC_WFMT_NVFP4 && !mx4) || nsh < 0 ||
+      nsh > 1 ||
       (nv && (!g13 || !g2)))
     return -1;
   if (T == 0) return 0;
@@ -378,6 +444,13 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     for (int t = 0; t < T; ++t)
       decode_nvfp4_row(xq + (size_t)t * xq_r, xsc + (size_t)t * (H / 16), H, xd + (size_t)t * H);
     if (dbg_xsc) memcpy(dbg_xsc, xsc, (size_t)T * (H / 16));
+  } else if (mx4) {
+    xsc = (uint8_t*)malloc((size_t)T * (H / 32));
+    orc_quant_act_mxfp4(T, H, x, xq, xsc);
+    for (size_t i = 0; i < (size_t)T * HB; ++i) xs[i] = 1.0f;  /* every scale is in the codes */
+    for (int t = 0; t < T; ++t)
+      decode_mxfp4_row(xq + (size_t)t * xq_r, xsc + (size_t)t * (H / 32), H, xd + (size_t)t * H);
+    if (dbg_xsc) memcpy(dbg_xsc, xsc, (size_t)T * (H / 32));
   } else {
     orc_quant_act(T, H, x, xq, xs);
     for (size_t i = 0; i < (size_t)T * H; ++i) xd[i] = e4m3_tab[xq[i]];
@@ -416,7 +489,7 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     hd = (float*)malloc(sizeof(float) * (size_t)n * I);
     hs = (float*)malloc(sizeof(float) * (size_t)n * IB);
     hq = (uint8_t*)malloc((size_t)n * hq_r);
-    hsc = (uint8_t*)malloc((size_t)n * (I / 16));
+    hsc = (uint8_t*)malloc((size_t)n * (I / bs));
 
     /* step 3: GEMM1, G[i][r] for gate rows r < I and up rows r >= I */
 #pragma omp parallel
@@ -437,10 +510,10 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
         } else {
           sr = (const uint8_t*)s13v + ((size_t)g * 2 * I + (size_t)r) * (H / 32);
         }
-        decode_row(wfmt, wr, sr, H, e4m3_tab, wrow);
+        decode_row(wsc, wr, sr, H, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           G[(size_t)i * 2 * I + r] = row_dot(H, xd + (size_t)tok[i] * H, xs + (size_t)tok[i] * HB,
-                                             wrow, wfmt == ORC_WFMT_MXFP4 ? NULL : ws);
+                                             wrow, wsc == ORC_WFMT_MXFP4 ? NULL : ws);
       }
       free(wrow);
       free(ws);
@@ -457,6 +530,11 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
           orc_quant_row_nvfp4(I, h, hqi, hsc + (size_t)i * (I / 16), hs + (size_t)i * IB);
           decode_nvfp4_row(hqi, hsc + (size_t)i * (I / 16), I, hd + (size_t)i * I);
           if (dbg_hsc) memcpy(dbg_hsc + (size_t)pos[i] * (I / 16), hsc + (size_t)i * (I / 16), (size_t)(I / 16));
+        } else if (mx4) {
+          orc_quant_row_mxfp4(I, h, hqi, hsc + (size_t)i * (I / 32));
+          for (int kb = 0; kb < IB; ++kb) hs[(size_t)i * IB + kb] = 1.0f;
+          decode_mxfp4_row(hqi, hsc + (size_t)i * (I / 32), I, hd + (size_t)i * I);
+          if (dbg_hsc) memcpy(dbg_hsc + (size_t)pos[i] * (I / 32), hsc + (size_t)i * (I / 32), (size_t)(I / 32));
         } else {
           orc_quant_row_f32(I, h, hqi, hs + (size_t)i * IB);
           for (int c = 0; c < I; ++c) hd[(size_t)i * I + c] = e4m3_tab[hqi[c]];
@@ -486,10 +564,10 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
         } else {
           sr = (const uint8_t*)s2v + ((size_t)g * H + (size_t)r) * (I / 32);
         }
-        decode_row(wfmt, wr, sr, I, e4m3_tab, wrow);
+        decode_row(wsc, wr, sr, I, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           Y[(size_t)cidx[pos[i]] * H + r] = row_dot(I, hd + (size_t)i * I, hs + (size_t)i * IB,
-                                                    wrow, wfmt == ORC_WFMT_MXFP4 ? NULL : ws);
+                                                    wrow, wsc == ORC_WFMT_MXFP4 ? NULL : ws);
       }
       free(wrow);
       free(ws);

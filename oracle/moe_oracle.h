@@ -39,7 +39,8 @@
  * linearity in the combine weights, zero input) and, for NVFP4, in
  * tests/test_oracle_nvfp4.py (E2M1 rounding against the OCP table by brute
  * force, exact round trips of representable groups, error bounds, the fp64
- * restatement of the layer).
+ * restatement of the layer) and, for MXFP4 activations, in
+ * tests/test_oracle_mxfp4_a4.py.
  */
 #ifndef MOE_ORACLE_H
 #define MOE_ORACLE_H
@@ -50,7 +51,7 @@
 extern "C" {
 #endif
 
-enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1, ORC_WFMT_NVFP4 = 2 };
+enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1, ORC_WFMT_NVFP4 = 2, ORC_WFMT_MXFP4_A4 = 3 };
 
 /* ---- codecs (OCP FP8 / OCP MX v1.0) ---------------------------------- */
 float   orc_e4m3_decode(uint8_t code);          /* exact value, NaN for S.1111.111 */
@@ -95,10 +96,21 @@ void orc_quant_row_f32(int K, const float* v, uint8_t* q, float* s);
 void orc_quant_row_nvfp4(int K, const float* v, uint8_t* q, uint8_t* sc, float* s);
 void orc_quant_act_nvfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc, float* xs);
 
+/* MXFP4 form of steps 2 and 5 (OCP MX v1.0, "MX-compliant" conversion, with
+ * E2M1 elements and an E8M0 shared scale per 32 consecutive elements):
+ *   X = floor(log2(amax32)) - 2 (2 = the largest E2M1 exponent), clamped to
+ *   [-127, 127]; an all-zero block takes X = -127;
+ *   code = X + 127 (E8M0), q = e2m1(v / 2^X)  (round-to-nearest-even,
+ *   saturating at +-6).
+ * One fp32 row of K (multiple of 32) values -> q packed E2M1 [K/2] (element
+ * 2c in the low nibble of byte c) and sc E8M0 codes [K/32]. */
+void orc_quant_row_mxfp4(int K, const float* v, uint8_t* q, uint8_t* sc);
+void orc_quant_act_mxfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc);
+
 /* ---- steps 1-8: the whole layer -------------------------------------- */
 typedef struct {
   int T, H, I, E, k;
-  int wfmt;       /* ORC_WFMT_FP8, ORC_WFMT_MXFP4 or ORC_WFMT_NVFP4 */
+  int wfmt;       /* ORC_WFMT_FP8, ORC_WFMT_MXFP4, ORC_WFMT_NVFP4 or ORC_WFMT_MXFP4_A4 */
   int n_shared;   /* 0 or 1: shared expert stored as expert index E */
 } orc_dims;
 
@@ -120,7 +132,13 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
                 float* out_f32, uint16_t* out_bf16,
                 uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs);
 
-/* All three formats.  For ORC_WFMT_NVFP4 (g13, g2 required; ignored otherwise):
+/* All four formats.  ORC_WFMT_MXFP4_A4 takes the MXFP4 weight layout above
+ * and quantises the activations (x and the SwiGLU output) to MXFP4 with
+ * orc_quant_row_mxfp4; every product is then (element x 2^X) x (element x
+ * 2^X), summed per 128-wide K block in ascending k and the blocks added in
+ * ascending order with no further scale.  Its debug outputs: xq [T, H/2],
+ * xsc [T, H/32]; hq [P, I/2], hsc [P, I/32] (xs / hs unused).
+ * For ORC_WFMT_NVFP4 (g13, g2 required; ignored otherwise):
  *   w13 u8 [NE, 2I, H/2] packed E2M1, s13 u8 E4M3 [NE, 2I, H/16], g13 f32 [NE]
  *   w2  u8 [NE, H, I/2],              s2  u8 E4M3 [NE, H, I/16],  g2  f32 [NE]
  * weight value = e2m1(q) * e4m3(s) * g[expert].  Activations are quantised

@@ -2,7 +2,7 @@
  * (built by tests/test_oracle_sanitizers.py with -fsanitize=address,undefined
  * -fno-sanitize-recover=all, single-threaded).  Every entry point runs on
  * small seeded inputs that include ragged shapes, the shared expert, dropped
- * ids, all three weight formats and the router; any out-of-bounds access, leak or
+ * ids, all four weight formats and the router; any out-of-bounds access, leak or
  * undefined operation aborts with a non-zero exit status. */
 #include <math.h>
 #include <stdint.h>
@@ -91,7 +91,7 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
   uint8_t* hsc = malloc(P * (I / 16) + 1);
   float* hs = malloc(sizeof(float) * (P * (I / 128) + 1));
   orc_dims d = {T, H, I, E, k, wfmt, n_shared};
-  const int dropped = (wfmt == ORC_WFMT_NVFP4)
+  const int dropped = (wfmt == ORC_WFMT_NVFP4 || wfmt == ORC_WFMT_MXFP4_A4)
       ? orc_forward_ex(&d, x, ids, w, w13, s13, g13, w2, s2, g2, NULL, out, outb, xq, xsc, xs, hq, hsc, hs)
       : orc_forward(&d, x, ids, w, w13, s13, w2, s2, NULL, out, outb, xq, xs, hq, hs);
   int ok = dropped == (bad_ids && S > 2 ? 2 : 0) && check_finite(out, (size_t)T * H);
@@ -128,6 +128,7 @@ int main(void) {
   ok &= run_layer(1, 128, 128, 1, 1, ORC_WFMT_MXFP4, 0, 0);
   ok &= run_layer(5, 256, 128, 6, 2, ORC_WFMT_NVFP4, 1, 1);
   ok &= run_layer(2, 384, 256, 3, 3, ORC_WFMT_NVFP4, 0, 0);
+  ok &= run_layer(4, 256, 128, 5, 2, ORC_WFMT_MXFP4_A4, 1, 1);
   ok &= run_router(9, 256, 16, 4);
   ok &= run_router(2, 128, 8, 8);
   uint8_t codes[256];
