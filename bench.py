@@ -49,9 +49,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", type=int, default=1,
-                    help="index into synth.CONFIGS (0-4), then synth.EXTRA_CONFIGS (5: NVFP4 T=128, 6: NVFP4 T=32)")
+                    help="index into synth.CONFIGS (0-4), then synth.EXTRA_CONFIGS (5: NVFP4 T=128, 6: NVFP4 T=32, "
+                         "7: MXFP4 weights and activations T=128)")
     ap.add_argument("--shape", default=None,
-                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4|nvfp4) instead of --workload")
+                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4|nvfp4|mxfp4a4) instead of --workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -175,8 +176,8 @@ def gpu_uuid(dev):
 
 
 # ---------------------------------------------------------------------------
-WFMT_NAMES = ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32", "nvfp4_e2m1_e4m3_k16"]
-DTYPES = ["fp8_e4m3", "mxfp4_e2m1 x fp8_e4m3", "nvfp4_e2m1 x nvfp4_e2m1"]
+WFMT_NAMES = ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32", "nvfp4_e2m1_e4m3_k16", "mxfp4_w4a4_e2m1_e8m0_k32"]
+DTYPES = ["fp8_e4m3", "mxfp4_e2m1 x fp8_e4m3", "nvfp4_e2m1 x nvfp4_e2m1", "mxfp4_e2m1 x mxfp4_e2m1"]
 
 
 def weight_bytes_per_expert(L) -> int:
@@ -209,6 +210,8 @@ def workload_stats(L, ids_np):
     flops = 2.0 * P * 3 * L.I * L.H
     if L.wfmt == 2:  # activations in and out as NVFP4: nibbles, block codes, per-128 scales
         act = P * (L.H // 2 + L.H // 16 + (L.H // 128) * 4 + L.I // 2 + L.I // 16 + (L.I // 128) * 4)
+    elif L.wfmt == 3:  # activations in and out as MXFP4: nibbles and E8M0 codes
+        act = P * (L.H // 2 + L.H // 32 + L.I // 2 + L.I // 32)
     else:
         act = P * L.H + P * (L.H // 128) * 4 + P * L.I + P * (L.I // 128) * 4
     g1 = n_exp * gemm1_weight_bytes_per_expert(L) + act
@@ -220,7 +223,8 @@ def build_layer(args, device):
     if args.shape:
         f = args.shape.split(",")
         T, H, E, k, I = (int(v) for v in f[:5])
-        wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4, "nvfp4": synth.WFMT_NVFP4}[f[5]]
+        wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4, "nvfp4": synth.WFMT_NVFP4,
+                "mxfp4a4": synth.WFMT_MXFP4_A4}[f[5]]
         nsh = int(f[6]) if len(f) > 6 else 0
         cfg = dict(name=f"custom_T{T}_H{H}_E{E}_k{k}_I{I}_{f[5]}" + ("_shared" if nsh else ""), T=T, H=H, E=E,
                    k=k, I=I, wfmt=wfmt, routing="uniform", n_shared=nsh)
@@ -392,7 +396,7 @@ def main():
     st = workload_stats(L, ids_np)
     layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
     green = layer.set_green_ctx(args.green_ctx) if args.green_ctx else None
-    if L.wfmt == synth.WFMT_MXFP4:
+    if L.wfmt in (synth.WFMT_MXFP4, synth.WFMT_MXFP4_A4):
         w13, s13, w2, s2 = L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2)
     elif L.wfmt == synth.WFMT_NVFP4:
         w13, s13, w2, s2 = L.w13, moe.pack_nvfp4_scales(L.s13), L.w2, moe.pack_nvfp4_scales(L.s2)
@@ -489,9 +493,9 @@ def main():
     # bf16 x the nominal ratio: 2 for FP8, 4 for FP4 x FP4)
     g1_flops = 2.0 * st["positions"] * 2 * L.I * L.H
     g1_tflops = g1_flops / (g1_ms * 1e-3) / 1e12 if g1_ms > 0 else None
-    ratio = 4.0 if L.wfmt == synth.WFMT_NVFP4 else 2.0
+    ratio = 4.0 if L.wfmt in (synth.WFMT_NVFP4, synth.WFMT_MXFP4_A4) else 2.0
     fp8_peak = ratio * bf16_peak
-    req = "NVFP4" if L.wfmt == synth.WFMT_NVFP4 else "FP8"
+    req = {synth.WFMT_NVFP4: "NVFP4", synth.WFMT_MXFP4_A4: "MXFP4"}.get(L.wfmt, "FP8")
     roofline = {"kernel": f"GEMM1 (grouped GEMM1 + SwiGLU + {req} requant)", "bound": "hbm",
                 "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": (g1_gbs / hbm_peak) if g1_gbs else None,

@@ -25,9 +25,10 @@ struct moe_ctx {
   int4* tiles;
   uint8_t *xq, *hq;
   float *xs, *hs, *out_acc;
-  // NVFP4: E4M3 block codes of the activations, [K/64][S_pad][16] bytes
-  // (per 64-column MMA step and position: four codes, then zeros), and their
-  // TMA maps (boxes of 16 bytes x 32 rows = one block-scale atom)
+  // 4-bit activations: block codes, 16-byte entries of four codes then zeros
+  // (NVFP4: E4M3, [K/64][S_pad][16], one entry per 64-column MMA step;
+  // MXFP4 x MXFP4: E8M0, [K/128][S_pad][16], one entry per K block), and
+  // their TMA maps (boxes of 16 bytes x 32 rows = one block-scale atom)
   uint8_t *xsc, *hsc;
   CUtensorMap tm_xsc, tm_hsc;
   // tensor-map cache
@@ -144,7 +145,8 @@ int pick_tile_n(const moe_ctx* c, int T) {
   int bn = avg <= 8 ? 16 : avg <= 20 ? 32 : avg <= 48 ? 64 : 128;
   if (c->tile_n_override) bn = c->tile_n_override;
   if (c->wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 && bn > 64) bn = 64;
-  if (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 && bn > 32) bn = 32;  // token scale atom: 32 tokens
+  if ((c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 || c->wfmt == MOE_WFMT_MXFP4_W4A4) && bn > 32)
+    bn = 32;  // token scale atom: 32 tokens
   return bn;
 }
 
@@ -175,7 +177,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   if (H <= 0 || I <= 0 || E <= 0 || k <= 0 || max_T <= 0 || n_shared < 0) return MOE_ERR_INVALID_ARG;
   if (H % 128 || I % 128 || H > 8192 || I > 8192 || E > 1024 || k > moe::kMaxK || n_shared > 1)
     return MOE_ERR_UNSUPPORTED;
-  if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16)
+  if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 &&
+      wfmt != MOE_WFMT_MXFP4_W4A4)
     return MOE_ERR_UNSUPPORTED;
   if ((long long)max_T * (k + n_shared) > (1LL << 26)) return MOE_ERR_UNSUPPORTED;
 
@@ -206,7 +209,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   if (const char* env = getenv("MOE_GREEN_CTX")) c->gc_sms = atoi(env);  // applied below, once created
   if (const char* env = getenv("MOE_TILE_N")) {
     const int v = atoi(env);
-    if (v == 16 || v == 32 || (v == 64 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) ||
+    if (v == 16 || v == 32 ||
+        (v == 64 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 && wfmt != MOE_WFMT_MXFP4_W4A4) ||
         (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128))
       c->tile_n_override = v;
   }
@@ -230,9 +234,10 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_xs = take(sizeof(float) * (size_t)c->S_pad * HB);
   const size_t o_hs = take(sizeof(float) * (size_t)c->S_pad * IB);
   const size_t o_acc = take(sizeof(float) * (size_t)max_T * H);
-  const bool nvfp4 = wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16;
-  const size_t o_xsc = nvfp4 ? take((size_t)(H / 64) * c->S_pad * 16) : 0;
-  const size_t o_hsc = nvfp4 ? take((size_t)(I / 64) * c->S_pad * 16) : 0;
+  const bool a4 = wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 || wfmt == MOE_WFMT_MXFP4_W4A4;  // 4-bit activations
+  const int code_step = (wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) ? 64 : 128;  // K columns per code entry
+  const size_t o_xsc = a4 ? take((size_t)(H / code_step) * c->S_pad * 16) : 0;
+  const size_t o_hsc = a4 ? take((size_t)(I / code_step) * c->S_pad * 16) : 0;
   const bool want_rows = c->combine_mode == 2;
   const size_t o_rows = want_rows ? take(sizeof(float) * (size_t)c->S_pad * H) : 0;
   // fused router workspace (E <= 256, E % 4 == 0): logits of every token tile
@@ -264,12 +269,14 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->xs = reinterpret_cast<float*>(b + o_xs);
   c->hs = reinterpret_cast<float*>(b + o_hs);
   c->out_acc = reinterpret_cast<float*>(b + o_acc);
-  c->xsc = nvfp4 ? reinterpret_cast<uint8_t*>(b + o_xsc) : nullptr;
-  c->hsc = nvfp4 ? reinterpret_cast<uint8_t*>(b + o_hsc) : nullptr;
-  if (nvfp4 && (!make_map(&c->tm_xsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xsc, 16, (uint64_t)(H / 64) * c->S_pad, 16,
-                          32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-                !make_map(&c->tm_hsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hsc, 16, (uint64_t)(I / 64) * c->S_pad, 16,
-                          32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16, CU_TENSOR_MAP_SWIZZLE_NONE))) {
+  c->xsc = a4 ? reinterpret_cast<uint8_t*>(b + o_xsc) : nullptr;
+  c->hsc = a4 ? reinterpret_cast<uint8_t*>(b + o_hsc) : nullptr;
+  if (a4 && (!make_map(&c->tm_xsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xsc, 16,
+                       (uint64_t)(H / code_step) * c->S_pad, 16, 32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16,
+                       CU_TENSOR_MAP_SWIZZLE_NONE) ||
+             !make_map(&c->tm_hsc, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hsc, 16,
+                       (uint64_t)(I / code_step) * c->S_pad, 16, 32, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 16,
+                       CU_TENSOR_MAP_SWIZZLE_NONE))) {
     cudaFree(base);
     delete c;
     return MOE_ERR_CUDA;
@@ -380,6 +387,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
       !aligned(s2, 16) || !aligned(ids, 4) || !aligned(topk_w, 4))
     return MOE_ERR_INVALID_ARG;
   const bool nvfp4 = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16);
+  const bool a4 = nvfp4 || c->wfmt == MOE_WFMT_MXFP4_W4A4;  // 4-bit activations, packed operands
   if (nvfp4 && (!g13 || !g2 || !aligned(g13, 4) || !aligned(g2, 4))) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = c->H, I = c->I, NE = c->NG;
@@ -402,7 +410,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   if (w13 != c->c_w13) {
     const bool ok = fp8 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H, (uint64_t)NE * 2 * I, H, 128,
                                    wpromo)
-                    : nvfp4 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H / 2, (uint64_t)NE * 2 * I,
+                    : a4 ? make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_UINT8, w13, H / 2, (uint64_t)NE * 2 * I,
                                        H / 2, 128, wpromo, 64, sw64)
                         : make_map(&c->tm_w13, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w13, H, (uint64_t)NE * 2 * I,
                                    H / 2, 128, wpromo);
@@ -415,7 +423,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   if (w2 != c->c_w2) {
     const bool ok = fp8 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I, (uint64_t)NE * H, I, 128,
                                    wpromo)
-                    : nvfp4 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I / 2, (uint64_t)NE * H, I / 2,
+                    : a4 ? make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_UINT8, w2, I / 2, (uint64_t)NE * H, I / 2,
                                        128, wpromo, 64, sw64)
                         : make_map(&c->tm_w2, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, w2, I, (uint64_t)NE * H, I / 2,
                                    128, wpromo);
@@ -426,7 +434,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
     c->c_w2 = w2;
   }
   if (BN != c->c_bn) {
-    const bool ok = nvfp4
+    const bool ok = a4
         ? make_map(&c->tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H / 2, c->S_pad, H / 2, BN,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B, 64, sw64) &&
               make_map(&c->tm_hq, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->hq, I / 2, c->S_pad, I / 2, BN,
@@ -470,8 +478,10 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   qp.out_acc = rows ? nullptr : c->out_acc;
   qp.xsc = c->xsc;
   mark(MOE_STAGE_QUANT);
-  if ((nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp) : moe::launch_quant(qp, s_disp)) != cudaSuccess)
-    return MOE_ERR_CUDA;
+  const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)
+                         : a4  ? moe::launch_quant_mxfp4(qp, s_disp)
+                               : moe::launch_quant(qp, s_disp);
+  if (qe != cudaSuccess) return MOE_ERR_CUDA;
   if (green) {
     if (cudaEventRecord(c->gev_disp, s_disp) != cudaSuccess || cudaStreamWaitEvent(s_gemm, c->gev_disp, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
@@ -490,9 +500,9 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   g.inject = c->inject;
   g.wglobal = g13;
   g.hsc = c->hsc;
-  // the token block-code maps exist for NVFP4 only; the other formats ignore the argument
-  const CUtensorMap& tsx = nvfp4 ? c->tm_xsc : c->tm_xq;
-  const CUtensorMap& tsh = nvfp4 ? c->tm_hsc : c->tm_hq;
+  // the token block-code maps exist for 4-bit activations only; the other formats ignore the argument
+  const CUtensorMap& tsx = a4 ? c->tm_xsc : c->tm_xq;
+  const CUtensorMap& tsh = a4 ? c->tm_hsc : c->tm_hq;
   mark(MOE_STAGE_GEMM1);
   if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -611,7 +621,7 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
   cudaError_t e = cudaSuccess;
-  const size_t cw = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) ? 2 : 1;  // codes per byte
+  const size_t cw = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 || c->wfmt == MOE_WFMT_MXFP4_W4A4) ? 2 : 1;  // codes per byte
   if (xq && P && e == cudaSuccess) e = cudaMemcpy(xq, c->xq, P * c->H / cw, cudaMemcpyDefault);
   if (hq && P && e == cudaSuccess) e = cudaMemcpy(hq, c->hq, P * c->I / cw, cudaMemcpyDefault);
   // The scales are stored K-block major on the device ([K/128][S_pad]); the
@@ -645,14 +655,16 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
 
 moe_status moe_get_block_scales(moe_ctx* c, uint8_t* xsc, uint8_t* hsc, void* stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
-  if (c->wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_UNSUPPORTED;
+  if (c->wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 && c->wfmt != MOE_WFMT_MXFP4_W4A4) return MOE_ERR_UNSUPPORTED;
+  const int code_step = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) ? 64 : 128;  // K columns per 4-code entry
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
   const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
   cudaError_t e = cudaSuccess;
-  // device [K/64][S_pad][16] (four codes per step and position) -> caller [P][K/16]
+  // device [K/code_step][S_pad][16] (four codes per entry and position) ->
+  // caller [P][4 K/code_step] (NVFP4 [P][K/16], MXFP4 [P][K/32])
   auto gather = [&](uint8_t* dst, const uint8_t* src, int K) {
     if (!dst || !P || e != cudaSuccess) return;
-    const size_t steps = (size_t)K / 64;
+    const size_t steps = (size_t)K / code_step;
     uint8_t* tmp = new (std::nothrow) uint8_t[steps * P * 4];
     uint8_t* out = new (std::nothrow) uint8_t[steps * P * 4];
     if (!tmp || !out) {

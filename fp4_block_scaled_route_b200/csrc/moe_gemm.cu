@@ -57,19 +57,25 @@ struct GemmCfg {
   // K block, 64-byte swizzle; the block scales of a K block travel with the
   // stage as 512-byte atoms, two per weight tile and two for the token tile
   // (one per K = 64 MMA step each).
+  // MXFP4 x MXFP4 (WFMT 3): the same packed operands with E8M0 scales per
+  // 32, one 512-byte atom per weight tile and one for the token tile per K
+  // block (its two K = 64 steps use scale bytes 0-1 and 2-3); every scale is
+  // applied by the MMA.
   static constexpr bool NV = WFMT == 2;
-  static constexpr int KBYTES = NV ? 64 : 128;            // smem bytes per row per K block
+  static constexpr bool MXA = WFMT == 3;
+  static constexpr bool P4 = NV || MXA;                   // packed E2M1 on both operands
+  static constexpr int KBYTES = P4 ? 64 : 128;            // smem bytes per row per K block
   static constexpr int A_BYTES = 128 * KBYTES;            // FP8 / E2M1 padded to 8 bits: 128 B rows
   static constexpr int B_BYTES = BN * KBYTES;
-  static constexpr int SFA_BYTES = (WFMT == 1) ? 512 : NV ? 1024 : 0;  // per weight tile
-  static constexpr int SFB_BYTES = NV ? 1024 : 0;
+  static constexpr int SFA_BYTES = (WFMT == 1 || MXA) ? 512 : NV ? 1024 : 0;  // per weight tile
+  static constexpr int SFB_BYTES = NV ? 1024 : MXA ? 512 : 0;
   static constexpr int SF_BYTES = NA * SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int KB_MAX = 64;                       // K <= 8192
   // Epilogue column groups (warpgroups, each taking CPT of the BN columns):
-  // two for NVFP4 stages of four tiles, whose per-unit SwiGLU + requant tail
+  // two for 4-bit-activation stages of four tiles, whose per-unit SwiGLU + requant tail
   // would otherwise stall the MMAs (only NBUF K blocks fit ahead of it).
-  static constexpr int CG = (BN > 64) ? BN / 64 : (NV && NT == 4) ? 2 : 1;
+  static constexpr int CG = (BN > 64) ? BN / 64 : (P4 && NT == 4) ? 2 : 1;
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
   // Warpgroup 0: NPROD TMA producer warps (warp p issues all loads of the
@@ -92,7 +98,7 @@ struct GemmCfg {
   static constexpr int MMA_WARP = NPROD;  // first MMA warp; allocates TMEM
   static constexpr int EPI_WARP0 = NPROD + NMMA;
   static constexpr int THREADS = 32 * EPI_WARP0 + EPI_THREADS;
-  static constexpr int MAX_STAGES = NV ? 24 : 12;
+  static constexpr int MAX_STAGES = P4 ? 24 : 12;
   // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
   // the promoting epilogue (short K steps would otherwise be latency bound).
   static constexpr int NBUF_RAW = 256 / (NA * BN);
@@ -112,7 +118,8 @@ struct GemmCfg {
   static constexpr int SFA_PER_BUF = NV ? NA * 8 : NA * 4;
   static constexpr int SFA_COL = ACC_COLS;
   static constexpr int SFB_COL = SFA_COL + NBUF * SFA_PER_BUF;
-  static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : NV ? SFB_COL + NBUF * 8 : ACC_COLS;
+  static constexpr int SFB_PER_BUF = NV ? 8 : 4;
+  static constexpr int USED_COLS = (WFMT == 1) ? SFB_COL + 4 : P4 ? SFB_COL + NBUF * SFB_PER_BUF : ACC_COLS;
   static constexpr int TMEM_COLS = USED_COLS <= 32 ? 32 : USED_COLS <= 64 ? 64 : USED_COLS <= 128 ? 128
                                  : USED_COLS <= 256 ? 256 : 512;
   // Transaction bytes per stage: a packed-E2M1 weight tile moves 64 bytes per
@@ -125,7 +132,7 @@ struct GemmCfg {
   static_assert(CPT % 8 == 0, "columns per epilogue thread");
   // NVFP4 token scales: an atom is one box of 32 positions, token n of the
   // tile in row n (TMEM lane n, the atom's first column).
-  static_assert(!NV || BN <= 32, "NVFP4 tiles hold at most 32 tokens");
+  static_assert(!P4 || BN <= 32, "4-bit activation tiles hold at most 32 tokens");
 };
 
 // Bounded wait that ignores the abort word (used to drain in-flight copies
@@ -144,6 +151,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
   using C = GemmCfg<KIND, BN, WFMT, NT>;
   constexpr int NA = C::NA, STAGES = C::STAGES, KB_MAX = C::KB_MAX, CPT = C::CPT;
   constexpr bool NV = C::NV;
+  constexpr bool MXA = C::MXA;
+  constexpr bool P4 = C::P4;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
@@ -197,7 +206,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA);
     tma_prefetch_map(&tmB);
-    if constexpr (NV) tma_prefetch_map(&tmS);
+    if constexpr (P4) tma_prefetch_map(&tmS);
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(tmem_holder, C::TMEM_COLS);
@@ -258,6 +267,8 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
         tma_load_2d(&tmS, &full[st], dst, 0, (2 * kb) * p.scale_ld + p0, pol_a);
         tma_load_2d(&tmS, &full[st], dst + 512, 0, (2 * kb + 1) * p.scale_ld + p0, pol_a);
       }
+      if constexpr (MXA)
+        tma_load_2d(&tmS, &full[st], sSF + st * C::SF_BYTES + NA * C::SFA_BYTES, 0, kb * p.scale_ld + p0, pol_a);
     };
     int it = 0;
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
@@ -292,7 +303,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
           __syncwarp();
           if (lane < NJ - 1) {
             tma_load_2d(&tmA, &full[stage], sA + (stage * NA + lane) * C::A_BYTES, kb * C::KBYTES, row, pol_w);
-            if constexpr (WFMT == 1 || NV) {
+            if constexpr (WFMT == 1 || P4) {
               // the K block's block-scale atoms of these 128 rows (packed layout)
               const uint8_t* sf = reinterpret_cast<const uint8_t*>(p.wscale);
               bulk_load(sSF + stage * C::SF_BYTES + lane * C::SFA_BYTES,
@@ -340,9 +351,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
           tc_fence_after();
           if (lane == 0) {
             const uint32_t d0 = tmem + buf * (NA * BN);
-            const uint64_t ad = NV ? sdesc_k_sw64(smem_u32(sA + stage * NA * C::A_BYTES))
+            const uint64_t ad = P4 ? sdesc_k_sw64(smem_u32(sA + stage * NA * C::A_BYTES))
                                    : sdesc_k_sw128(smem_u32(sA + stage * NA * C::A_BYTES));
-            const uint64_t bd = NV ? sdesc_k_sw64(smem_u32(sB + stage * C::B_BYTES))
+            const uint64_t bd = P4 ? sdesc_k_sw64(smem_u32(sB + stage * C::B_BYTES))
                                    : sdesc_k_sw128(smem_u32(sB + stage * C::B_BYTES));
             constexpr uint32_t ATILE = C::A_BYTES >> 4;  // descriptor step between weight tiles
             if constexpr (NV) {
@@ -350,7 +361,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
               // buf): per weight tile a, atoms of K steps 0 and 1 at sfa + 8a
               // and sfa + 8a + 4; the token atoms at sfb and sfb + 4.
               const uint32_t sfa = tmem + C::SFA_COL + buf * C::SFA_PER_BUF;
-              const uint32_t sfb = tmem + C::SFB_COL + buf * 8;
+              const uint32_t sfb = tmem + C::SFB_COL + buf * C::SFB_PER_BUF;
               uint8_t* sfs = sSF + stage * C::SF_BYTES;
               auto cp_atom = [&](uint32_t taddr, const uint8_t* src) {
                 uint64_t sd = 0;
@@ -373,6 +384,30 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
                 for (int a = 0; a < NA; ++a)
                   mma_mxf4nvf4(d0 + a * BN, ad + a * ATILE + 2 * ks, bd + 2 * ks, idesc, sfa + a * 8 + ks * 4,
                                sfb + ks * 4, ks > 0);
+            } else if constexpr (MXA) {
+              // scale atoms of this K block, smem -> TMEM: weight tile a at
+              // sfa + 4a, the token tile at sfb; K step ks uses scale bytes
+              // 2ks and 2ks + 1 of each row's column (scale id 2ks)
+              const uint32_t sfa = tmem + C::SFA_COL + buf * C::SFA_PER_BUF;
+              const uint32_t sfb = tmem + C::SFB_COL + buf * C::SFB_PER_BUF;
+              uint8_t* sfs = sSF + stage * C::SF_BYTES;
+              auto cp_atom = [&](uint32_t taddr, const uint8_t* src) {
+                uint64_t sd = 0;
+                sd |= static_cast<uint64_t>((smem_u32(src) & 0x3FFFFu) >> 4);
+                sd |= static_cast<uint64_t>(128 >> 4) << 32;  // 8 rows x 16 bytes per core group
+                sd |= static_cast<uint64_t>(1) << 46;
+                tmem_cp_32x128b_warpx4(taddr, sd);
+              };
+#pragma unroll
+              for (int a = 0; a < NA; ++a) cp_atom(sfa + a * 4, sfs + a * 512);
+              cp_atom(sfb, sfs + NA * 512);
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks) {
+                const uint32_t idesc = idesc_mxf4(128, BN, 2 * ks, 2 * ks);
+#pragma unroll
+                for (int a = 0; a < NA; ++a)
+                  mma_mxf4(d0 + a * BN, ad + a * ATILE + 2 * ks, bd + 2 * ks, idesc, sfa + a * 4, sfb, ks > 0);
+              }
             } else if constexpr (WFMT == 0) {
               constexpr uint32_t idesc = idesc_f8f6f4(128, BN, AF, 0);
 #pragma unroll
@@ -444,10 +479,13 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     auto pref_scales = [&](int un) {
       if (!have_next) return;
       const int rtn = unit_rt(un);
+      (void)rtn;
+      if constexpr (!MXA) {
 #pragma unroll
-      for (int r = 0; r < NPA; ++r) {
-        const int i = etid + r * C::EPI_THREADS;
-        pa[r] = (i < BN * KB) ? p.ascale[(size_t)(i / BN) * p.scale_ld + tile_n.y + (i % BN)] : 0.0f;
+        for (int r = 0; r < NPA; ++r) {
+          const int i = etid + r * C::EPI_THREADS;
+          pa[r] = (i < BN * KB) ? p.ascale[(size_t)(i / BN) * p.scale_ld + tile_n.y + (i % BN)] : 0.0f;
+        }
       }
       if constexpr (WFMT == 0) {
         if (etid < NA * KB) {
@@ -465,10 +503,12 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
       const int4 tile = from_regs ? tile_n : p.tiles[ti];
       const int e = tile.x, p0 = tile.y, nv = tile.z;
       if (from_regs) {
+        if constexpr (!MXA) {
 #pragma unroll
-        for (int r = 0; r < NPA; ++r) {
-          const int i = etid + r * C::EPI_THREADS;
-          if (i < BN * KB) asc[i] = pa[r];
+          for (int r = 0; r < NPA; ++r) {
+            const int i = etid + r * C::EPI_THREADS;
+            if (i < BN * KB) asc[i] = pa[r];
+          }
         }
         if constexpr (WFMT == 0) {
           if (etid < NA * KB) wsc[(etid / KB) * KB_MAX + etid % KB] = pw;
@@ -477,9 +517,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
           if (etid == 0) wsc[0] = pw;
         }
       } else {
-        for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
-          const int kb = i / BN, j = i % BN;
-          asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
+        if constexpr (!MXA) {
+          for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
+            const int kb = i / BN, j = i % BN;
+            asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
+          }
         }
         if constexpr (WFMT == 0) {
           for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
@@ -523,6 +565,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
           const int a = i / BN, j = i - (i / BN) * BN;
           dst[i] = (WFMT == 0) ? asc[kb * BN + j] * wsc[a * KB_MAX + kb]
                    : NV        ? asc[kb * BN + j] * wsc[0]
+                   : MXA       ? 1.0f  // every scale was applied by the MMA
                                : asc[kb * BN + j];
         }
       };
@@ -605,6 +648,40 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
           const float* up = acc[2 * pr + 1];
           const int ct = rt * CT + pr;  // output channel tile
           const int ch = ct * 128 + row;
+          if constexpr (MXA) {
+            // MXFP4 requantisation (the rule of quant_mxfp4_kernel): a 32-
+            // channel block is one warp, so its amax is a warp reduction and
+            // lane 0 writes the block's E8M0 code (byte q of the tile's entry)
+#pragma unroll
+            for (int c = 0; c < CPT; ++c) {
+              const float g = h[c];
+              const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+              h[c] = g * sig * up[c];
+            }
+            if (ok) {
+#pragma unroll
+              for (int c = 0; c < CPT; ++c) {
+                const int j = cg * CPT + c;
+                float m = fabsf(h[c]);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+                float sc;
+                const int X = mx_e2m1_exponent(m, &sc);
+                const uint32_t nib = f32_to_e2m1(__fdiv_rn(h[c], sc));
+                uint32_t word = nib << (4 * (lane & 7));
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+                if (j < nv) {
+                  if ((lane & 7) == 0)
+                    *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
+                  if (lane == 0)
+                    p.hsc[((size_t)ct * p.scale_ld + p0 + j) * 16 + q] = static_cast<uint8_t>(X + 127);
+                }
+              }
+            }
+            continue;
+          }
           float a16[NV ? CPT : 1];
 #pragma unroll
           for (int c = 0; c < CPT; ++c) {
@@ -715,13 +792,14 @@ static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb
   return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT>, ta, tb, ts, p);
 }
 
-// NVFP4 weight tiles per stage: a stage of two packed 128-row tiles carries
+// Weight tiles per stage with 4-bit activations (NVFP4, MXFP4 x MXFP4): a
+// stage of two packed 128-row tiles carries
 // only 16 KB of weights, and per stage the tensor pipe also copies the
 // block-scale atoms and commits, which at that size issues slower than HBM
 // delivers.  16-token tiles therefore take four tiles per stage (32 KB)
 // where the channel count divides: GEMM1 two gate/up pairs (I % 256 == 0),
 // GEMM2 four output tiles (H % 512 == 0), else two (H % 256 == 0), else one.
-static int nvfp4_tiles(int kind, int BN, const GemmParams& p) {
+static int fp4_tiles(int kind, int BN, const GemmParams& p) {
   if (kind == 1) return (BN == 16 && p.I % 256 == 0) ? 4 : 2;
   if (BN == 16 && p.H % 512 == 0) return 4;
   return (p.H % 256 == 0) ? 2 : 1;
@@ -741,10 +819,14 @@ cudaError_t gemm_setup(int wfmt) {
   } else if (wfmt == 1) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
     MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
-  } else {
+  } else if (wfmt == 2) {
     MOE_SET_NT(1, 16, 2, 4) MOE_SET_NT(1, 16, 2, 2) MOE_SET_NT(1, 32, 2, 2)
     MOE_SET_NT(2, 16, 2, 4) MOE_SET_NT(2, 16, 2, 2) MOE_SET_NT(2, 16, 2, 1)
     MOE_SET_NT(2, 32, 2, 2) MOE_SET_NT(2, 32, 2, 1)
+  } else {
+    MOE_SET_NT(1, 16, 3, 4) MOE_SET_NT(1, 16, 3, 2) MOE_SET_NT(1, 32, 3, 2)
+    MOE_SET_NT(2, 16, 3, 4) MOE_SET_NT(2, 16, 3, 2) MOE_SET_NT(2, 16, 3, 1)
+    MOE_SET_NT(2, 32, 3, 2) MOE_SET_NT(2, 32, 3, 1)
   }
 #undef MOE_SET
 #undef MOE_SET_NT
@@ -766,10 +848,14 @@ cudaError_t launch_gemm1(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 32: return launch<1, 32, 1>(grid, tw, tx, tsf, p, s);
       case 64: return launch<1, 64, 1>(grid, tw, tx, tsf, p, s);
     }
-  } else {
-    const int nt = nvfp4_tiles(1, BN, p);
+  } else if (wfmt == 2) {
+    const int nt = fp4_tiles(1, BN, p);
     if (BN == 16) return nt == 4 ? launch<1, 16, 2, 4>(grid, tw, tx, tsf, p, s) : launch<1, 16, 2, 2>(grid, tw, tx, tsf, p, s);
     if (BN == 32) return launch<1, 32, 2, 2>(grid, tw, tx, tsf, p, s);
+  } else {
+    const int nt = fp4_tiles(1, BN, p);
+    if (BN == 16) return nt == 4 ? launch<1, 16, 3, 4>(grid, tw, tx, tsf, p, s) : launch<1, 16, 3, 2>(grid, tw, tx, tsf, p, s);
+    if (BN == 32) return launch<1, 32, 3, 2>(grid, tw, tx, tsf, p, s);
   }
   return cudaErrorInvalidValue;
 }
@@ -792,14 +878,22 @@ cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 32: return launch<2, 32, 1>(grid, tw, th, tsf, p, s);
       case 64: return launch<2, 64, 1>(grid, tw, th, tsf, p, s);
     }
-  } else {
-    const int nt = nvfp4_tiles(2, BN, p);
+  } else if (wfmt == 2) {
+    const int nt = fp4_tiles(2, BN, p);
     if (BN == 16) {
       if (nt == 4) return launch<2, 16, 2, 4>(grid, tw, th, tsf, p, s);
       if (nt == 2) return launch<2, 16, 2, 2>(grid, tw, th, tsf, p, s);
       return launch<2, 16, 2, 1>(grid, tw, th, tsf, p, s);
     }
     if (BN == 32) return nt == 2 ? launch<2, 32, 2, 2>(grid, tw, th, tsf, p, s) : launch<2, 32, 2, 1>(grid, tw, th, tsf, p, s);
+  } else {
+    const int nt = fp4_tiles(2, BN, p);
+    if (BN == 16) {
+      if (nt == 4) return launch<2, 16, 3, 4>(grid, tw, th, tsf, p, s);
+      if (nt == 2) return launch<2, 16, 3, 2>(grid, tw, th, tsf, p, s);
+      return launch<2, 16, 3, 1>(grid, tw, th, tsf, p, s);
+    }
+    if (BN == 32) return nt == 2 ? launch<2, 32, 3, 2>(grid, tw, th, tsf, p, s) : launch<2, 32, 3, 1>(grid, tw, th, tsf, p, s);
   }
   return cudaErrorInvalidValue;
 }

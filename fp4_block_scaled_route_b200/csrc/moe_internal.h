@@ -32,11 +32,14 @@ struct QuantParams {
   float* xs;              // [H/128, xs_ld]    K-block major: one row of position scales per K block
   int xs_ld;              // = S_pad
   float* out_acc;         // [T, H] zeroed here (null: not needed)
-  // NVFP4 activations (quant_nvfp4_kernel): xq holds packed E2M1 [S_pad, H/2]
-  // and xsc the E4M3 block codes as [H/64][xs_ld][16] bytes: per 64-column
-  // MMA step and position, the step's four codes in bytes 0..3 (bytes 4..15
-  // stay zero), so that 32 consecutive positions of one step form a
-  // block-scale atom of the MMA's B operand.
+  // 4-bit activations: xq holds packed E2M1 [S_pad, H/2] and xsc the block
+  // codes in 16-byte entries, four codes in bytes 0..3 (bytes 4..15 stay
+  // zero), so that 32 consecutive positions form a block-scale atom of the
+  // MMA's B operand:
+  //   NVFP4 (quant_nvfp4_kernel): E4M3 codes, [H/64][xs_ld][16], one entry
+  //     per 64-column MMA step;
+  //   MXFP4 (quant_mxfp4_kernel): E8M0 codes, [H/128][xs_ld][16], one entry
+  //     per 128-column K block (its two MMA steps use bytes 0-1 and 2-3).
   uint8_t* xsc;
 };
 
@@ -59,7 +62,7 @@ struct GemmParams {
   // NVFP4: wscale = packed E4M3 block-scale atoms; wglobal = fp32 [NE] global
   // scales; GEMM1 writes hq as packed E2M1 [S_pad, I/2] plus hsc block codes.
   const float* wglobal;
-  uint8_t* hsc;           // GEMM1: E4M3 block codes [I/64][scale_ld][16] (layout of QuantParams::xsc)
+  uint8_t* hsc;           // GEMM1: block codes of hq (layout of QuantParams::xsc for the format)
 };
 
 struct CombineParams {
@@ -91,6 +94,7 @@ size_t route_smem_bytes(int n_groups);
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s);
+cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s);
 cudaError_t gemm_setup(int wfmt);  // raise shared-memory limits once per process
 // tw: weight tiles; tx / th: token tiles.

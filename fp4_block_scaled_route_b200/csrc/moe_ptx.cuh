@@ -183,6 +183,20 @@ __host__ __device__ constexpr uint32_t idesc_mxf4nvf4(int M, int N) {
          | (static_cast<uint32_t>(M >> 4) << 24);    // M / 16
 }
 
+// Instruction descriptor, kind::mxf4.block_scale with E8M0 (UE8M0) scales per
+// 32 elements: both operands packed E2M1 (format 1), K-major, dense K = 64,
+// fp32 accumulate.  A K = 64 step uses two scale bytes of its row's 32-bit
+// scale column: bytes (sf_id, sf_id + 1), sf_id 0 or 2.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, int a_sf_id, int b_sf_id) {
+  return (static_cast<uint32_t>(b_sf_id) << 4)       // B scale factor id
+         | (1u << 7)                                 // A format E2M1
+         | (1u << 10)                                // B format E2M1
+         | (static_cast<uint32_t>(N >> 3) << 17)     // N / 8
+         | (1u << 23)                                // scale format UE8M0
+         | (static_cast<uint32_t>(M >> 4) << 24)     // M / 16
+         | (static_cast<uint32_t>(a_sf_id) << 29);   // A scale factor id
+}
+
 __device__ __forceinline__ void mma_f8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                            uint32_t accumulate) {
   asm volatile(
@@ -213,6 +227,18 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, ui
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// One K = 64 step of packed-E2M1 operands with E8M0 scales per 32 elements.
+__device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], p;\n\t}\n" ::"r"(
           d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
@@ -328,6 +354,17 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
 __device__ __forceinline__ float e4m3_code_value(uint32_t code) {
   const uint32_t e = (code >> 3) & 0xFu, m = code & 7u;
   return e ? __uint_as_float(((e + 120u) << 23) | (m << 20)) : static_cast<float>(m) * 0.001953125f;
+}
+
+// MXFP4 shared exponent of a block with maximum magnitude amax (OCP MX v1.0
+// with E2M1 elements): X = floor(log2 amax) - 2, clamped to [-127, 127], and
+// -127 for amax = 0 or a subnormal amax (whose floor(log2) is below -126).
+// Returns X; *scale = 2^X exactly (2^-127 is a subnormal float).
+__device__ __forceinline__ int mx_e2m1_exponent(float amax, float* scale) {
+  const int ef = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);  // amax >= 0
+  const int X = ef == 0 ? -127 : max(ef - 129, -127);
+  *scale = X >= -126 ? __uint_as_float(static_cast<uint32_t>(X + 127) << 23) : __uint_as_float(0x00400000u);
+  return X;
 }
 
 // fp32 -> E2M1 code (low nibble), round-to-nearest-even, saturating to +-6;

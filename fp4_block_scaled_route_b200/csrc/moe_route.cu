@@ -284,6 +284,67 @@ cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
+// MXFP4 form of step 2, for MXFP4 weights with MXFP4 activations (OCP MX
+// v1.0 conversion with E2M1 elements): per 32 columns X = floor(log2 amax) - 2
+// clamped to [-127, 127] (-127 for an all-zero block), code X + 127 (E8M0),
+// elements e2m1(v / 2^X).  Same grid as quant_kernel; a lane holds 4
+// consecutive columns, so a 32-column block is 8 lanes and the 128-column
+// K block is the warp.  Outputs per routed position: packed codes and the
+// K block's four E8M0 codes as one 32-bit word (layout of QuantParams::xsc).
+__global__ void __launch_bounds__(kQuantThreads) quant_mxfp4_kernel(QuantParams p) {
+  griddep_launch_dependents();
+  const int t = blockIdx.x;
+  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  __shared__ int rows[kMaxK + 1];
+  __shared__ int nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j < p.k; ++j) {
+      const int r = p.inv[t * p.k + j];
+      if (r >= 0) rows[n++] = r;
+    }
+    if (p.n_shared) rows[n++] = p.inv[S + t];
+    nrows = n;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xr = p.x + (size_t)t * H;
+  for (int g = warp; g < HB; g += kQuantThreads / 32) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    float f[4];
+    f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
+    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
+    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float a32 = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+    a32 = fmaxf(a32, __shfl_xor_sync(0xFFFFFFFFu, a32, 1));
+    a32 = fmaxf(a32, __shfl_xor_sync(0xFFFFFFFFu, a32, 2));
+    a32 = fmaxf(a32, __shfl_xor_sync(0xFFFFFFFFu, a32, 4));
+    float sc;
+    const int X = mx_e2m1_exponent(a32, &sc);
+    const uint32_t packed =
+        f32x4_to_e2m1x4(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc), __fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc));
+    // the K block's four codes into one word (lane 0)
+    uint32_t word = ((lane & 7) == 0) ? static_cast<uint32_t>(X + 127) << (8 * (lane >> 3)) : 0u;
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 8);
+    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 16);
+    for (int r = 0; r < nrows; ++r) {
+      *reinterpret_cast<uint16_t*>(p.xq + (size_t)rows[r] * (H / 2) + g * 64 + lane * 2) = (uint16_t)packed;
+      if (lane == 0) *reinterpret_cast<uint32_t*>(p.xsc + ((size_t)g * p.xs_ld + rows[r]) * 16) = word;
+    }
+  }
+  if (p.out_acc) {
+    float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
+    for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s) {
+  quant_mxfp4_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 __global__ void finalize_kernel(const float4* __restrict__ acc, uint2* __restrict__ out, long long n4) {
   griddep_wait();  // the combine buffer is complete once GEMM2 has finished
   for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {

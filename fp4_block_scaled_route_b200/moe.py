@@ -28,6 +28,7 @@ MOE_ERR_BAD_ROUTING = 6
 MOE_WFMT_FP8_E4M3_B128 = 0
 MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1
 MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2
+MOE_WFMT_MXFP4_W4A4 = 3
 
 # Every entry point declared in include/moe.h: name -> (restype, argtypes)
 _vp = ctypes.c_void_p
@@ -252,7 +253,7 @@ class MoeLayer:
         (NVFP4: xq / hq packed, two codes per byte)."""
         import numpy as np
         P = T * self.k + self.n_shared * T
-        cw = 2 if self.wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 else 1
+        cw = 2 if self.wfmt in (MOE_WFMT_NVFP4_E2M1_E4M3_K16, MOE_WFMT_MXFP4_W4A4) else 1
         xq = np.zeros((max(P, 1), self.H // cw), np.uint8)
         xs = np.zeros((max(P, 1), self.H // 128), np.float32)
         hq = np.zeros((max(P, 1), self.I // cw), np.uint8)
@@ -262,11 +263,13 @@ class MoeLayer:
         return xq[:P], xs[:P], hq[:P], hs[:P]
 
     def block_scales(self, T, stream=None):
-        """NVFP4: (xsc [P, H/16], hsc [P, I/16]) E4M3 block codes of the last forward, host numpy."""
+        """4-bit activations: (xsc, hsc) block codes of the last forward, host numpy
+        (NVFP4: E4M3 [P, H/16], [P, I/16]; MXFP4 x MXFP4: E8M0 [P, H/32], [P, I/32])."""
         import numpy as np
         P = T * self.k + self.n_shared * T
-        xsc = np.zeros((max(P, 1), self.H // 16), np.uint8)
-        hsc = np.zeros((max(P, 1), self.I // 16), np.uint8)
+        bs = 16 if self.wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 else 32
+        xsc = np.zeros((max(P, 1), self.H // bs), np.uint8)
+        hsc = np.zeros((max(P, 1), self.I // bs), np.uint8)
         _check(moe_get_block_scales(self.ctx, xsc.ctypes.data, hsc.ctypes.data, _stream_handle(stream)),
                "moe_get_block_scales")
         return xsc[:P], hsc[:P]

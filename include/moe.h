@@ -75,7 +75,15 @@ enum {
    * Weight value = e2m1 * e4m3(scale) * g.  The tensor cores take NVFP4 only
    * with FP4 on both sides, so the activations are quantised to NVFP4 too
    * (see moe_forward_nvfp4).  Used through moe_forward_nvfp4(). */
-  MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2
+  MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2,
+  /* MXFP4 weights (the MOE_WFMT_MXFP4_E2M1_E8M0_K32 layout and packed scales)
+   * with MXFP4 activations: x and the SwiGLU output are quantised per 32
+   * columns to E2M1 with an E8M0 scale 2^X, X = floor(log2 amax) - 2 clamped
+   * to [-127, 127] (OCP MX v1.0; -127 for an all-zero block), so that the
+   * tensor cores (kind::mxf4, UE8M0 scales on both operands) apply every
+   * scale and no fp32 scale is promoted.  Used through moe_forward(); tiles
+   * hold at most 32 tokens. */
+  MOE_WFMT_MXFP4_W4A4 = 3
 };
 
 /* moe_create -- context for a layer with hidden size H, expert intermediate
@@ -169,14 +177,17 @@ moe_status moe_get_routing(moe_ctx* ctx, int32_t* counts, int32_t* offsets, int3
  *   xq u8 E4M3 [P, H], xs fp32 [P, H/128]  (GEMM1 input, P = T*k + n_shared*T)
  *   hq u8 E4M3 [P, I], hs fp32 [P, I/128]  (GEMM2 input)
  * (NVFP4 contexts: xq [P, H/2] and hq [P, I/2] packed E2M1, xs / hs the
- * per-128 scales S.)  Rows of dropped positions are unspecified.  Any
+ * per-128 scales S; MXFP4 x MXFP4 contexts: the same packed codes, xs / hs
+ * unspecified.)  Rows of dropped positions are unspecified.  Any
  * pointer may be NULL. */
 moe_status moe_get_activations(moe_ctx* ctx, uint8_t* xq, float* xs, uint8_t* hq, float* hs, void* stream);
 
-/* moe_get_block_scales -- NVFP4 contexts only (else MOE_ERR_UNSUPPORTED):
- * the E4M3 block codes of the last call's activations, after a stream
- * synchronisation, rows in routing-position order: xsc u8 [P, H/16],
- * hsc u8 [P, I/16].  Either pointer may be NULL.  Debug / test entry point. */
+/* moe_get_block_scales -- contexts with 4-bit activations only (else
+ * MOE_ERR_UNSUPPORTED): the block codes of the last call's activations,
+ * after a stream synchronisation, rows in routing-position order.  NVFP4:
+ * E4M3 codes xsc u8 [P, H/16], hsc u8 [P, I/16]; MXFP4 x MXFP4: E8M0 codes
+ * xsc u8 [P, H/32], hsc u8 [P, I/32].  Either pointer may be NULL.  Debug /
+ * test entry point. */
 moe_status moe_get_block_scales(moe_ctx* ctx, uint8_t* xsc, uint8_t* hsc, void* stream);
 
 /* moe_get_device_status -- synchronises `stream`, returns MOE_OK,
