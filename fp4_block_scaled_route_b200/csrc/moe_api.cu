@@ -376,15 +376,19 @@ void moe_destroy(moe_ctx* c) {
 }
 
 // The launch sequence of one layer for every weight format; g13 / g2 are the
-// NVFP4 global scales (null for the other formats).
+// NVFP4 global scales (null for the other formats).  With partial_out the
+// fp32 combine result goes to that caller buffer (GEMM2 reduces into it) and
+// no bf16 output is written (out is ignored).
 static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,
                                const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
-                               const float* g2, void* out, void* stream) {
+                               const float* g2, void* out, void* stream, float* partial_out = nullptr) {
   if (!c || T < 0 || T > c->max_T) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  if (!x || !ids || !topk_w || !w13 || !s13 || !w2 || !s2 || !out) return MOE_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(w13, 128) || !aligned(w2, 128) || !aligned(s13, 16) ||
-      !aligned(s2, 16) || !aligned(ids, 4) || !aligned(topk_w, 4))
+  const bool partial = partial_out != nullptr;
+  if (!x || !ids || !topk_w || !w13 || !s13 || !w2 || !s2 || (!out && !partial)) return MOE_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || (!partial && !aligned(out, 16)) || (partial && !aligned(partial_out, 16)) ||
+      !aligned(w13, 128) || !aligned(w2, 128) || !aligned(s13, 16) || !aligned(s2, 16) || !aligned(ids, 4) ||
+      !aligned(topk_w, 4))
     return MOE_ERR_INVALID_ARG;
   const bool nvfp4 = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16);
   const bool a4 = nvfp4 || c->wfmt == MOE_WFMT_MXFP4_W4A4;  // 4-bit activations, packed operands
@@ -468,14 +472,15 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 
   const int P = S + c->n_shared * T;
-  const bool rows = c->y_rows != nullptr;
+  const bool rows = c->y_rows != nullptr && !partial;  // a partial sum always uses the fused combine
+  float* acc = partial ? partial_out : c->out_acc;
   (void)P;
 
   QuantParams qp;
   qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs;
   qp.xs_ld = c->S_pad;
-  qp.out_acc = rows ? nullptr : c->out_acc;
+  qp.out_acc = rows ? nullptr : acc;
   qp.xsc = c->xsc;
   mark(MOE_STAGE_QUANT);
   const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)
@@ -494,7 +499,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   g.ascale = c->xs;
   g.scale_ld = c->S_pad;
   g.hq = c->hq; g.hs = c->hs;
-  g.perm = c->perm; g.topk_w = topk_w; g.out_acc = c->out_acc;
+  g.perm = c->perm; g.topk_w = topk_w; g.out_acc = acc;
   g.tiles = c->tiles; g.num_tiles = c->num_tiles; g.status = c->status;
   g.y_rows = nullptr;
   g.inject = c->inject;
@@ -515,7 +520,10 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, tsh, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
   mark(MOE_STAGE_FINALIZE);
-  if (rows) {
+  if (partial) {
+    // the caller sums the partials (e.g. across tensor-parallel ranks) and
+    // converts them with moe_finalize_bf16
+  } else if (rows) {
     moe::CombineParams cp;
     cp.T = T; cp.H = H; cp.k = c->k; cp.n_shared = c->n_shared;
     cp.y_rows = c->y_rows; cp.inv = c->inv; cp.topk_w = topk_w; cp.out = static_cast<uint16_t*>(out);
@@ -538,6 +546,22 @@ moe_status moe_forward(moe_ctx* c, int T, const void* x, const int32_t* ids, con
                        const void* s13, const void* w2, const void* s2, void* out, void* stream) {
   if (c && c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_INVALID_ARG;  // needs moe_forward_nvfp4
   return forward_impl(c, T, x, ids, topk_w, w13, s13, nullptr, w2, s2, nullptr, out, stream);
+}
+
+moe_status moe_forward_partial(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,
+                               const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
+                               const float* g2, float* out_f32, void* stream) {
+  if (!out_f32) return MOE_ERR_INVALID_ARG;
+  return forward_impl(c, T, x, ids, topk_w, w13, s13, g13, w2, s2, g2, nullptr, stream, out_f32);
+}
+
+moe_status moe_finalize_bf16(const float* in, void* out, long long n, void* stream) {
+  if (n < 0 || n % 4) return MOE_ERR_INVALID_ARG;
+  if (n == 0) return MOE_OK;
+  if (!in || !out || !aligned(in, 16) || !aligned(out, 8)) return MOE_ERR_INVALID_ARG;
+  if (moe::launch_finalize(in, static_cast<uint16_t*>(out), n, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return MOE_OK;
 }
 
 moe_status moe_forward_nvfp4(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,

@@ -39,6 +39,8 @@ SIGNATURES = {
     "moe_destroy": (None, [_vp]),
     "moe_forward": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_forward_nvfp4": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_forward_partial": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "moe_finalize_bf16": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
     "moe_pack_mxfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
     "moe_pack_nvfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
     "moe_get_routing": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
@@ -113,6 +115,14 @@ def moe_forward(ctx, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, stream) -> i
 
 def moe_forward_nvfp4(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out, stream) -> int:
     return lib().moe_forward_nvfp4(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out, stream)
+
+
+def moe_forward_partial(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out_f32, stream) -> int:
+    return lib().moe_forward_partial(ctx, T, x, topk_ids, topk_w, w13, s13, g13, w2, s2, g2, out_f32, stream)
+
+
+def moe_finalize_bf16(inp, out, n, stream) -> int:
+    return lib().moe_finalize_bf16(inp, out, n, stream)
 
 
 def moe_forward_noalloc(H, I, E, k, wfmt, n_shared, T, x, topk_ids, topk_w, w13, s13, w2, s2, out, d_status,
@@ -235,6 +245,20 @@ class MoeLayer:
                                _ptr(w2), _ptr(s2), _ptr(out), _stream_handle(stream)), "moe_forward")
         return out
 
+    def forward_partial(self, x, topk_ids, topk_w, w13, s13, w2, s2, out=None, stream=None, g13=None, g2=None):
+        """fp32 [T, H] partial combine result of this context's I slice (moe_forward_partial)."""
+        import torch
+        T = x.shape[0]
+        if out is None:
+            out = torch.empty((T, self.H), dtype=torch.float32, device=x.device)
+        for t in (x, topk_ids, topk_w, w13, s13, w2, s2, out):
+            if not t.is_cuda or not t.is_contiguous():
+                raise ValueError("MoeLayer.forward_partial needs contiguous CUDA tensors")
+        _check(moe_forward_partial(self.ctx, T, _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(w13), _ptr(s13),
+                                   _ptr(g13), _ptr(w2), _ptr(s2), _ptr(g2), _ptr(out), _stream_handle(stream)),
+               "moe_forward_partial")
+        return out
+
     def routing(self, T, stream=None):
         """(counts, offsets, perm, inv) of the last forward, as host int32 numpy arrays."""
         import numpy as np
@@ -318,3 +342,13 @@ def pack_mxfp4_scales(s, stream=None):
     _check(moe_pack_mxfp4_scales(_ptr(s.contiguous()), _ptr(dst), NE * rows, kg * 32, _stream_handle(stream)),
            "moe_pack_mxfp4_scales")
     return dst
+
+
+def finalize_bf16(acc, out=None, stream=None):
+    """bf16 rounding of a summed fp32 [T, H] result (moe_finalize_bf16)."""
+    import torch
+    if out is None:
+        out = torch.empty(acc.shape, dtype=torch.bfloat16, device=acc.device)
+    _check(moe_finalize_bf16(_ptr(acc.contiguous()), _ptr(out), acc.numel(), _stream_handle(stream)),
+           "moe_finalize_bf16")
+    return out

@@ -147,6 +147,26 @@ moe_status moe_forward_nvfp4(moe_ctx* ctx, int T, const void* x, const int32_t* 
                              const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
                              const float* g2, void* out, void* stream);
 
+/* moe_forward_partial -- the layer up to its fp32 combine result, for tensor
+ * parallelism over I (SURVEY's first multi-GPU extension): every rank holds
+ * an I/G slice of each expert (its gate and up rows of w13, the matching
+ * columns of w2 and their scales; I/G a multiple of 128, so no quantisation
+ * group straddles two ranks), and the layer output is the sum over ranks of
+ * these partial results.  Arguments as moe_forward() / moe_forward_nvfp4()
+ * (g13, g2 required for NVFP4 contexts, ignored otherwise), with the
+ * context's I the slice size; out_f32 is device fp32 [T, H], 16-byte aligned,
+ * overwritten with this rank's partial out[t] = sum_j w[t,j] * Y_slice(t, j)
+ * (+ the shared expert's slice).  Sum the ranks' buffers (for example an
+ * NCCL all-reduce on `stream`), then convert with moe_finalize_bf16(). */
+moe_status moe_forward_partial(moe_ctx* ctx, int T, const void* x, const int32_t* topk_ids, const float* topk_w,
+                               const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
+                               const float* g2, float* out_f32, void* stream);
+
+/* moe_finalize_bf16 -- out[i] = bf16_rn(in[i]) for n values (n % 4 == 0; in
+ * 16-byte and out 8-byte aligned, device pointers), on `stream`: the layer's
+ * output step applied to summed partial results. */
+moe_status moe_finalize_bf16(const float* in, void* out, long long n, void* stream);
+
 /* moe_pack_mxfp4_scales -- converts E8M0 scales from the plain layout
  * [rows, K/32] (rows = NE*2I for s13, NE*H for s2) into the 128x128 atom
  * layout moe_forward() reads for MOE_WFMT_MXFP4_E2M1_E8M0_K32 (same byte
