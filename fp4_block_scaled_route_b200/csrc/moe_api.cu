@@ -471,10 +471,8 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   mark(MOE_STAGE_ROUTE);
   if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 
-  const int P = S + c->n_shared * T;
   const bool rows = c->y_rows != nullptr && !partial;  // a partial sum always uses the fused combine
   float* acc = partial ? partial_out : c->out_acc;
-  (void)P;
 
   QuantParams qp;
   qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
