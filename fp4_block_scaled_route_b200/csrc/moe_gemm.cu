@@ -73,9 +73,9 @@ struct GemmCfg {
   static constexpr int STAGE_BYTES = NA * A_BYTES + B_BYTES + SF_BYTES;
   static constexpr int KB_MAX = 64;                       // K <= 8192
   // Epilogue column groups (warpgroups, each taking CPT of the BN columns):
-  // two for 4-bit-activation stages of four tiles, whose per-unit SwiGLU + requant tail
-  // would otherwise stall the MMAs (only NBUF K blocks fit ahead of it).
-  static constexpr int CG = (BN > 64) ? BN / 64 : (P4 && NT == 4) ? 2 : 1;
+  // two for stages of four tiles, whose per-unit SwiGLU + requant tail would
+  // otherwise stall the MMAs (only NBUF K blocks fit ahead of it).
+  static constexpr int CG = (BN > 64) ? BN / 64 : (NT == 4) ? 2 : 1;
   static constexpr int CPT = BN / CG;                     // columns per epilogue thread
   static constexpr int EPI_THREADS = 128 * CG;
   // Warpgroup 0: NPROD TMA producer warps (warp p issues all loads of the
@@ -99,10 +99,6 @@ struct GemmCfg {
   static constexpr int EPI_WARP0 = NPROD + NMMA;
   static constexpr int THREADS = 32 * EPI_WARP0 + EPI_THREADS;
   static constexpr int MAX_STAGES = P4 ? 24 : 12;
-  // TMEM accumulators in flight: the MMA warp may run NBUF K blocks ahead of
-  // the promoting epilogue (short K steps would otherwise be latency bound).
-  static constexpr int NBUF_RAW = 256 / (NA * BN);
-  static constexpr int NBUF = NBUF_RAW < 2 ? 2 : (NBUF_RAW > 8 ? 8 : NBUF_RAW);
   static constexpr int NBARS = 2 * MAX_STAGES + 2 * 8 + 1;
   static constexpr int AUX_BYTES =
       ((BN * KB_MAX + NA * KB_MAX + 6 * BN + 2 * NA * BN) * 4 + NBARS * 8 + 16 + 15) / 16 * 16;
@@ -110,6 +106,28 @@ struct GemmCfg {
   static constexpr int FIT = (SMEM_LIMIT - 1024 - AUX_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = FIT > MAX_STAGES ? MAX_STAGES : FIT;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + AUX_BYTES;
+  // TMEM accumulators in flight: the MMA warps may run NBUF K blocks ahead of
+  // the promoting epilogue (short K steps would otherwise be latency bound).
+  //
+  // Bound on NBUF from the stage ring.  The MMA warps take the iterations in
+  // turn and are not ordered among themselves.  When warp m waits for the
+  // stage of iteration it, the epilogue has released it - NBUF (so every
+  // iteration up to it - NBUF has landed), and warp m has consumed its own
+  // earlier iterations; an iteration it - d of another MMA warp (d not a
+  // multiple of NMMA, d < NBUF) may still be waiting for its bytes.  If it
+  // shares the stage (d a multiple of STAGES), warp m's parity wait sees that
+  // stage's phase before last as complete and passes before its own bytes
+  // land, and the producer can then post a second transaction count on a
+  // phase that has not completed.  So either STAGES is a multiple of NMMA
+  // (every iteration sharing warp m's stage is warp m's own) or NBUF <= STAGES.
+  static constexpr int NBUF_RAW = 256 / (NA * BN);
+  static constexpr int NBUF_WANT = NBUF_RAW < 2 ? 2 : (NBUF_RAW > 8 ? 8 : NBUF_RAW);
+  static constexpr int NBUF = (STAGES % NMMA == 0 || STAGES >= NBUF_WANT) ? NBUF_WANT : STAGES;
+  static_assert(STAGES % NMMA == 0 || NBUF <= STAGES, "an MMA warp could pass a stage's stale phase");
+  // The producers take the iterations in turn as well; a producer's wait for
+  // the MMAs of it - STAGES is exact when its previous iteration it - NPROD
+  // is no older than that (its own wait then implies the phase before).
+  static_assert(STAGES >= NPROD, "a producer could pass a stale MMA-done phase");
   static constexpr int ACC_COLS = NBUF * NA * BN;         // NBUF accumulators
   // Scale-factor columns per accumulator buffer: MXFP4 one 4-column atom per
   // weight tile (B: 4 shared columns of unit scales); NVFP4 two atoms per
@@ -792,13 +810,15 @@ static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb
   return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT>, ta, tb, ts, p);
 }
 
-// Weight tiles per stage with 4-bit activations (NVFP4, MXFP4 x MXFP4): a
-// stage of two packed 128-row tiles carries
-// only 16 KB of weights, and per stage the tensor pipe also copies the
-// block-scale atoms and commits, which at that size issues slower than HBM
-// delivers.  16-token tiles therefore take four tiles per stage (32 KB)
-// where the channel count divides: GEMM1 two gate/up pairs (I % 256 == 0),
-// GEMM2 four output tiles (H % 512 == 0), else two (H % 256 == 0), else one.
+// Weight tiles per stage with 4-bit weights: a stage of one or two 128-row
+// tiles carries only 8-16 KB of weights, and per stage the tensor pipe also
+// copies the block-scale atoms and commits, which at that size issues slower
+// than HBM delivers.  16-token tiles therefore take four tiles per stage
+// (32 KB) where the channel count divides: GEMM1 two gate/up pairs
+// (I % 256 == 0; 4-bit activations only -- MXFP4 weights with FP8
+// activations measured faster with one pair, whose padded tiles leave room
+// for twice the stages), GEMM2 four output tiles (H % 512 == 0), else two
+// (H % 256 == 0), else one.
 static int fp4_tiles(int kind, int BN, const GemmParams& p) {
   if (kind == 1) return (BN == 16 && p.I % 256 == 0) ? 4 : 2;
   if (BN == 16 && p.H % 512 == 0) return 4;
@@ -818,7 +838,8 @@ cudaError_t gemm_setup(int wfmt) {
     if (e == cudaSuccess) e = gemm_tm_setup();
   } else if (wfmt == 1) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
-    MOE_SET(2, 16, 1) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
+    MOE_SET_NT(2, 16, 1, 4) MOE_SET_NT(2, 16, 1, 2) MOE_SET(2, 16, 1)
+    MOE_SET_NT(2, 32, 1, 2) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
   } else if (wfmt == 2) {
     MOE_SET_NT(1, 16, 2, 4) MOE_SET_NT(1, 16, 2, 2) MOE_SET_NT(1, 32, 2, 2)
     MOE_SET_NT(2, 16, 2, 4) MOE_SET_NT(2, 16, 2, 2) MOE_SET_NT(2, 16, 2, 1)
@@ -873,9 +894,13 @@ cudaError_t launch_gemm2(int wfmt, int BN, int grid, const CUtensorMap& tw, cons
       case 128: return launch_gemm2_tm(grid, tw, th, p, s);
     }
   } else if (wfmt == 1) {
+    const int nt = fp4_tiles(2, BN, p);
     switch (BN) {
-      case 16: return launch<2, 16, 1>(grid, tw, th, tsf, p, s);
-      case 32: return launch<2, 32, 1>(grid, tw, th, tsf, p, s);
+      case 16:
+        if (nt == 4) return launch<2, 16, 1, 4>(grid, tw, th, tsf, p, s);
+        if (nt == 2) return launch<2, 16, 1, 2>(grid, tw, th, tsf, p, s);
+        return launch<2, 16, 1>(grid, tw, th, tsf, p, s);
+      case 32: return nt == 2 ? launch<2, 32, 1, 2>(grid, tw, th, tsf, p, s) : launch<2, 32, 1>(grid, tw, th, tsf, p, s);
       case 64: return launch<2, 64, 1>(grid, tw, th, tsf, p, s);
     }
   } else if (wfmt == 2) {

@@ -49,6 +49,12 @@ struct TmCfg {
   static constexpr int NBUF = 2;                 // TMEM accumulators (2 x 256 columns)
   static constexpr int NMD = STAGES + NBUF;      // MMA-done barrier ring
   static constexpr int NPROD = 2, NMMA = 2;
+  // The MMA warps and the producers take the iterations in turn without
+  // ordering among themselves; their parity waits are exact when every
+  // iteration sharing a warp's stage is its own or already released (the
+  // stage-ring bound of the decode kernel).
+  static_assert(STAGES % NMMA == 0 || NBUF <= STAGES, "an MMA warp could pass a stage's stale phase");
+  static_assert(STAGES >= NPROD, "a producer could pass a stale MMA-done phase");
   static constexpr int MMA_WARP = NPROD;
   static constexpr int EPI_WARP0 = NPROD + NMMA; // = 4: warpgroup 0 is producers + MMA
   static constexpr int CG = 2;                   // epilogue warpgroups (column halves)

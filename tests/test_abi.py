@@ -55,6 +55,11 @@ def test_host_argument_checks_without_gpu(libmoe):
     assert libmoe.moe_create_ex(256, 128, 8, 2, 7, 16, 0, ctypes.byref(ctx)) == moe.MOE_ERR_UNSUPPORTED
     assert libmoe.moe_create_ex(256, 128, 8, 2, 0, 0, 0, ctypes.byref(ctx)) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_create(256, 128, 8, 2, 0, None) == moe.MOE_ERR_INVALID_ARG
+    # one past each documented limit: H, I <= 8192, E <= 1024, k <= 32, one shared expert
+    for H, I, E, k, nsh in [(8320, 128, 4, 2, 0), (128, 8320, 4, 2, 0), (128, 128, 1025, 2, 0),
+                            (128, 128, 64, 33, 0), (128, 128, 4, 2, 2)]:
+        st = libmoe.moe_create_ex(H, I, E, k, 0, 16, nsh, ctypes.byref(ctx))
+        assert st in (moe.MOE_ERR_UNSUPPORTED, moe.MOE_ERR_INVALID_ARG), (H, I, E, k, nsh, st)
     assert libmoe.moe_forward(None, 1, None, None, None, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_pack_mxfp4_scales(None, None, 128, 128, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_set_fault_injection(None, 1) == moe.MOE_ERR_INVALID_ARG

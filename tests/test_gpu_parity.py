@@ -281,3 +281,25 @@ def test_every_tile_width(bn, monkeypatch):
     layer, out = run_gpu(L)
     assert layer.last_config()[0] == int(bn)
     assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], f"tile {bn}")
+
+
+# ---- MXFP4 weights at every GEMM2 weight-tile count per stage -----------------
+# 16-token tiles take four 128-row W2 tiles per stage where H % 512 == 0,
+# else two where H % 256 == 0, else one; 32-token tiles two where
+# H % 256 == 0.  GEMM1 keeps one gate/up pair per stage.
+MX_TILES = [
+    ("bn16_g2x4", "16", dict(T=40, H=1024, I=512, E=8, k=2, wfmt=1)),
+    ("bn16_g2x2_shared", "16", dict(T=40, H=768, I=256, E=8, k=2, wfmt=1, n_shared=1)),
+    ("bn16_g2x1", "16", dict(T=40, H=640, I=384, E=8, k=2, wfmt=1)),
+    ("bn32_g2x2", "32", dict(T=90, H=768, I=256, E=6, k=3, wfmt=1)),
+]
+
+
+@pytest.mark.parametrize("name,bn,cfg", MX_TILES, ids=[m[0] for m in MX_TILES])
+def test_mxfp4_weight_tiles_per_stage(name, bn, cfg, monkeypatch):
+    monkeypatch.setenv("MOE_TILE_N", bn)
+    L = synth.make_layer(dict(cfg, routing="uniform"), 63, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.last_config()[0] == int(bn)
+    assert layer.device_status() == moe.MOE_OK
+    assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], name)
