@@ -20,11 +20,25 @@ namespace moe {
 
 // ---------------------------------------------------------------------------
 // One CTA of 1024 threads.  Warp w owns the contiguous slot range
-// [w*chunk, (w+1)*chunk); __match_any_sync groups equal expert ids within a
+// [w*chunk, (w+1)*chunk); a ballot match groups equal expert ids within a
 // 32-slot step, so a slot's position is
 //   offsets[e] + (slots of e in earlier warps) + (earlier steps of this warp)
 //   + (lower lanes with the same id in this step),
 // which is exactly the stable counting-sort position.
+constexpr int kRouteBatch = 8;  // 32-slot steps whose ids are loaded together
+
+// Lanes of the warp holding the same key as this lane, from one ballot per
+// key bit (the warp-ballot form of a match): key < 2^nbits.
+__device__ __forceinline__ unsigned ballot_match(int key, int nbits) {
+  unsigned peers = 0xFFFFFFFFu;
+  for (int b = 0; b < nbits; ++b) {
+    const bool bit = (key >> b) & 1;
+    const unsigned m = __ballot_sync(0xFFFFFFFFu, bit);
+    peers &= bit ? m : ~m;
+  }
+  return peers;
+}
+
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) {
   extern __shared__ int sm[];
   const int E = p.E, NG = p.E + p.n_shared;
@@ -41,23 +55,43 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   __syncthreads();
 
   const int chunk = (((S + 31) / 32) + 31) & ~31;
+  const int kbits = 32 - __clz(E);  // bits of the largest key, E (a dropped id)
   const int beg = min(S, warp * chunk), end = min(S, beg + chunk);
 
-  // pass A: per-warp, per-expert counts
-  for (int base = beg; base < end; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < end) {
-      e = p.ids[s];
-      if (e < 0 || e >= E) {
-        e = -1;
-        s_bad = 1;
+  // The expert ids of kRouteBatch consecutive 32-slot steps, loaded before
+  // any of them is used, so a warp waits for one load latency per batch
+  // rather than one per step (out-of-range ids read as -1).
+  auto load_batch = [&](int b0, int (&ev)[kRouteBatch], bool& bad) {
+#pragma unroll
+    for (int r = 0; r < kRouteBatch; ++r) {
+      const int s = b0 + r * 32 + lane;
+      ev[r] = (s < end) ? p.ids[s] : -1;
+    }
+#pragma unroll
+    for (int r = 0; r < kRouteBatch; ++r) {
+      const int s = b0 + r * 32 + lane;
+      if (s < end && (ev[r] < 0 || ev[r] >= E)) {
+        ev[r] = -1;
+        bad = true;
       }
     }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
-    __syncwarp();
+  };
+
+  // pass A: per-warp, per-expert counts
+  bool bad = false;
+  for (int b0 = beg; b0 < end; b0 += 32 * kRouteBatch) {
+    int ev[kRouteBatch];
+    load_batch(b0, ev, bad);
+#pragma unroll
+    for (int r = 0; r < kRouteBatch; ++r) {
+      if (b0 + r * 32 >= end) break;  // uniform across the warp
+      const int e = ev[r];
+      const unsigned peers = ballot_match(e >= 0 ? e : E, kbits);
+      if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
+      __syncwarp();
+    }
   }
+  if (bad) s_bad = 1;
   __syncthreads();
 
   // per expert: total count, and counts of earlier warps (exclusive over warps)
@@ -99,27 +133,29 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   for (int g = tid; g <= NG; g += kRouteThreads) p.offsets[g] = off[g];
 
   // pass B: stable scatter
-  for (int base = beg; base < end; base += 32) {
-    const int s = base + lane;
-    int e = -1;
-    if (s < end) {
-      e = p.ids[s];
-      if (e < 0 || e >= E) e = -1;
-    }
-    const unsigned peers = __match_any_sync(0xFFFFFFFFu, e);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
-    if (s < end) {
-      if (e >= 0) {
-        const int pos = off[e] + wc[warp * NG + e] + rank;
-        p.perm[pos] = s;
-        p.inv[s] = pos;
-      } else {
-        p.inv[s] = -1;
+  for (int b0 = beg; b0 < end; b0 += 32 * kRouteBatch) {
+    int ev[kRouteBatch];
+    load_batch(b0, ev, bad);
+#pragma unroll
+    for (int r = 0; r < kRouteBatch; ++r) {
+      if (b0 + r * 32 >= end) break;  // uniform across the warp
+      const int s = b0 + r * 32 + lane;
+      const int e = ev[r];
+      const unsigned peers = ballot_match(e >= 0 ? e : E, kbits);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      if (s < end) {
+        if (e >= 0) {
+          const int pos = off[e] + wc[warp * NG + e] + rank;
+          p.perm[pos] = s;
+          p.inv[s] = pos;
+        } else {
+          p.inv[s] = -1;
+        }
       }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
+      __syncwarp();
     }
-    __syncwarp();
-    if (e >= 0 && lane == __ffs(peers) - 1) wc[warp * NG + e] += __popc(peers);
-    __syncwarp();
   }
 
   // shared expert: every token, as virtual slot S + t, after the routed groups
