@@ -148,7 +148,7 @@ moe_status moe_forward_nvfp4(moe_ctx* ctx, int T, const void* x, const int32_t* 
                              const float* g2, void* out, void* stream);
 
 /* moe_forward_partial -- the layer up to its fp32 combine result, for tensor
- * parallelism over I (SURVEY's first multi-GPU extension): every rank holds
+ * parallelism over the intermediate size I: every rank holds
  * an I/G slice of each expert (its gate and up rows of w13, the matching
  * columns of w2 and their scales; I/G a multiple of 128, so no quantisation
  * group straddles two ranks), and the layer output is the sum over ranks of
