@@ -35,7 +35,8 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer µs and weight-stream HBM GB/s (vs ~8 TB/s) at T=1–256; TFLOP/s at T=4096"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-GEMM_SOURCES = ["fp4_block_scaled_route_b200/csrc/moe_gemm.cu", "fp4_block_scaled_route_b200/csrc/moe_ptx.cuh"]
+GEMM_SOURCES = ["fp4_block_scaled_route_b200/csrc/moe_gemm.cu", "fp4_block_scaled_route_b200/csrc/moe_gemm_tm.cu",
+                "fp4_block_scaled_route_b200/csrc/moe_ptx.cuh"]
 
 
 def log(*a):
