@@ -34,9 +34,8 @@ class Barrier:
     """mbarrier with one expected arrival per phase (and, for a stage
     barrier, the bytes of one iteration)."""
 
-    def __init__(self, needs_bytes=False):
+    def __init__(self):
         self.completed = 0
-        self.needs_bytes = needs_bytes
         self.posted = False   # arrive.expect_tx of the current phase happened
         self.pending = 0      # iterations whose bytes the current phase waits for
 
@@ -51,7 +50,7 @@ def run(STAGES, NBUF, NPROD=3, NMMA=2, iters=48, seed=0):
     """One random schedule; returns the list of violations."""
     rng = random.Random(seed)
     NMD = STAGES + NBUF
-    full = [Barrier(True) for _ in range(STAGES)]
+    full = [Barrier() for _ in range(STAGES)]
     mdone = [Barrier() for _ in range(NMD)]
     tempty = [Barrier() for _ in range(NBUF)]
     landed = set()
