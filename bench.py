@@ -35,8 +35,10 @@ sys.path.insert(0, ROOT)
 METRIC = "MoE layer µs and weight-stream HBM GB/s (vs ~8 TB/s) at T=1–256; TFLOP/s at T=4096"
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
-GEMM_SOURCES = ["fp4_block_scaled_route_b200/csrc/moe_gemm.cu", "fp4_block_scaled_route_b200/csrc/moe_gemm_tm.cu",
-                "fp4_block_scaled_route_b200/csrc/moe_ptx.cuh"]
+CSRC = "fp4_block_scaled_route_b200/csrc/"
+# sources of the decode GEMM kernel (moe_gemm_kernel); a traffic record may
+# name its own list (the token-major kernel: moe_gemm_tm.cu + moe_ptx.cuh)
+GEMM_SOURCES = [CSRC + "moe_gemm.cu", CSRC + "moe_ptx.cuh"]
 
 
 def log(*a):
@@ -74,9 +76,9 @@ def peaks():
         return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def gemm_source_hash() -> str:
+def gemm_source_hash(sources=None) -> str:
     h = hashlib.sha256()
-    for rel in GEMM_SOURCES:
+    for rel in sources or GEMM_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -94,7 +96,8 @@ def recorded_traffic(workload_name: str):
             if ":" in line and not line.startswith("#"):
                 k, v = line.split(":", 1)
                 vals[k.strip()] = v.strip()
-    if vals.get("kernel_source_sha256_16") != gemm_source_hash():
+    sources = [CSRC + n for n in vals["kernel_sources"].split()] if "kernel_sources" in vals else None
+    if vals.get("kernel_source_sha256_16") != gemm_source_hash(sources):
         return None
     try:
         return float(vals["dram_bytes_per_launch_full_size"])
