@@ -305,8 +305,8 @@ moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
  * cudaFree or allocating library routine.  The scratch (routing arrays, tile
  * list, quantised activations, fp32 combine buffer) is one file-scope device
  * array of MOE_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
- * keeps until the process exits.  The paper has no counterpart of this entry
- * point; it exists only for such callers.
+ * keeps until the process exits.  The method's sources describe no
+ * counterpart of this entry point; it exists only for such callers.
  *   H, I, E, k, wfmt, n_shared   the layer, as in moe_create_ex()
  *   T, x, topk_ids, topk_w, w13, s13, w2, s2, out   as in moe_forward()
  *   d_status   optional device int32 (caller memory): cleared, then receives
