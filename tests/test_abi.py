@@ -78,3 +78,13 @@ def test_product_path_does_not_use_the_oracle():
 def test_sources_are_sm100a_only():
     src = open(os.path.join(ROOT, "fp4_block_scaled_route_b200", "build.py")).read()
     assert "arch=compute_100a,code=sm_100a" in src
+
+
+def test_every_entry_point_is_documented():
+    """Each declaration in include/moe.h has its documentation comment
+    (operation, arguments, layout, ownership, errors) right above it."""
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    decls = list(re.finditer(r"^(moe_status|void|const char\s*\*|int)\s+(moe_\w+)\s*\(", src, flags=re.M))
+    assert len(decls) == len(declared_symbols())
+    for m in decls:
+        assert src[:m.start()].rstrip().endswith("*/"), m.group(2)

@@ -167,6 +167,13 @@ def test_odd_stage_ring_below_the_accumulators_breaks(STAGES, NBUF):
     assert any(v[0].startswith("MMA passed") for v in found), found[:3]
 
 
+def test_token_major_kernel_keeps_the_protocol():
+    """moe_gemm_tm.cu: 4 stages, 2 accumulators, 2 producer warps."""
+    assert rule_holds(4, 2, NPROD=2)
+    for seed in range(150):
+        assert run(4, 2, NPROD=2, seed=seed) == []
+
+
 def test_one_mma_warp_needs_no_rule():
     """With a single MMA warp every iteration sharing a stage is its own."""
     for seed in range(150):
