@@ -33,6 +33,10 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MoE layer µs and weight-stream HBM GB/s (vs ~8 TB/s) at T=1–256; TFLOP/s at T=4096"
+L2_BYTES = 126 * 1000 * 1000
+# a workload whose weights streamed per step are below this is timed with the
+# L2 flushed between steps (a 2 x L2 buffer written outside the timed events)
+FLUSH_BELOW_BYTES = 8 * L2_BYTES
 FALLBACK_HBM_GBS = 6650.0
 FALLBACK_BF16_TFLOPS = 1590.0
 CSRC = "fp4_block_scaled_route_b200/csrc/"
@@ -63,6 +67,10 @@ def parse():
                     help="also time the fused router (moe_router_topk) on seeded router weights of this shape")
     ap.add_argument("--green-ctx", type=int, default=0,
                     help="run the dispatch kernels in a green context of >= N SMs and the GEMMs on the rest")
+    ap.add_argument("--workloads", default=None,
+                    help="comma-separated workload indices also timed (one GPU only) and reported under "
+                         "'workloads' in the same JSON line; default: every other workload when the headline is "
+                         "the default one, none otherwise; 'none' for none")
     return ap.parse_args()
 
 
@@ -239,6 +247,119 @@ def build_layer(args, device):
     return cfg, L
 
 
+def gpu_operands(L):
+    """The layer's weights in the form moe_forward reads (MXFP4 / NVFP4 scales
+    packed once, as at weight-load time) and the NVFP4 global scales."""
+    from fp4_block_scaled_route_b200 import moe, synth
+    if L.wfmt in (synth.WFMT_MXFP4, synth.WFMT_MXFP4_A4):
+        w = (L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2))
+    elif L.wfmt == synth.WFMT_NVFP4:
+        w = (L.w13, moe.pack_nvfp4_scales(L.s13), L.w2, moe.pack_nvfp4_scales(L.s2))
+    else:
+        w = (L.w13, L.s13, L.w2, L.s2)
+    gsc = dict(g13=L.g13, g2=L.g2) if L.wfmt == synth.WFMT_NVFP4 else {}
+    return w, gsc
+
+
+def l2_label(weight_bytes: int, flush: bool) -> str:
+    if flush:
+        return (f"L2 flushed between timed steps ({2 * L2_BYTES // 10**6} MB written outside the per-step events; "
+                f"weights streamed per step {weight_bytes / 1e6:.1f} MB)")
+    return (f"inputs larger than L2 (weights streamed per step {weight_bytes / 1e9:.2f} GB, more than 8 x the "
+            f"126 MB L2); no flush")
+
+
+def time_steps(step, steps: int, stream, flush_buf=None) -> float:
+    """Device milliseconds of `steps` calls of step() on `stream` (CUDA events).
+    With flush_buf, every call has its own event pair and the buffer (larger
+    than the L2) is rewritten between calls, outside the pairs."""
+    import torch
+    if flush_buf is None:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            step()
+        e1.record(stream)
+        e1.synchronize()
+        return e0.elapsed_time(e1)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    with torch.cuda.stream(stream):
+        for i in range(steps):
+            flush_buf.fill_(i & 0xFF)
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+    evs[-1][1].synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs)
+
+
+def workload_record(idx: int, args, dev, stream, sampler):
+    """One workload of synth.CONFIGS + synth.EXTRA_CONFIGS timed on this GPU:
+    microseconds per layer, weight GB/s, TFLOP/s, the fraction of the
+    roofline max(weight bytes / HBM peak, FLOP / dense tensor peak), GEMM1's
+    own rate from per-kernel events, and the clocks seen."""
+    import torch
+    from fp4_block_scaled_route_b200 import moe, synth
+    allc = synth.CONFIGS + synth.EXTRA_CONFIGS
+    cfg = allc[idx]
+    L = synth.make_layer(cfg, synth.config_seed(idx), device=dev)
+    st = workload_stats(L, L.ids.cpu().numpy())
+    layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
+    (w13, s13, w2, s2), gsc = gpu_operands(L)
+    out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        layer.forward(L.x, L.ids, L.topk_w, w13, s13, w2, s2, out=out, stream=stream, **gsc)
+
+    flush = st["weight_bytes"] < FLUSH_BELOW_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
+    steps = max(args.steps, 100) if flush else args.steps
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    t0 = time.time()
+    ms = time_steps(step, steps, stream, flush_buf)
+    t1 = time.time()
+    moe.moe_profile_enable(layer.ctx, 1)
+    time_steps(step, steps, stream, flush_buf)
+    stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
+    moe.moe_profile_enable(layer.ctx, 0)
+    if layer.device_status() != moe.MOE_OK:
+        raise RuntimeError(f"device status not OK after workload {cfg['name']}")
+    hbm, bf16, src = peaks()
+    ratio = 4.0 if L.wfmt in (synth.WFMT_NVFP4, synth.WFMT_MXFP4_A4) else 2.0
+    tpeak = ratio * bf16
+    us = ms / steps * 1e3
+    floor_us = max(st["weight_bytes"] / (hbm * 1e9), st["flops"] / (tpeak * 1e12)) * 1e6
+    g1 = stage_ms[2]
+    g1_flops = 2.0 * st["positions"] * 2 * L.I * L.H
+    rec = {
+        "workload": cfg["name"], "T": L.T, "H": L.H, "E": L.E, "k": L.k, "I": L.I, "wfmt": WFMT_NAMES[L.wfmt],
+        "n_shared": L.n_shared, "dtype": DTYPES[L.wfmt], "experts_touched": st["experts_touched"],
+        "weight_bytes_per_step": st["weight_bytes"], "flop_per_step": st["flops"],
+        "us_per_layer": us, "weight_GBps": st["weight_bytes"] / (us * 1e-6) / 1e9,
+        "hbm_frac": st["weight_bytes"] / (us * 1e-6) / 1e9 / hbm,
+        "tflops": st["flops"] / (us * 1e-6) / 1e12, "tensor_frac": st["flops"] / (us * 1e-6) / 1e12 / tpeak,
+        "roofline_us": floor_us, "roofline_frac": floor_us / us,
+        "roofline_bound": "hbm" if st["weight_bytes"] / hbm >= st["flops"] / (tpeak * 1e3) else "tensor",
+        "gemm1": {"ms": g1, "GBps": st["gemm1_bytes"] / (g1 * 1e-3) / 1e9 if g1 > 0 else None,
+                  "hbm_frac": st["gemm1_bytes"] / (g1 * 1e-3) / 1e9 / hbm if g1 > 0 else None,
+                  "tflops": g1_flops / (g1 * 1e-3) / 1e12 if g1 > 0 else None,
+                  "tensor_frac": g1_flops / (g1 * 1e-3) / 1e12 / tpeak if g1 > 0 else None,
+                  "traffic": recorded_traffic(cfg["name"]), "algorithmic_bytes_per_launch": st["gemm1_bytes"]},
+        "stage_ms": dict(zip(moe.STAGE_NAMES, stage_ms)),
+        "peaks": {"hbm_gbs": hbm, "tensor_tflops": tpeak,
+                  "source": f"{src} hbm_gbs; {src} bf16_tflops x {ratio:g} ({'FP4' if ratio == 4 else 'FP8'}/bf16 "
+                            f"nominal ratio)"},
+        "l2": l2_label(st["weight_bytes"], flush), "steps": steps, "warmup": max(args.warmup, 3),
+        "gpu_launches": moe.MOE_NUM_STAGES * steps, "clocks": sampler.summary(t0, t1),
+    }
+    layer.close()
+    del L, out, flush_buf, w13, s13, w2, s2, gsc
+    torch.cuda.empty_cache()
+    return rec
+
+
 # ---------------------------------------------------------------------------
 def replica_throughput(dist, device, local_ms: float, local_bytes: float, steps: int):
     """Whole-job rate of independent replicas: the slowest rank's device time
@@ -400,14 +521,10 @@ def main():
     st = workload_stats(L, ids_np)
     layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
     green = layer.set_green_ctx(args.green_ctx) if args.green_ctx else None
-    if L.wfmt in (synth.WFMT_MXFP4, synth.WFMT_MXFP4_A4):
-        w13, s13, w2, s2 = L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2)
-    elif L.wfmt == synth.WFMT_NVFP4:
-        w13, s13, w2, s2 = L.w13, moe.pack_nvfp4_scales(L.s13), L.w2, moe.pack_nvfp4_scales(L.s2)
-    else:
-        w13, s13, w2, s2 = L.w13, L.s13, L.w2, L.s2
-    gsc = dict(g13=L.g13, g2=L.g2) if L.wfmt == synth.WFMT_NVFP4 else {}
+    (w13, s13, w2, s2), gsc = gpu_operands(L)
     out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device=dev)
+    flush = st["weight_bytes"] < FLUSH_BELOW_BYTES
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
     stream = torch.cuda.current_stream(dev)
 
     def step():
@@ -428,28 +545,19 @@ def main():
         dist.barrier()
     torch.cuda.synchronize(dev)
     tw0 = time.time()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
+    ms = time_steps(step, args.steps, stream, flush_buf)
     torch.cuda.synchronize(dev)
     tw1 = time.time()
     if dist:
         dist.barrier()
-    ms = ev0.elapsed_time(ev1)
     clocks = sampler.summary(tw0, tw1)
-    sampler.stop()
 
     # ---- second timed region: the same K steps with CUDA events around each
     # kernel of the layer (on the launching stream), for the per-kernel times ----
     moe.moe_profile_enable(layer.ctx, 1)
     torch.cuda.synchronize(dev)
-    ev0.record(stream)
-    for _ in range(args.steps):
-        step()
-    ev1.record(stream)
+    ms_prof = time_steps(step, args.steps, stream, flush_buf)
     torch.cuda.synchronize(dev)
-    ms_prof = ev0.elapsed_time(ev1)
     stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
     moe.moe_profile_enable(layer.ctx, 0)
     if layer.device_status() != moe.MOE_OK:
@@ -550,11 +658,34 @@ def main():
     if dist:
         dist.barrier()
     if rank != 0:
+        sampler.stop()
         if dist:
             dist.destroy_process_group()
         return
 
     router = time_router(args, L, layer, dev, stream) if args.router else None
+
+    # ---- the other workloads, each timed on its own (one GPU only) ----
+    extra = []
+    if world == 1:
+        if args.workloads is None:
+            default = args.shape is None and args.workload == 1
+            extra = [i for i in range(len(synth.CONFIGS) + len(synth.EXTRA_CONFIGS)) if i != 1] if default else []
+        elif args.workloads != "none":
+            extra = [int(v) for v in args.workloads.split(",") if v.strip()]
+    workloads = None
+    if extra:
+        # free the headline layer's device memory first (the prefill layer holds 11 GB of weights)
+        layer.close()
+        del w13, s13, w2, s2, gsc, out, flush_buf
+        torch.cuda.empty_cache()
+        workloads = {}
+        for i in extra:
+            rec = workload_record(i, args, dev, stream, sampler)
+            workloads[rec["workload"]] = rec
+            log(f"workload {rec['workload']}: {rec['us_per_layer']:.1f} us, {rec['weight_GBps']:.0f} GB/s, "
+                f"{rec['tflops']:.1f} TFLOP/s, roofline frac {rec['roofline_frac']:.3f}")
+    sampler.stop()
 
     cpu = None
     if world == 1 and not args.no_cpu_baseline:
@@ -569,7 +700,7 @@ def main():
         "config": {"workload": cfg["name"], "T": L.T, "H": L.H, "E": L.E, "k": L.k, "I": L.I,
                    "wfmt": WFMT_NAMES[L.wfmt], "n_shared": L.n_shared,
                    "experts_touched": st["experts_touched"], "weight_bytes_per_step": st["weight_bytes"],
-                   "l2": "inputs larger than L2 (weights streamed per step exceed the 126 MB L2); no flush",
+                   "l2": l2_label(st["weight_bytes"], flush),
                    "parallelism": "replicas" if world > 1 else "single GPU",
                    "green_ctx": {"dispatch_sms": green[0], "gemm_sms": green[1]} if green else None},
         "us_per_layer": ms_step * 1e3,
@@ -583,6 +714,8 @@ def main():
         "gpu_launches": moe.MOE_NUM_STAGES * args.steps,  # per timed region
         "clocks": clocks,
     }
+    if workloads:
+        line["workloads"] = workloads
     if router:
         line["router"] = router
     print(json.dumps(line), flush=True)
