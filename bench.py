@@ -67,6 +67,9 @@ def parse():
                     help="also time the fused router (moe_router_topk) on seeded router weights of this shape")
     ap.add_argument("--green-ctx", type=int, default=0,
                     help="run the dispatch kernels in a green context of >= N SMs and the GEMMs on the rest")
+    ap.add_argument("--dispatch-ctas", type=int, default=0,
+                    help="dispatch overlap: the last N CTAs of the GEMM1 launch quantise the activations and "
+                         "publish per-expert ready counters (one cooperative launch); 0 = off")
     ap.add_argument("--workloads", default=None,
                     help="comma-separated workload indices also timed (one GPU only) and reported under "
                          "'workloads' in the same JSON line; default: every other workload when the headline is "
@@ -521,6 +524,7 @@ def main():
     st = workload_stats(L, ids_np)
     layer = moe.MoeLayer(L.H, L.I, L.E, L.k, L.wfmt, max_T=L.T, n_shared=L.n_shared)
     green = layer.set_green_ctx(args.green_ctx) if args.green_ctx else None
+    disp = layer.set_dispatch_overlap(args.dispatch_ctas) if args.dispatch_ctas else None
     (w13, s13, w2, s2), gsc = gpu_operands(L)
     out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device=dev)
     flush = st["weight_bytes"] < FLUSH_BELOW_BYTES
@@ -702,7 +706,8 @@ def main():
                    "experts_touched": st["experts_touched"], "weight_bytes_per_step": st["weight_bytes"],
                    "l2": l2_label(st["weight_bytes"], flush),
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "green_ctx": {"dispatch_sms": green[0], "gemm_sms": green[1]} if green else None},
+                   "green_ctx": {"dispatch_sms": green[0], "gemm_sms": green[1]} if green else None,
+                   "dispatch_overlap_ctas": disp},
         "us_per_layer": ms_step * 1e3,
         "tflops": st["flops"] / (ms_step * 1e-3) / 1e12,
         "hbm_frac_of_step": frac_step,

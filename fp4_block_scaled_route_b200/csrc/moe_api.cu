@@ -6,6 +6,9 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <iterator>
+#include <map>
+#include <mutex>
 #include <new>
 
 #include "moe.h"
@@ -55,6 +58,10 @@ struct moe_ctx {
   float* rt_logits;
   const void* c_wr;
   CUtensorMap tm_wr;
+  // dispatch overlap (moe_set_dispatch_overlap): CTAs of the GEMM1 launch
+  // that quantise the activations first, and the per-group ready counters
+  int disp_ctas;
+  int32_t* ready;
 };
 
 
@@ -138,6 +145,25 @@ bool make_map(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t
 
 size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
+// Device ranges holding packed block scales: start -> (end, format).  A new
+// range replaces every range it overlaps (their contents were overwritten).
+std::mutex g_packed_mu;
+std::map<uintptr_t, std::pair<uintptr_t, int>> g_packed;
+
+void register_packed(const void* p, size_t bytes, int fmt) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p), hi = lo + bytes;
+  std::lock_guard<std::mutex> lock(g_packed_mu);
+  auto it = g_packed.lower_bound(lo);
+  if (it != g_packed.begin() && std::prev(it)->second.first > lo) --it;
+  while (it != g_packed.end() && it->first < hi) it = g_packed.erase(it);
+  g_packed[lo] = {hi, fmt};
+}
+
+// Bytes of packed s13 and s2 of a layer (same count as the plain layout).
+size_t packed_bytes(int fmt, int NE, int rows, int K) {
+  return (size_t)NE * rows * (K / (fmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16 ? 16 : 32));
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int pick_tile_n(const moe_ctx* c, int T) {
@@ -207,6 +233,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
     if (!strcmp(env, "rows")) c->combine_mode = 2;
   }
   if (const char* env = getenv("MOE_GREEN_CTX")) c->gc_sms = atoi(env);  // applied below, once created
+  int want_disp = 0;
+  if (const char* env = getenv("MOE_DISPATCH_CTAS")) want_disp = atoi(env);  // applied below, once created
   if (const char* env = getenv("MOE_TILE_N")) {
     const int v = atoi(env);
     if (v == 16 || v == 32 ||
@@ -228,6 +256,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_inv = take(sizeof(int32_t) * c->P_max);
   const size_t o_ntiles = take(sizeof(int32_t) * 4);
   const size_t o_status = take(sizeof(int32_t) * 4);
+  const size_t o_ready = take(sizeof(int32_t) * c->NG);
   const size_t o_tiles = take(sizeof(int4) * c->max_tiles);
   const size_t o_xq = take((size_t)c->S_pad * H);
   const size_t o_hq = take((size_t)c->S_pad * I);
@@ -263,6 +292,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->inv = reinterpret_cast<int32_t*>(b + o_inv);
   c->num_tiles = reinterpret_cast<int32_t*>(b + o_ntiles);
   c->status = reinterpret_cast<int32_t*>(b + o_status);
+  c->ready = reinterpret_cast<int32_t*>(b + o_ready);
   c->tiles = reinterpret_cast<int4*>(b + o_tiles);
   c->xq = reinterpret_cast<uint8_t*>(b + o_xq);
   c->hq = reinterpret_cast<uint8_t*>(b + o_hq);
@@ -297,6 +327,13 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
       return gs;
     }
   }
+  if (want_disp > 0) {
+    const moe_status ds = moe_set_dispatch_overlap(c, want_disp);
+    if (ds != MOE_OK) {
+      moe_destroy(c);
+      return ds;
+    }
+  }
   *out = c;
   return MOE_OK;
 }
@@ -325,6 +362,7 @@ static void green_free(moe_ctx* c) {
 
 moe_status moe_set_green_ctx(moe_ctx* c, int dispatch_sms) {
   if (!c || dispatch_sms < 0) return MOE_ERR_INVALID_ARG;
+  if (dispatch_sms > 0 && c->disp_ctas) return MOE_ERR_UNSUPPORTED;  // dispatch overlap is the other form
   if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
   green_free(c);
   if (dispatch_sms == 0) return MOE_OK;
@@ -393,6 +431,15 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   const bool nvfp4 = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16);
   const bool a4 = nvfp4 || c->wfmt == MOE_WFMT_MXFP4_W4A4;  // 4-bit activations, packed operands
   if (nvfp4 && (!g13 || !g2 || !aligned(g13, 4) || !aligned(g2, 4))) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt != MOE_WFMT_FP8_E4M3_B128) {
+    // 4-bit weights read their block scales in the packed layout only; plain
+    // scales would give wrong results without any error, so refuse scale
+    // buffers that no pack call wrote (or moe_declare_packed_scales declared)
+    const int sf = nvfp4 ? MOE_WFMT_NVFP4_E2M1_E4M3_K16 : MOE_WFMT_MXFP4_E2M1_E8M0_K32;
+    if (!moe::packed_scales_known(s13, packed_bytes(sf, c->NG, 2 * c->I, c->H), sf) ||
+        !moe::packed_scales_known(s2, packed_bytes(sf, c->NG, c->H, c->I), sf))
+      return MOE_ERR_INVALID_ARG;
+  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int H = c->H, I = c->I, NE = c->NG;
   const int S = T * c->k;
@@ -464,33 +511,39 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
       return MOE_ERR_CUDA;
   }
 
-  RouteParams rp;
+  // Dispatch overlap: no quantisation kernel; the GEMM1 launch quantises in
+  // its last disp_ctas CTAs and publishes per-group ready counters.
+  const bool overlap = c->disp_ctas > 0 && !green && !a4;
+  RouteParams rp{};
   rp.T = T; rp.k = c->k; rp.E = c->E; rp.n_shared = c->n_shared; rp.BN = BN;
   rp.ids = ids; rp.counts = c->counts; rp.offsets = c->offsets; rp.perm = c->perm; rp.inv = c->inv;
   rp.tiles = c->tiles; rp.num_tiles = c->num_tiles; rp.status = c->status;
+  rp.ready = overlap ? c->ready : nullptr;
   mark(MOE_STAGE_ROUTE);
   if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 
   const bool rows = c->y_rows != nullptr && !partial;  // a partial sum always uses the fused combine
   float* acc = partial ? partial_out : c->out_acc;
 
-  QuantParams qp;
+  QuantParams qp{};
   qp.T = T; qp.H = H; qp.k = c->k; qp.n_shared = c->n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = c->inv; qp.xq = c->xq; qp.xs = c->xs;
   qp.xs_ld = c->S_pad;
   qp.out_acc = rows ? nullptr : acc;
   qp.xsc = c->xsc;
   mark(MOE_STAGE_QUANT);
-  const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)
-                         : a4  ? moe::launch_quant_mxfp4(qp, s_disp)
-                               : moe::launch_quant(qp, s_disp);
-  if (qe != cudaSuccess) return MOE_ERR_CUDA;
+  if (!overlap) {
+    const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)
+                           : a4  ? moe::launch_quant_mxfp4(qp, s_disp)
+                                 : moe::launch_quant(qp, s_disp);
+    if (qe != cudaSuccess) return MOE_ERR_CUDA;
+  }
   if (green) {
     if (cudaEventRecord(c->gev_disp, s_disp) != cudaSuccess || cudaStreamWaitEvent(s_gemm, c->gev_disp, 0) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
 
-  GemmParams g;
+  GemmParams g{};
   g.H = H; g.I = I; g.k = c->k; g.S = S;
   g.kblocks = H / 128;
   g.wscale = static_cast<const float*>(s13);
@@ -506,9 +559,18 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   // the token block-code maps exist for 4-bit activations only; the other formats ignore the argument
   const CUtensorMap& tsx = a4 ? c->tm_xsc : c->tm_xq;
   const CUtensorMap& tsh = a4 ? c->tm_hsc : c->tm_hq;
+  if (overlap) {
+    g.disp = c->disp_ctas;
+    g.ready = c->ready; g.counts = c->counts; g.offsets = c->offsets;
+    g.x = static_cast<const uint16_t*>(x); g.xq = c->xq; g.xs = c->xs;
+    g.zero_acc = rows ? nullptr : acc;
+    g.T = T; g.NG = c->NG;
+  }
   mark(MOE_STAGE_GEMM1);
   if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
 
+  g.disp = 0;  // GEMM2 reads GEMM1's outputs after the kernel boundary
+  g.zero_acc = nullptr;
   g.kblocks = I / 128;
   g.wscale = static_cast<const float*>(s2);
   g.wglobal = g2;
@@ -562,6 +624,21 @@ moe_status moe_finalize_bf16(const float* in, void* out, long long n, void* stre
   return MOE_OK;
 }
 
+}  // extern "C"
+
+namespace moe {
+bool packed_scales_known(const void* p, size_t bytes, int fmt) {
+  const uintptr_t lo = reinterpret_cast<uintptr_t>(p);
+  std::lock_guard<std::mutex> lock(g_packed_mu);
+  auto it = g_packed.upper_bound(lo);
+  if (it == g_packed.begin()) return false;
+  --it;
+  return it->second.second == fmt && lo + bytes <= it->second.first;
+}
+}  // namespace moe
+
+extern "C" {
+
 moe_status moe_forward_nvfp4(moe_ctx* c, int T, const void* x, const int32_t* ids, const float* topk_w,
                              const void* w13, const void* s13, const float* g13, const void* w2, const void* s2,
                              const float* g2, void* out, void* stream) {
@@ -614,6 +691,7 @@ moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
   if (!src || !dst || src == dst || rows <= 0 || K <= 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
   if (moe::launch_pack_e8m0(src, dst, rows, K / 32, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
+  register_packed(dst, (size_t)rows * (K / 32), MOE_WFMT_MXFP4_E2M1_E8M0_K32);
   return MOE_OK;
 }
 
@@ -621,6 +699,15 @@ moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
   if (!src || !dst || src == dst || rows <= 0 || K <= 0 || rows % 128 || K % 128) return MOE_ERR_INVALID_ARG;
   if (moe::launch_pack_e8m0(src, dst, rows, K / 16, static_cast<cudaStream_t>(stream)) != cudaSuccess)
     return MOE_ERR_CUDA;
+  register_packed(dst, (size_t)rows * (K / 16), MOE_WFMT_NVFP4_E2M1_E4M3_K16);
+  return MOE_OK;
+}
+
+moe_status moe_declare_packed_scales(const void* p, long long bytes, int wfmt) {
+  if (!p || bytes <= 0) return MOE_ERR_INVALID_ARG;
+  if (wfmt == MOE_WFMT_MXFP4_W4A4) wfmt = MOE_WFMT_MXFP4_E2M1_E8M0_K32;  // the same E8M0 atoms
+  if (wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_INVALID_ARG;
+  register_packed(p, (size_t)bytes, wfmt);
   return MOE_OK;
 }
 
@@ -759,8 +846,30 @@ moe_status moe_profile_read(moe_ctx* c, float* avg_ms, int* calls) {
   return MOE_OK;
 }
 
+moe_status moe_set_dispatch_overlap(moe_ctx* c, int dispatch_ctas) {
+  if (!c || dispatch_ctas < 0 || dispatch_ctas > c->num_sms) return MOE_ERR_INVALID_ARG;
+  if (dispatch_ctas == 0) {
+    c->disp_ctas = 0;
+    return MOE_OK;
+  }
+  // FP8 activations only (the two formats whose step 2 is the FP8 quantiser)
+  if (c->wfmt != MOE_WFMT_FP8_E4M3_B128 && c->wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32) return MOE_ERR_UNSUPPORTED;
+  if (c->gc_small) return MOE_ERR_UNSUPPORTED;  // the Green-Context partition is the other form of the split
+  int coop = 0;
+  if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c->dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (!coop) return MOE_ERR_UNSUPPORTED;
+  c->disp_ctas = dispatch_ctas;
+  return MOE_OK;
+}
+
+moe_status moe_dispatch_overlap_ctas(moe_ctx* c, int* dispatch_ctas) {
+  if (!c || !dispatch_ctas) return MOE_ERR_INVALID_ARG;
+  *dispatch_ctas = c->disp_ctas;
+  return MOE_OK;
+}
+
 moe_status moe_set_fault_injection(moe_ctx* c, int mode) {
-  if (!c || mode < 0 || mode > 1) return MOE_ERR_INVALID_ARG;
+  if (!c || mode < 0 || mode > 2) return MOE_ERR_INVALID_ARG;
   c->inject = mode;
   return MOE_OK;
 }

@@ -40,6 +40,7 @@
 // not powers of two and so cannot be fed to the block-scaled MMA.
 #include <cuda_bf16.h>
 
+#include "moe_dispatch.cuh"
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
 
@@ -162,7 +163,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int KIND, int BN, int WFMT, int NT>
+// DISP: the GEMM1 launch with dispatch overlap (moe_dispatch.cuh); the other
+// instantiations hold none of its code.
+template <int KIND, int BN, int WFMT, int NT, bool DISP>
 __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     moe_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmS, const GemmParams p) {
@@ -201,6 +204,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = p.kblocks;
+  // dispatch overlap: launched as a programmatic dependent of the route
+  // kernel, whose tile list and counts it needs from the start
+  if constexpr (DISP) griddep_wait();
   const int num_tiles = *p.num_tiles;
   const int rows_e = (KIND == 1) ? 2 * p.I : p.H;      // weight rows per expert
   constexpr int CT = (KIND == 1) ? NA / 2 : NA;        // 128-channel output tiles per unit
@@ -276,6 +282,22 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     constexpr int NPEND = (STAGES + C::NPROD - 1) / C::NPROD;
     int npend = 0;
     int pend_kb[NPEND], pend_p0[NPEND], pend_st[NPEND];
+    // Dispatch overlap: the kernel follows the route kernel in plain stream
+    // order, and a token tile is loaded once its group's ready counter is
+    // complete (the load is issued even after that wait ran out, so that
+    // the stage completes and the pipeline drains; the call then reports
+    // MOE_ERR_TIMEOUT).
+    constexpr int NPD = DISP ? NPEND : 1;
+    int pend_e[NPD], pend_ti[NPD];
+    int ready_ti = -1;  // token lane: the last tile whose group was seen ready
+    auto tokens_ready = [&](int e, int ti) {
+      if constexpr (DISP) {
+        if (ti != ready_ti) {
+          dispatch_ready(p, e, abort);
+          ready_ti = ti;
+        }
+      }
+    };
     // token tile of K block kb at positions p0.. (NVFP4: plus the block-code
     // atoms of its two MMA steps, rows ks * scale_ld + p0 .. + 31)
     auto load_tokens = [&](int st, int kb, int p0) {
@@ -300,7 +322,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
         const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
         if (tok_lane && !waited && it >= STAGES) {
           griddep_wait();
-          for (int i = 0; i < npend; ++i) load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
+          for (int i = 0; i < npend; ++i) {
+            if constexpr (DISP) tokens_ready(pend_e[i], pend_ti[i]);
+            load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
+          }
           waited = true;
         }
         if (lane == 0 && ok && it >= STAGES) {  // the stage's previous iteration has been consumed
@@ -329,11 +354,16 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
             }
           } else if (tok_lane) {
             if (waited) {
+              tokens_ready(e, ti);
               load_tokens(stage, kb, p0);
             } else {
               pend_kb[npend] = kb;
               pend_p0[npend] = p0;
               pend_st[npend] = stage;
+              if constexpr (DISP) {
+                pend_e[npend] = e;
+                pend_ti[npend] = ti;
+              }
               ++npend;
             }
           }
@@ -342,7 +372,10 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     }
     if (tok_lane && !waited) {
       griddep_wait();
-      for (int i = 0; i < npend; ++i) load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
+      for (int i = 0; i < npend; ++i) {
+        if constexpr (DISP) tokens_ready(pend_e[i], pend_ti[i]);
+        load_tokens(pend_st[i], pend_kb[i], pend_p0[i]);
+      }
     }
     // Without an abort every issued load was consumed by the MMA warps.  After
     // one, wait (bounded) for this warp's last loads into each stage; a later
@@ -475,6 +508,11 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     bool ok = true;
     int eit = 0;  // pipeline iteration
     griddep_wait();  // activation scales / combine buffer come from earlier kernels
+    if constexpr (DISP) {
+      // dispatch overlap: the last p.disp CTAs' epilogue warps quantise first
+      const int dc = blockIdx.x - (int)(gridDim.x - p.disp);
+      if (dc >= 0) dispatch_quant_fp8(p, dc * (C::EPI_THREADS / 32) + ew, p.disp * (C::EPI_THREADS / 32));
+    }
     // Per-unit inputs of the epilogue: the activation scales of the tile's
     // columns [KB][BN], the weight block scales [NA][KB] and (GEMM2) the
     // combine target of every column.  In GEMM1 with tiles of up to 32 tokens
@@ -482,7 +520,7 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     // the current unit's K loop (record at K block 0, scales at K block 1), so
     // a unit starts without waiting on memory.  (Doing the same in GEMM2,
     // routing slot and combine weight included, made it slower.)
-    constexpr bool PREF = BN <= 32 && KIND == 1;
+    constexpr bool PREF = BN <= 32 && KIND == 1 && !DISP;  // (dispatch overlap: scales read after the ready wait)
     constexpr int NPA = PREF ? (BN * KB_MAX + C::EPI_THREADS - 1) / C::EPI_THREADS : 1;
     auto unit_rt = [&](int uu) { return C::TILE_MAJOR ? uu % NRT : uu / num_tiles; };
     auto unit_ti = [&](int uu) { return C::TILE_MAJOR ? uu / NRT : uu % num_tiles; };
@@ -520,6 +558,9 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
       const int rt = unit_rt(u), ti = unit_ti(u);
       const int4 tile = from_regs ? tile_n : p.tiles[ti];
       const int e = tile.x, p0 = tile.y, nv = tile.z;
+      if constexpr (DISP) {
+        if (ok) ok = dispatch_ready(p, e, abort);
+      }
       if (from_regs) {
         if constexpr (!MXA) {
 #pragma unroll
@@ -786,28 +827,38 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-template <int KIND, int BN, int WFMT, int NT>
+template <int KIND, int BN, int WFMT, int NT, bool DISP = false>
 static cudaError_t set_attr() {
   using C = GemmCfg<KIND, BN, WFMT, NT>;
-  return cudaFuncSetAttribute(moe_gemm_kernel<KIND, BN, WFMT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              C::SMEM_BYTES);
+  return cudaFuncSetAttribute(moe_gemm_kernel<KIND, BN, WFMT, NT, DISP>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
 }
 
 template <int KIND, int BN, int WFMT, int NT = (KIND == 1 ? 2 : 1)>
 static cudaError_t launch(int grid, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& ts,
                           const GemmParams& p, cudaStream_t s) {
   using C = GemmCfg<KIND, BN, WFMT, NT>;
+  constexpr bool CAN_DISP = KIND == 1 && WFMT <= 1;  // FP8 activations: the dispatch-overlap variant exists
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // dispatch overlap: CTAs wait for other CTAs' ready counters, so all of
+  // them must be resident at once
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT>, ta, tb, ts, p);
+  cfg.numAttrs = p.disp ? 2 : 1;
+  if constexpr (CAN_DISP) {
+    if (p.disp) return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT, true>, ta, tb, ts, p);
+  } else {
+    if (p.disp) return cudaErrorInvalidValue;
+  }
+  return cudaLaunchKernelEx(&cfg, moe_gemm_kernel<KIND, BN, WFMT, NT, false>, ta, tb, ts, p);
 }
 
 // Weight tiles per stage with 4-bit weights: a stage of one or two 128-row
@@ -829,15 +880,19 @@ cudaError_t gemm_setup(int wfmt) {
   cudaError_t e = cudaSuccess;
 #define MOE_SET(K, B, W) \
   if (e == cudaSuccess) e = set_attr<K, B, W, (K == 1 ? 2 : 1)>();
+#define MOE_SET_DISP(B, W) \
+  if (e == cudaSuccess) e = set_attr<1, B, W, 2, true>();
 #define MOE_SET_NT(K, B, W, N) \
   if (e == cudaSuccess) e = set_attr<K, B, W, N>();
   if (wfmt == 0) {
     MOE_SET(1, 16, 0) MOE_SET(1, 32, 0) MOE_SET(1, 64, 0)
+    MOE_SET_DISP(16, 0) MOE_SET_DISP(32, 0) MOE_SET_DISP(64, 0)
     MOE_SET(2, 16, 0) MOE_SET(2, 32, 0) MOE_SET(2, 64, 0)
     MOE_SET_NT(2, 16, 0, 2) MOE_SET_NT(2, 32, 0, 2)
     if (e == cudaSuccess) e = gemm_tm_setup();
   } else if (wfmt == 1) {
     MOE_SET(1, 16, 1) MOE_SET(1, 32, 1) MOE_SET(1, 64, 1)
+    MOE_SET_DISP(16, 1) MOE_SET_DISP(32, 1) MOE_SET_DISP(64, 1)
     MOE_SET_NT(2, 16, 1, 4) MOE_SET_NT(2, 16, 1, 2) MOE_SET(2, 16, 1)
     MOE_SET_NT(2, 32, 1, 2) MOE_SET(2, 32, 1) MOE_SET(2, 64, 1)
   } else if (wfmt == 2) {
@@ -850,6 +905,7 @@ cudaError_t gemm_setup(int wfmt) {
     MOE_SET_NT(2, 32, 3, 2) MOE_SET_NT(2, 32, 3, 1)
   }
 #undef MOE_SET
+#undef MOE_SET_DISP
 #undef MOE_SET_NT
   return e;
 }

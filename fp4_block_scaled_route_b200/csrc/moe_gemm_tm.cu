@@ -33,6 +33,7 @@
 // (setmaxnreg), which hold 128 fp32 accumulators per thread.
 #include <cuda_bf16.h>
 
+#include "moe_dispatch.cuh"
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
 
@@ -82,7 +83,9 @@ __device__ __forceinline__ void tm_drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int KIND>
+// DISP: GEMM1 launched with dispatch overlap (moe_dispatch.cuh); the other
+// instantiations hold none of its code.
+template <int KIND, bool DISP>
 __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
     moe_gemm_tm_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                        const GemmParams p) {
@@ -102,6 +105,9 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int KB = p.kblocks;
+  // dispatch overlap: launched as a programmatic dependent of the route
+  // kernel, whose tile list and counts it needs from the start
+  if constexpr (DISP) griddep_wait();
   const int num_tiles = *p.num_tiles;
   // Row tiles per token tile: GEMM1 128 channels (gate + up rows), GEMM2 256
   // output rows (the last one 128 when H is an odd multiple of 128).
@@ -152,6 +158,21 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
       constexpr int NPEND = (STAGES + C::NPROD - 1) / C::NPROD;
       int npend = 0;
       int pend_k[NPEND], pend_p0[NPEND], pend_st[NPEND];
+      constexpr int NPD = DISP ? NPEND : 1;
+      int pend_e[NPD], pend_ti[NPD];
+      // Dispatch overlap: plain stream order after the route kernel; a token
+      // tile is loaded once its group's ready counter is complete (issued
+      // even after that wait ran out, so the stage completes and the
+      // pipeline drains; the call then reports MOE_ERR_TIMEOUT).
+      int ready_ti = -1;  // lane 0: the last tile whose group was seen ready
+      auto tokens_ready = [&](int e, int ti) {
+        if constexpr (DISP) {
+          if (ti != ready_ti) {
+            dispatch_ready(p, e, abort);
+            ready_ti = ti;
+          }
+        }
+      };
       int it = 0;
       for (int u = blockIdx.x; u < total; u += gridDim.x) {
         const int ti = u / NRT, rt = u % NRT;
@@ -169,9 +190,11 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
           const uint32_t phase = (uint32_t)(it / STAGES) & 1u;
           if (lane == 0 && !waited && it >= STAGES) {
             griddep_wait();
-            for (int i = 0; i < npend; ++i)
+            for (int i = 0; i < npend; ++i) {
+              if constexpr (DISP) tokens_ready(pend_e[i], pend_ti[i]);
               tma_load_2d(&tmX, &full[pend_st[i]], smem + pend_st[i] * C::STAGE_BYTES, pend_k[i], pend_p0[i],
                           pol_a);
+            }
             waited = true;
           }
           if (lane == 0 && ok && it >= STAGES) {
@@ -194,11 +217,16 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
               tma_load_2d(&tmW, &full[stage], st + C::A_BYTES + (lane - 1) * C::W_BOX, kb * 128, wrow, pol_w);
             } else if (lane == 0) {
               if (waited) {
+                tokens_ready(e, ti);
                 tma_load_2d(&tmX, &full[stage], st, kb * 128, p0, pol_a);
               } else {
                 pend_k[npend] = kb * 128;
                 pend_p0[npend] = p0;
                 pend_st[npend] = stage;
+                if constexpr (DISP) {
+                  pend_e[npend] = e;
+                  pend_ti[npend] = ti;
+                }
                 ++npend;
               }
             }
@@ -207,8 +235,10 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
       }
       if (lane == 0 && !waited) {
         griddep_wait();
-        for (int i = 0; i < npend; ++i)
+        for (int i = 0; i < npend; ++i) {
+          if constexpr (DISP) tokens_ready(pend_e[i], pend_ti[i]);
           tma_load_2d(&tmX, &full[pend_st[i]], smem + pend_st[i] * C::STAGE_BYTES, pend_k[i], pend_p0[i], pol_a);
+        }
       }
       __syncwarp();
       if (lane == 0 && *abort)
@@ -259,6 +289,11 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
     bool ok = true;
     int eit = 0, uparity = 0;
     griddep_wait();  // activation scales / combine buffer come from earlier kernels
+    if constexpr (DISP) {
+      // dispatch overlap: the last p.disp CTAs' epilogue warps quantise first
+      const int dc = blockIdx.x - (int)(gridDim.x - p.disp);
+      if (dc >= 0) dispatch_quant_fp8(p, dc * (C::EPI_THREADS / 32) + ew, p.disp * (C::EPI_THREADS / 32));
+    }
 
     // Scale prefetch, two pipeline iterations ahead: the activation scale of
     // this thread's token and the weight block scales of its columns.
@@ -285,6 +320,9 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
       w1 = 0.0f;
       if (c.u >= total) return;
       const int rt = c.u % NRT;
+      if constexpr (DISP) {
+        if (c.kb == 0 && ok) ok = dispatch_ready(p, c.e, abort);  // the unit's activation scales
+      }
       a = p.ascale[(size_t)c.kb * ld + c.p0 + tok];
       const float* ws = p.wscale + (size_t)c.e * RB * KB + c.kb;
       if (KIND == 1) {
@@ -434,16 +472,16 @@ __global__ void __launch_bounds__(TmCfg<KIND>::THREADS, 1)
 }
 
 // ---------------------------------------------------------------------------
-template <int KIND>
+template <int KIND, bool DISP = false>
 static cudaError_t tm_set_attr() {
   using C = TmCfg<KIND>;
-  cudaError_t e = cudaFuncSetAttribute(moe_gemm_tm_kernel<KIND>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(moe_gemm_tm_kernel<KIND, DISP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // The register split (setmaxnreg) is only safe if the block is launched
   // with the registers it was laid out for.
   cudaFuncAttributes fa;
-  e = cudaFuncGetAttributes(&fa, moe_gemm_tm_kernel<KIND>);
+  e = cudaFuncGetAttributes(&fa, moe_gemm_tm_kernel<KIND, DISP>);
   if (e != cudaSuccess) return e;
   if (fa.numRegs < C::LAUNCH_REGS) return cudaErrorInvalidConfiguration;
   return cudaSuccess;
@@ -451,6 +489,7 @@ static cudaError_t tm_set_attr() {
 
 cudaError_t gemm_tm_setup() {
   cudaError_t e = tm_set_attr<1>();
+  if (e == cudaSuccess) e = tm_set_attr<1, true>();
   if (e == cudaSuccess) e = tm_set_attr<2>();
   return e;
 }
@@ -464,12 +503,21 @@ static cudaError_t tm_launch(int grid, const CUtensorMap& tw, const CUtensorMap&
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  // dispatch overlap: CTAs wait for other CTAs' ready counters, so all of
+  // them must be resident at once
+  attr[1].id = cudaLaunchAttributeCooperative;
+  attr[1].val.cooperative = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, moe_gemm_tm_kernel<KIND>, tw, tx, p);
+  cfg.numAttrs = p.disp ? 2 : 1;
+  if constexpr (KIND == 1) {
+    if (p.disp) return cudaLaunchKernelEx(&cfg, moe_gemm_tm_kernel<1, true>, tw, tx, p);
+  } else {
+    if (p.disp) return cudaErrorInvalidValue;
+  }
+  return cudaLaunchKernelEx(&cfg, moe_gemm_tm_kernel<KIND, false>, tw, tx, p);
 }
 
 cudaError_t launch_gemm1_tm(int grid, const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,

@@ -22,6 +22,7 @@ struct RouteParams {
   int4* tiles;            // (group, first position, valid rows, 0)
   int32_t* num_tiles;     // [1]
   int32_t* status;        // [1]
+  int32_t* ready;         // [E + n_shared] dispatch-overlap counters, zeroed here (null: not used)
 };
 
 struct QuantParams {
@@ -63,6 +64,21 @@ struct GemmParams {
   // scales; GEMM1 writes hq as packed E2M1 [S_pad, I/2] plus hsc block codes.
   const float* wglobal;
   uint8_t* hsc;           // GEMM1: block codes of hq (layout of QuantParams::xsc for the format)
+  // Dispatch overlap (GEMM1 with FP8 activations, one cooperative launch):
+  // the epilogue warps of the last `disp` CTAs first quantise the
+  // activations (step 2) in routing-position order and add each finished
+  // position to ready[group]; a token tile and the activation scales of
+  // group g are read only once ready[g] == counts[g].  disp = 0: the
+  // activations come from the quantisation kernel launched before.
+  int disp;
+  int32_t* ready;         // [NG] finished positions per group (zeroed by the route kernel)
+  const int32_t* counts;  // [NG]
+  const int32_t* offsets; // [NG + 1]
+  const uint16_t* x;      // bf16 [T, H]
+  uint8_t* xq;            // E4M3 [S_pad, H], written by the dispatch warps
+  float* xs;              // [H/128, scale_ld], written by the dispatch warps (= ascale)
+  float* zero_acc;        // fp32 [T, H] combine buffer the dispatch warps clear (null: none)
+  int T, NG;
 };
 
 struct CombineParams {
@@ -112,5 +128,12 @@ cudaError_t launch_gemm2_tm(int grid, const CUtensorMap& tw, const CUtensorMap& 
                             cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s);
+
+// Packed block-scale registry (moe_api.cu): device ranges written by
+// moe_pack_mxfp4_scales / moe_pack_nvfp4_scales or declared with
+// moe_declare_packed_scales, by format (MOE_WFMT_MXFP4_E2M1_E8M0_K32 for
+// E8M0 atoms, MOE_WFMT_NVFP4_E2M1_E4M3_K16 for E4M3 atoms).  True when
+// [p, p + bytes) lies inside one registered range of that format.
+bool packed_scales_known(const void* p, size_t bytes, int fmt);
 
 }  // namespace moe

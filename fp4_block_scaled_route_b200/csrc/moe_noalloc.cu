@@ -8,7 +8,9 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
+#include <mutex>
 
 #include "moe.h"
 #include "moe_internal.h"
@@ -20,25 +22,56 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MOE_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
-// Device address of g_noalloc_scratch per device (looked up once per device).
+// Device address of g_noalloc_scratch and SM count per device, written once
+// by the first call on that device under g_setup_mu and published by the
+// release store of g_setup_done[dev]; later calls read them after an acquire
+// load of that flag, so concurrent first calls from several host threads are
+// safe.
 void* g_scratch_addr[kMaxDevices] = {nullptr};
-bool g_setup_done[kMaxDevices] = {false};
 int g_num_sms[kMaxDevices] = {0};
+std::atomic<bool> g_setup_done[kMaxDevices];
+std::mutex g_setup_mu;
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+EncodeTiledFn lookup_encoder() {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    return reinterpret_cast<EncodeTiledFn>(p);
+  return nullptr;
+}
+
 EncodeTiledFn encoder() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
+  static const EncodeTiledFn fn = lookup_encoder();  // initialised once, thread-safe
   return fn;
+}
+
+// One-time set-up on device `dev`, which is current: the array's device
+// address, the SM count and the kernels' shared-memory limits.  Returns
+// MOE_OK once done; on failure nothing is published and the next call
+// tries again.
+moe_status setup_device(int dev) {
+  if (g_setup_done[dev].load(std::memory_order_acquire)) return MOE_OK;
+  std::lock_guard<std::mutex> lock(g_setup_mu);
+  if (g_setup_done[dev].load(std::memory_order_relaxed)) return MOE_OK;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (major != 10) return MOE_ERR_UNSUPPORTED;
+  void* addr = nullptr;
+  if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return MOE_ERR_CUDA;
+  int sms = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (moe::gemm_setup(MOE_WFMT_FP8_E4M3_B128) != cudaSuccess ||
+      moe::gemm_setup(MOE_WFMT_MXFP4_E2M1_E8M0_K32) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  g_scratch_addr[dev] = addr;
+  g_num_sms[dev] = sms;
+  g_setup_done[dev].store(true, std::memory_order_release);
+  return MOE_OK;
 }
 
 bool map2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t rows,
@@ -106,25 +139,16 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   if (!al(x, 16) || !al(out, 16) || !al(w13, 128) || !al(w2, 128) || !al(s13, 16) || !al(s2, 16) ||
       !al(topk_ids, 4) || !al(topk_w, 4) || !al(d_status, 4))
     return MOE_ERR_INVALID_ARG;
+  if (wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 &&
+      (!moe::packed_scales_known(s13, (size_t)(E + n_shared) * 2 * I * (H / 32), wfmt) ||
+       !moe::packed_scales_known(s2, (size_t)(E + n_shared) * H * (I / 32), wfmt)))
+    return MOE_ERR_INVALID_ARG;  // scales not in the packed layout (see moe_declare_packed_scales)
 
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_ERR_CUDA;
-  if (!g_setup_done[dev]) {
-    // One-time set-up on this device (the device is current here): the
-    // array's device address, the SM count and the kernels' smem limits.
-    int major = 0;
-    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return MOE_ERR_CUDA;
-    if (major != 10) return MOE_ERR_UNSUPPORTED;
-    void* addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_noalloc_scratch) != cudaSuccess || !addr) return MOE_ERR_CUDA;
-    if (cudaDeviceGetAttribute(&g_num_sms[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    if (moe::gemm_setup(MOE_WFMT_FP8_E4M3_B128) != cudaSuccess ||
-        moe::gemm_setup(MOE_WFMT_MXFP4_E2M1_E8M0_K32) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    g_scratch_addr[dev] = addr;
-    g_setup_done[dev] = true;
-  }
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) return MOE_ERR_CUDA;
+  if (dev >= kMaxDevices) return MOE_ERR_UNSUPPORTED;  // more GPUs than the per-device tables hold
+  const moe_status st = setup_device(dev);
+  if (st != MOE_OK) return st;
   char* b = static_cast<char*>(g_scratch_addr[dev]);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool fp8 = (wfmt == MOE_WFMT_FP8_E4M3_B128);
@@ -156,7 +180,7 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   // cleared by the quantisation kernel as in moe_forward().
   if (cudaMemsetAsync(status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
 
-  moe::RouteParams rp;
+  moe::RouteParams rp{};
   rp.T = T; rp.k = k; rp.E = E; rp.n_shared = n_shared; rp.BN = BN;
   rp.ids = topk_ids;
   rp.counts = reinterpret_cast<int32_t*>(b + cv.counts);
@@ -171,13 +195,13 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   float* acc = reinterpret_cast<float*>(b + cv.acc);
   float* xs = reinterpret_cast<float*>(b + cv.xs);
   float* hs = reinterpret_cast<float*>(b + cv.hs);
-  moe::QuantParams qp;
+  moe::QuantParams qp{};
   qp.T = T; qp.H = H; qp.k = k; qp.n_shared = n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = rp.inv; qp.xq = xq; qp.xs = xs; qp.out_acc = acc;
   qp.xs_ld = (int)S_pad;
   if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
-  moe::GemmParams g;
+  moe::GemmParams g{};
   g.H = H; g.I = I; g.k = k; g.S = T * k;
   g.kblocks = H / 128;
   g.wscale = static_cast<const float*>(s13);

@@ -332,6 +332,38 @@ __device__ __forceinline__ void griddep_launch_dependents() {
 // is visible; a no-op when this kernel was launched without overlap.
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ---- ready counters across CTAs of one launch ----------------------------------
+// A producer CTA publishes finished work with a release add on a global
+// counter; a consumer reads it with acquire loads.  Data that the consumer
+// then reads through TMA (the async proxy) is also fenced between the
+// proxies on both sides.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+__device__ __forceinline__ void red_release_add_gpu(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Bounded wait until *ctr >= target (about a second of SM clock, or until the
+// CTA's abort word is set); on running out it sets the abort word.
+__device__ __forceinline__ bool ready_wait(const int* ctr, int target, volatile int* abort) {
+  if (ld_acquire_gpu(ctr) >= target) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (ld_acquire_gpu(ctr) >= target) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitCycles) {
+      *abort = 1;
+      return false;
+    }
+    __nanosleep(100);
+  }
+}
+
 // ---- FP8 conversion --------------------------------------------------------------
 // fp32 -> E4M3 with round-to-nearest-even and saturation to +-448.
 __device__ __forceinline__ uint32_t f32_to_e4m3(float v) {
@@ -388,6 +420,27 @@ __device__ __forceinline__ uint32_t f32x4_to_e2m1x4(float v0, float v1, float v2
       : "=r"(r)
       : "f"(v0), "f"(v1), "f"(v2), "f"(v3));
   return r;
+}
+
+// Step 2 on one 128-column group held by a warp (4 consecutive bf16 values
+// per lane, `raw`): s = amax / 448 (1 for an all-zero group) and the four
+// E4M3 codes of this lane's values, round-to-nearest-even of x / s with
+// saturation (FusedDeepMoE QuantToken, E4M3 maximum in place of int8's 127).
+__device__ __forceinline__ uint32_t quant_group_e4m3(uint2 raw, float* scale) {
+  float f[4];
+  f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
+  f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+  f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
+  f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+  float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+  const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+  uint32_t packed = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) packed |= f32_to_e4m3(__fdiv_rn(f[i], sc)) << (8 * i);
+  *scale = sc;
+  return packed;
 }
 
 }  // namespace moe

@@ -40,6 +40,10 @@ __device__ __forceinline__ unsigned ballot_match(int key, int nbits) {
 }
 
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) {
+  // a GEMM1 launched with dispatch overlap may be scheduled now; it waits
+  // for this grid's completion before it reads the routing (no effect on a
+  // following kernel launched without programmatic dependence)
+  griddep_launch_dependents();
   extern __shared__ int sm[];
   const int E = p.E, NG = p.E + p.n_shared;
   const int S = p.T * p.k, P = S + p.n_shared * p.T;
@@ -51,6 +55,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   for (int i = tid; i < 32 * NG; i += kRouteThreads) wc[i] = 0;
+  if (p.ready)  // dispatch-overlap counters of the GEMM1 launch that follows
+    for (int g = tid; g < NG; g += kRouteThreads) p.ready[g] = 0;
   if (tid == 0) s_bad = 0;
   __syncthreads();
 
@@ -220,18 +226,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
   const uint16_t* xr = p.x + (size_t)t * H;
   for (int g = warp; g < HB; g += kQuantThreads / 32) {
     const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
-    float f[4];
-    f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
-    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
-    f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
-    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
-    float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-    uint32_t packed = 0;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) packed |= f32_to_e4m3(__fdiv_rn(f[i], sc)) << (8 * i);
+    float sc;
+    const uint32_t packed = quant_group_e4m3(raw, &sc);
     for (int r = 0; r < nrows; ++r) {
       *reinterpret_cast<uint32_t*>(p.xq + (size_t)rows[r] * H + g * 128 + lane * 4) = packed;
       if (lane == 0) p.xs[(size_t)g * p.xs_ld + rows[r]] = sc;

@@ -43,6 +43,7 @@ SIGNATURES = {
     "moe_finalize_bf16": (_i, [_vp, _vp, ctypes.c_longlong, _vp]),
     "moe_pack_mxfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
     "moe_pack_nvfp4_scales": (_i, [_vp, _vp, _i, _i, _vp]),
+    "moe_declare_packed_scales": (_i, [_vp, ctypes.c_longlong, _i]),
     "moe_get_routing": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_get_activations": (_i, [_vp, _vp, _vp, _vp, _vp, _vp]),
     "moe_get_block_scales": (_i, [_vp, _vp, _vp, _vp]),
@@ -55,6 +56,8 @@ SIGNATURES = {
     "moe_router_topk": (_i, [_vp, _i, _vp, _vp, _vp, _vp, _vp]),
     "moe_set_green_ctx": (_i, [_vp, _i]),
     "moe_green_ctx_sms": (_i, [_vp, ctypes.POINTER(_i), ctypes.POINTER(_i)]),
+    "moe_set_dispatch_overlap": (_i, [_vp, _i]),
+    "moe_dispatch_overlap_ctas": (_i, [_vp, ctypes.POINTER(_i)]),
     "moe_status_string": (ctypes.c_char_p, [_i]),
 }
 
@@ -139,6 +142,10 @@ def moe_pack_nvfp4_scales(src, dst, rows, K, stream) -> int:
     return lib().moe_pack_nvfp4_scales(src, dst, rows, K, stream)
 
 
+def moe_declare_packed_scales(p, nbytes, wfmt) -> int:
+    return lib().moe_declare_packed_scales(p, nbytes, wfmt)
+
+
 def moe_get_block_scales(ctx, xsc, hsc, stream) -> int:
     return lib().moe_get_block_scales(ctx, xsc, hsc, stream)
 
@@ -181,6 +188,16 @@ def moe_green_ctx_sms(ctx):
     d, g = _i(), _i()
     _check(lib().moe_green_ctx_sms(ctx, ctypes.byref(d), ctypes.byref(g)), "moe_green_ctx_sms")
     return d.value, g.value
+
+
+def moe_set_dispatch_overlap(ctx, dispatch_ctas) -> int:
+    return lib().moe_set_dispatch_overlap(ctx, dispatch_ctas)
+
+
+def moe_dispatch_overlap_ctas(ctx) -> int:
+    d = _i()
+    _check(lib().moe_dispatch_overlap_ctas(ctx, ctypes.byref(d)), "moe_dispatch_overlap_ctas")
+    return d.value
 
 
 def moe_profile_enable(ctx, on) -> int:
@@ -323,6 +340,11 @@ class MoeLayer:
         """Green-Context partition: dispatch kernels on >= dispatch_sms SMs, GEMMs on the rest (0 = off)."""
         _check(moe_set_green_ctx(self.ctx, dispatch_sms), "moe_set_green_ctx")
         return moe_green_ctx_sms(self.ctx)
+
+    def set_dispatch_overlap(self, dispatch_ctas):
+        """Dispatch overlap: the last dispatch_ctas CTAs of the GEMM1 launch quantise first (0 = off)."""
+        _check(moe_set_dispatch_overlap(self.ctx, dispatch_ctas), "moe_set_dispatch_overlap")
+        return moe_dispatch_overlap_ctas(self.ctx)
 
 
 def pack_nvfp4_scales(s, stream=None):

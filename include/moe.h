@@ -65,7 +65,12 @@ enum {
   /* w13 u8 [NE, 2I, H/2]: E2M1 nibbles, element 2c in the low nibble of byte c;
    * w2 u8 [NE, H, I/2]; scales are E8M0 (2^(e-127)) per 32 elements along K,
    * plain layout [NE, rows, K/32], converted once with moe_pack_mxfp4_scales()
-   * into the layout moe_forward() reads. */
+   * into the layout moe_forward() reads: the shared-memory image of the
+   * block-scale atoms that the tensor cores' scale copy takes, which a plain
+   * [rows, K/32] array cannot be loaded into by TMA (4 bytes per row and K
+   * block, below TMA's 16-byte minimum).  moe_forward() refuses, with
+   * MOE_ERR_INVALID_ARG, scale pointers that no moe_pack_mxfp4_scales() call
+   * wrote and no moe_declare_packed_scales() call declared. */
   MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1,
   /* NVFP4 (named among the 4-bit expert layouts of the onnxruntime QMoE
    * offload PR page; NVIDIA's definition): w13 u8 [NE, 2I, H/2] and w2 u8
@@ -74,7 +79,9 @@ enum {
    * moe_pack_nvfp4_scales(); g13 / g2 fp32 [NE] per-expert global scales.
    * Weight value = e2m1 * e4m3(scale) * g.  The tensor cores take NVFP4 only
    * with FP4 on both sides, so the activations are quantised to NVFP4 too
-   * (see moe_forward_nvfp4).  Used through moe_forward_nvfp4(). */
+   * (see moe_forward_nvfp4).  Used through moe_forward_nvfp4(), which, like
+   * moe_forward() for MXFP4, refuses scale pointers that no
+   * moe_pack_nvfp4_scales() call wrote and none was declared packed. */
   MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2,
   /* MXFP4 weights (the MOE_WFMT_MXFP4_E2M1_E8M0_K32 layout and packed scales)
    * with MXFP4 activations: x and the SwiGLU output are quantised per 32
@@ -88,8 +95,10 @@ enum {
 
 /* moe_create -- context for a layer with hidden size H, expert intermediate
  * size I, E routed experts, top-k = k, weight format wfmt (MOE_WFMT_*), no
- * shared expert, up to 4096 tokens per call.  Same as
- * moe_create_ex(H, I, E, k, wfmt, 4096, 0, out). */
+ * shared expert, up to 4096 tokens per call (the layer of the GC-MoE
+ * abstract: token dispatch to E experts, grouped GEMMs on FP8/FP4
+ * block-scaled expert weights, combine; the decode regime it targets is 1 to
+ * 256 tokens).  Same as moe_create_ex(H, I, E, k, wfmt, 4096, 0, out). */
 moe_status moe_create(int H, int I, int E, int k, int wfmt, moe_ctx** out);
 
 /* moe_create_ex -- as moe_create, with the token capacity max_T (>= 1) and
@@ -114,7 +123,14 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
  * device first).  NULL is a no-op. */
 void moe_destroy(moe_ctx* ctx);
 
-/* moe_forward -- one MoE layer.
+/* moe_forward -- one MoE layer, the step sequence of the GC-MoE abstract
+ * (dispatch, grouped GEMM1, fused SwiGLU + requantisation, grouped GEMM2,
+ * combine) with the step math of the FusedDeepMoE execution-flow page:
+ * QuantToken (per-token activation quantisation), OpDequant (accumulator x
+ * weight block scale x token scale), OpSwiglu (gate = first half of the
+ * GEMM1 rows), OpBlockQuant (requantisation of the SwiGLU output) and
+ * ReducePermute (per-token sum of the top-k expert outputs, times their
+ * weights).
  *   T          tokens, 0 <= T <= max_T (T = 0 enqueues nothing)
  *   x          device bf16 [T, H], 16-byte aligned
  *   topk_ids   device int32 [T, k]; ids outside [0, E) drop their slot and
@@ -182,6 +198,19 @@ moe_status moe_pack_mxfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
  * Weight-load-time step, asynchronous on `stream`. */
 moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int K, void* stream);
 
+/* moe_declare_packed_scales -- declares that the device range [p, p + bytes)
+ * holds block scales already in the packed layout of format wfmt
+ * (MOE_WFMT_MXFP4_E2M1_E8M0_K32 or MOE_WFMT_MXFP4_W4A4: the layout of
+ * moe_pack_mxfp4_scales(); MOE_WFMT_NVFP4_E2M1_E4M3_K16: that of
+ * moe_pack_nvfp4_scales()), for scales packed earlier and loaded from
+ * storage.  The forward entry points accept only scale pointers inside a
+ * range so declared or written by a pack call; a later pack or declaration
+ * that overlaps a range replaces it.  The record is process-wide and
+ * host-side (thread-safe); it does not follow frees, so declare again after
+ * reusing memory.  Returns MOE_ERR_INVALID_ARG for a NULL pointer, bytes <= 0
+ * or another format. */
+moe_status moe_declare_packed_scales(const void* p, long long bytes, int wfmt);
+
 /* moe_get_routing -- copies the routing of the last moe_forward() (after a
  * stream synchronisation) into caller buffers (host or device):
  *   counts  int32 [E + n_shared]     tokens per expert (shared expert: T)
@@ -224,8 +253,11 @@ moe_status moe_last_config(moe_ctx* ctx, int* tile_n, int* grid);
  * GEMM1 run out (CTA 0's first stage expects 16 bytes that never arrive), so
  * the bounded wait gives up after about a second, the kernel drains, frees
  * its tensor memory and returns, and moe_get_device_status() reports
- * MOE_ERR_TIMEOUT; that call's output is invalid.  mode 0 (default) turns
- * it off; the context stays usable.  Nothing faults, traps or hangs. */
+ * MOE_ERR_TIMEOUT; that call's output is invalid.  mode 2 (with dispatch
+ * overlap on, see moe_set_dispatch_overlap): the dispatch warps never
+ * publish routing position 0, so the consumers of its expert's ready counter
+ * run out of time the same way.  mode 0 (default) turns it off; the context
+ * stays usable.  Nothing faults, traps or hangs. */
 moe_status moe_set_fault_injection(moe_ctx* ctx, int mode);
 
 /* moe_router_topk -- fused router ("Mega Gate", DeepGEMM 26/09 news page:
@@ -273,6 +305,34 @@ moe_status moe_set_green_ctx(moe_ctx* ctx, int dispatch_sms);
 /* moe_green_ctx_sms -- SM counts of the current partition (0, 0 when off). */
 moe_status moe_green_ctx_sms(moe_ctx* ctx, int* dispatch_sms, int* gemm_sms);
 
+/* moe_set_dispatch_overlap -- optional dispatch/GEMM overlap through ready
+ * flags, the GC-MoE abstract's split of the GPU into a small dispatch
+ * partition and a large GEMM partition whose GEMM starts on the tokens that
+ * are ready.  Green contexts cannot carry it here: a kernel that spins on
+ * flags another, separately launched kernel sets may wait on work that is
+ * never scheduled beside it.  So both partitions are CTAs of ONE cooperative
+ * launch (all CTAs resident at once): with dispatch_ctas > 0, every
+ * following moe_forward() / moe_forward_partial() on this context launches
+ * no quantisation kernel; instead the epilogue warps of the last
+ * dispatch_ctas CTAs of the GEMM1 grid (one CTA per SM) first quantise the
+ * activations (step 2, bit for bit the quantisation kernel's codes) in
+ * routing-position order and add each finished position to its expert's
+ * ready counter (release), then take their GEMM1 work; every CTA streams its
+ * weight tiles from the start and loads an expert's token tile and scales
+ * once that counter reaches the expert's token count (acquire; bounded wait,
+ * MOE_ERR_TIMEOUT in the device status when it runs out).  The route kernel
+ * clears the counters.  1 <= dispatch_ctas <= the SM count; 0 turns it off
+ * (the default; the environment variable MOE_DISPATCH_CTAS=<n> sets it at
+ * create time).  FP8 activations only (MOE_WFMT_FP8_E4M3_B128 and
+ * MOE_WFMT_MXFP4_E2M1_E8M0_K32; other contexts: MOE_ERR_UNSUPPORTED), not
+ * together with moe_set_green_ctx (MOE_ERR_UNSUPPORTED), and the GPU must
+ * support cooperative launches.  The profiling stage MOE_STAGE_QUANT then
+ * measures zero.  A measured option: the library's default is off. */
+moe_status moe_set_dispatch_overlap(moe_ctx* ctx, int dispatch_ctas);
+
+/* moe_dispatch_overlap_ctas -- the dispatch CTA count in use (0 when off). */
+moe_status moe_dispatch_overlap_ctas(moe_ctx* ctx, int* dispatch_ctas);
+
 /* Kernel stages of one moe_forward(), in launch order (profiling index). */
 enum {
   MOE_STAGE_ROUTE = 0,     /* counts, prefix sum, permutation, tile list */
@@ -307,7 +367,11 @@ moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
  * array of MOE_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
  * keeps until the process exits.  The method's sources describe no
  * counterpart of this entry point; it exists only for such callers.
- *   H, I, E, k, wfmt, n_shared   the layer, as in moe_create_ex()
+ *   H, I, E, k, n_shared   the layer, as in moe_create_ex()
+ *   wfmt       MOE_WFMT_FP8_E4M3_B128 or MOE_WFMT_MXFP4_E2M1_E8M0_K32 (scales
+ *              packed with moe_pack_mxfp4_scales()); the two formats with
+ *              4-bit activations (NVFP4, MXFP4_W4A4) return
+ *              MOE_ERR_UNSUPPORTED
  *   T, x, topk_ids, topk_w, w13, s13, w2, s2, out   as in moe_forward()
  *   d_status   optional device int32 (caller memory): cleared, then receives
  *              the device status bits of this call (1 = expert id out of
@@ -319,7 +383,10 @@ moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
  * MOE_ERR_UNSUPPORTED before any device work.
  * The first call on a device performs a one-time set-up on the current
  * device (looks up the array's device address, sets kernel attributes);
- * make that first call before any stream capture.  Every call, on every
+ * make that first call before any stream capture.  That set-up is
+ * thread-safe: host threads making their first calls at the same time
+ * wait for one another.  A device index of 64 or more returns
+ * MOE_ERR_UNSUPPORTED.  Every call, on every
  * stream, shares the one array and leaves its contents behind: calls whose
  * execution overlaps on the GPU race and corrupt each other's results, so
  * order them (one stream, or events). */

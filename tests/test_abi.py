@@ -88,3 +88,13 @@ def test_every_entry_point_is_documented():
     assert len(decls) == len(declared_symbols())
     for m in decls:
         assert src[:m.start()].rstrip().endswith("*/"), m.group(2)
+
+
+def test_declare_packed_scales_arguments():
+    """Host-only bookkeeping: argument checks of moe_declare_packed_scales."""
+    from fp4_block_scaled_route_b200 import moe
+    assert moe.moe_declare_packed_scales(None, 64, 1) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_declare_packed_scales(4096, 0, 1) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_declare_packed_scales(4096, 64, 0) == moe.MOE_ERR_INVALID_ARG   # FP8 has no packed scales
+    for fmt in (1, 2, 3):
+        assert moe.moe_declare_packed_scales(4096 * (fmt + 1), 512, fmt) == moe.MOE_OK

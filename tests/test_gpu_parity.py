@@ -308,3 +308,36 @@ def test_mxfp4_weight_tiles_per_stage(name, bn, cfg, monkeypatch):
     assert layer.last_config()[0] == int(bn)
     assert layer.device_status() == moe.MOE_OK
     assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], name)
+
+
+# ---- 4-bit scales: only the packed layout is accepted ---------------------------
+def test_mxfp4_refuses_scales_not_packed():
+    """moe_forward with MXFP4 weights refuses scale buffers that no pack call
+    wrote (plain [rows, K/32] scales would give wrong results silently), and
+    accepts them once declared packed."""
+    L = synth.make_layer(dict(T=6, H=256, I=256, E=4, k=2, wfmt=1), 64, device="cuda")
+    layer = moe.MoeLayer(L.H, L.I, L.E, L.k, 1, max_T=8)
+    out = torch.empty(L.T, L.H, dtype=torch.bfloat16, device="cuda")
+    st = torch.cuda.current_stream().cuda_stream
+    w13, s13, w2, s2 = gpu_weights(L)
+    plain13, plain2 = L.s13.clone(), L.s2.clone()
+
+    def call(a13, a2):
+        return moe.moe_forward(layer.ctx, L.T, L.x.data_ptr(), L.ids.data_ptr(), L.topk_w.data_ptr(),
+                               w13.data_ptr(), a13.data_ptr(), w2.data_ptr(), a2.data_ptr(), out.data_ptr(), st)
+
+    assert call(plain13, s2) == moe.MOE_ERR_INVALID_ARG
+    assert call(s13, plain2) == moe.MOE_ERR_INVALID_ARG
+    assert call(s13, s2) == moe.MOE_OK
+    torch.cuda.synchronize()
+    assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], "packed")
+    # a copy of packed scales (as if loaded from storage) is accepted once declared
+    c13, c2 = s13.clone(), s2.clone()
+    assert call(c13, c2) == moe.MOE_ERR_INVALID_ARG
+    assert moe.moe_declare_packed_scales(c13.data_ptr(), c13.numel(), 1) == moe.MOE_OK
+    assert moe.moe_declare_packed_scales(c2.data_ptr(), c2.numel(), 1) == moe.MOE_OK
+    out.zero_()
+    assert call(c13, c2) == moe.MOE_OK
+    torch.cuda.synchronize()
+    assert_close(bf16_to_f32(out), oracle_full(L)["out_f32"], "declared")
+    assert layer.device_status() == moe.MOE_OK

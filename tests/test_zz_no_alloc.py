@@ -38,11 +38,23 @@ def test_noalloc_rejects_shapes_beyond_the_scratch():
     rc = moe.moe_forward_noalloc(100, 2048, 256, 8, 0, 0, 4, None, None, None, None, None, None, None,
                                  None, None, None)
     assert rc == moe.MOE_ERR_UNSUPPORTED
+    # the formats with 4-bit activations are not offered here
+    for wfmt in (moe.MOE_WFMT_NVFP4_E2M1_E4M3_K16, moe.MOE_WFMT_MXFP4_W4A4):
+        rc = moe.moe_forward_noalloc(512, 256, 8, 2, wfmt, 0, 4, None, None, None, None, None, None, None,
+                                     None, None, None)
+        assert rc == moe.MOE_ERR_UNSUPPORTED
 
 
+# Each case reaches one token-tile width, which this entry point chooses and
+# builds tensor maps for on its own: 16 (decode), 32, 64 (FP8 and MXFP4) and
+# the 128-token token-major kernel (FP8).
 CASES = [
     ("decode_fp8_T32_H7168_E256_k8_I2048", dict(T=32, H=7168, E=256, k=8, I=2048, wfmt=0), 501),
     ("mxfp4_shared_T12_H512_E8_k2_I256", dict(T=12, H=512, E=8, k=2, I=256, wfmt=1, n_shared=1), 502),
+    ("fp8_bn32_T48_H512_E8_k2_I256", dict(T=48, H=512, E=8, k=2, I=256, wfmt=0), 503),
+    ("fp8_bn64_T120_H512_E8_k2_I256", dict(T=120, H=512, E=8, k=2, I=256, wfmt=0), 504),
+    ("fp8_bn128_T1024_H512_E8_k2_I256", dict(T=1024, H=512, E=8, k=2, I=256, wfmt=0), 505),
+    ("mxfp4_bn64_T160_H512_E8_k2_I256", dict(T=160, H=512, E=8, k=2, I=256, wfmt=1), 506),
 ]
 
 
