@@ -27,6 +27,8 @@ weights = softmax over the k chosen of N(0,1) logits (fp32); expert weights
 ~ N(0, 0.02), stored as FP8 E4M3 with one fp32 scale amax/448 per 128x128
 block, or as MXFP4 (E2M1 nibbles, element 2c in the low nibble, one E8M0
 scale per 32 elements along K with exponent floor(log2 amax) - 2), or as
+MXFP8 (E4M3 codes, one E8M0 scale per 32 elements along K with exponent
+floor(log2 amax) - 8, elements saturated at 448), or as
 NVFP4 (the same nibbles, one E4M3 scale per 16 elements along K and one fp32
 global scale per expert matrix: g = amax / (448 * 6), block scale
 e4m3(amax16 / 6 / g), element e2m1(w / (block scale * g))).
@@ -46,6 +48,7 @@ WFMT_FP8 = 0
 WFMT_MXFP4 = 1
 WFMT_NVFP4 = 2
 WFMT_MXFP4_A4 = 3  # MXFP4 weights (the WFMT_MXFP4 bytes) with MXFP4 activations
+WFMT_MXFP8 = 4     # MXFP8: E4M3 weights and activations, E8M0 scale per 32 along K
 
 CONFIGS = [
     dict(name="tiny_T4_H256_E8_k2_I128_fp8", T=4, H=256, E=8, k=2, I=128,
@@ -138,6 +141,18 @@ def _mxfp4_group(w: torch.Tensor):
     return packed.contiguous(), (e + 127).to(torch.uint8)
 
 
+def _mxfp8_group(w: torch.Tensor):
+    """w f32 [R, K] -> (E4M3 codes uint8 [R, K], e8m0 uint8 [R, K/32])."""
+    R, K = w.shape
+    grp = w.reshape(R, K // 32, 32)
+    amax = grp.abs().amax(dim=2)
+    e = torch.floor(torch.log2(amax)) - 8.0           # OCP MX: emax(E4M3) = 8
+    e = e.clamp(-127, 127)
+    scaled = (grp / torch.exp2(e)[:, :, None]).clamp(-448.0, 448.0)  # the cast does not saturate
+    codes = scaled.to(torch.float8_e4m3fn).view(torch.uint8).reshape(R, K)
+    return codes.contiguous(), (e + 127).to(torch.uint8)
+
+
 def _nvfp4_matrix(w: torch.Tensor):
     """w f32 [R, K] -> (packed uint8 [R, K/2], E4M3 block codes uint8 [R, K/16], g f32 scalar)."""
     R, K = w.shape
@@ -170,6 +185,9 @@ def make_weights(NE: int, rows: int, K: int, wfmt: int, gen: torch.Generator, de
     if wfmt == WFMT_FP8:
         w = torch.empty(NE, rows, K, dtype=torch.uint8, device=device)
         s = torch.empty(NE, rows // 128, K // 128, dtype=torch.float32, device=device)
+    elif wfmt == WFMT_MXFP8:
+        w = torch.empty(NE, rows, K, dtype=torch.uint8, device=device)
+        s = torch.empty(NE, rows, K // 32, dtype=torch.uint8, device=device)
     else:
         w = torch.empty(NE, rows, K // 2, dtype=torch.uint8, device=device)
         s = torch.empty(NE, rows, K // 32, dtype=torch.uint8, device=device)
@@ -177,6 +195,8 @@ def make_weights(NE: int, rows: int, K: int, wfmt: int, gen: torch.Generator, de
         dense = torch.randn(rows, K, generator=gen, device=device, dtype=torch.float32) * std
         if wfmt == WFMT_FP8:
             w[e], s[e] = _fp8_block(dense)
+        elif wfmt == WFMT_MXFP8:
+            w[e], s[e] = _mxfp8_group(dense)
         else:
             w[e], s[e] = _mxfp4_group(dense)
     return w, s

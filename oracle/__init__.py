@@ -28,6 +28,7 @@ WFMT_FP8 = 0
 WFMT_MXFP4 = 1
 WFMT_NVFP4 = 2
 WFMT_MXFP4_A4 = 3
+WFMT_MXFP8 = 4
 
 
 def build(force: bool = False) -> str:
@@ -87,6 +88,10 @@ def lib() -> ctypes.CDLL:
             L.orc_quant_row_mxfp4.argtypes = [ctypes.c_int, vp, vp, vp]
             L.orc_quant_act_mxfp4.restype = None
             L.orc_quant_act_mxfp4.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
+            L.orc_quant_row_mxfp8.restype = None
+            L.orc_quant_row_mxfp8.argtypes = [ctypes.c_int, vp, vp, vp]
+            L.orc_quant_act_mxfp8.restype = None
+            L.orc_quant_act_mxfp8.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
             L.orc_forward.restype = ctypes.c_int
             L.orc_forward.argtypes = [ctypes.POINTER(_Dims)] + [vp] * 13
             L.orc_forward_ex.restype = ctypes.c_int
@@ -232,6 +237,26 @@ def quant_act_mxfp4(x_bf16_bits: np.ndarray):
     return xq, xsc
 
 
+def quant_row_mxfp8(v: np.ndarray):
+    """fp32 row [K] -> (E4M3 codes [K], E8M0 codes [K/32])."""
+    v = _c(np.asarray(v, dtype=np.float32), np.float32)
+    K = v.shape[-1]
+    q = np.empty(K, np.uint8)
+    sc = np.empty(K // 32, np.uint8)
+    lib().orc_quant_row_mxfp8(K, _p(v), _p(q), _p(sc))
+    return q, sc
+
+
+def quant_act_mxfp8(x_bf16_bits: np.ndarray):
+    """bf16 [T,H] -> (E4M3 codes [T,H], E8M0 codes [T,H/32])."""
+    x = _c(x_bf16_bits, np.uint16)
+    T, H = x.shape
+    xq = np.empty((T, H), np.uint8)
+    xsc = np.empty((T, H // 32), np.uint8)
+    lib().orc_quant_act_mxfp8(T, H, _p(x), _p(xq), _p(xsc))
+    return xq, xsc
+
+
 def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
             n_shared=0, token_mask=None, debug=False, g13=None, g2=None):
     """Whole layer on the CPU.
@@ -274,7 +299,7 @@ def forward(x_bf16_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt,
         dbg = dict(xq=np.zeros((T, H // cw), np.uint8), xs=np.zeros((T, H // 128), np.float32),
                    hq=np.zeros((max(P, 1), I // cw), np.uint8),
                    hs=np.zeros((max(P, 1), I // 128), np.float32))
-        if a4:
+        if a4 or wfmt == WFMT_MXFP8:
             bs = 16 if nv else 32
             dbg.update(xsc=np.zeros((T, H // bs), np.uint8), hsc=np.zeros((max(P, 1), I // bs), np.uint8))
     rc = lib().orc_forward_ex(ctypes.byref(d), _p(x), _p(ids), _p(topk_w), _p(w13), _p(s13), _p(g13),

@@ -323,6 +323,43 @@ void orc_quant_act_mxfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* 
   free(row);
 }
 
+/* MXFP8 (OCP MX v1.0 with E4M3 elements): X = floor(log2(amax32)) - 8,
+ * clamped to [-127, 127] (an all-zero block: X = -127); elements
+ * e4m3(v / 2^X), which saturates at 448 where v / 2^X reaches [448, 512). */
+void orc_quant_row_mxfp8(int K, const float* v, uint8_t* q, uint8_t* sc) {
+  for (int g = 0; g < K / 32; ++g) {
+    const float* vg = v + (size_t)g * 32;
+    float amax = 0.0f;
+    int X;
+    float s;
+    for (int c = 0; c < 32; ++c) {
+      float a = fabsf(vg[c]);
+      if (a > amax) amax = a;
+    }
+    X = (amax == 0.0f) ? -127 : floor_log2f(amax) - 8;
+    if (X < -127) X = -127;
+    if (X > 127) X = 127;
+    sc[g] = (uint8_t)(X + 127);
+    s = ldexpf(1.0f, X); /* exact */
+    for (int c = 0; c < 32; ++c) q[g * 32 + c] = orc_e4m3_encode(vg[c] / s);
+  }
+}
+
+void orc_quant_act_mxfp8(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc) {
+  float* row = (float*)malloc(sizeof(float) * (size_t)H);
+  for (int t = 0; t < T; ++t) {
+    for (int c = 0; c < H; ++c) row[c] = orc_bf16_decode(x[(size_t)t * H + c]);
+    orc_quant_row_mxfp8(H, row, xq + (size_t)t * H, xsc + (size_t)t * (H / 32));
+  }
+  free(row);
+}
+
+/* One MXFP8 row (E4M3 codes + E8M0 codes per 32) -> element x 2^X values
+ * (exact in fp32). */
+static void decode_mxfp8_row(const uint8_t* q, const uint8_t* sc, int K, float* out) {
+  for (int c = 0; c < K; ++c) out[c] = orc_e4m3_decode(q[c]) * orc_e8m0_decode(sc[c / 32]);
+}
+
 /* One MXFP4 row (packed E2M1 + E8M0 codes per 32) -> element x 2^X values
  * (exact in fp32). */
 static void decode_mxfp4_row(const uint8_t* q, const uint8_t* sc, int K, float* out) {
@@ -350,6 +387,8 @@ static void decode_row(int wfmt, const uint8_t* wrow, const uint8_t* srow_e8m0, 
                        const float* e4m3_tab, float* out) {
   if (wfmt == ORC_WFMT_FP8) {
     for (int c = 0; c < K; ++c) out[c] = e4m3_tab[wrow[c]];
+  } else if (wfmt == ORC_WFMT_MXFP8) {
+    decode_mxfp8_row(wrow, srow_e8m0, K, out);
   } else if (wfmt == ORC_WFMT_NVFP4) {
     decode_nvfp4_row(wrow, srow_e8m0 /* E4M3 block codes here */, K, out);
   } else {
@@ -400,26 +439,28 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
   const int HB = H / 128, IB = I / 128;
   const int nv = (wfmt == ORC_WFMT_NVFP4);
   const int mx4 = (wfmt == ORC_WFMT_MXFP4_A4);      /* MXFP4 weights and MXFP4 activations */
+  const int mx8 = (wfmt == ORC_WFMT_MXFP8);          /* MXFP8 weights and MXFP8 activations */
   const int a4 = nv || mx4;                          /* 4-bit activations */
   const int wsc = mx4 ? ORC_WFMT_MXFP4 : wfmt;       /* weight decoding */
+  const int byte_w = (wfmt == ORC_WFMT_FP8) || mx8;  /* one byte per weight */
   const uint8_t* w13 = (const uint8_t*)w13v;
   const uint8_t* w2 = (const uint8_t*)w2v;
   /* per-expert strides in bytes (weights) */
-  const size_t w13_e = (wfmt == ORC_WFMT_FP8) ? (size_t)2 * I * H : (size_t)2 * I * H / 2;
-  const size_t w2_e = (wfmt == ORC_WFMT_FP8) ? (size_t)H * I : (size_t)H * I / 2;
-  const size_t w13_r = (wfmt == ORC_WFMT_FP8) ? (size_t)H : (size_t)H / 2;
-  const size_t w2_r = (wfmt == ORC_WFMT_FP8) ? (size_t)I : (size_t)I / 2;
+  const size_t w13_e = byte_w ? (size_t)2 * I * H : (size_t)2 * I * H / 2;
+  const size_t w2_e = byte_w ? (size_t)H * I : (size_t)H * I / 2;
+  const size_t w13_r = byte_w ? (size_t)H : (size_t)H / 2;
+  const size_t w2_r = byte_w ? (size_t)I : (size_t)I / 2;
   /* activation codes per row: E4M3 bytes, or packed E2M1 (+ block codes) */
   const size_t xq_r = a4 ? (size_t)H / 2 : (size_t)H;
   const size_t hq_r = a4 ? (size_t)I / 2 : (size_t)I;
-  const int bs = mx4 ? 32 : 16;                      /* 4-bit activations: elements per block code */
+  const int bs = (mx4 || mx8) ? 32 : 16;             /* elements per block code */
   int32_t *counts, *offsets, *perm, *inv, *cidx;
   uint8_t *xq, *xsc = NULL;
   float *xs, *xd, *Y, e4m3_tab[256];
   int dropped, ncomp = 0;
 
   if (T < 0 || H <= 0 || I <= 0 || E <= 0 || k <= 0 || H % 128 || I % 128 ||
-      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4 && wfmt != ORC_WFMT_NVFP4 && !mx4) || nsh < 0 ||
+      (wfmt != ORC_WFMT_FP8 && wfmt != ORC_WFMT_MXFP4 && wfmt != ORC_WFMT_NVFP4 && !mx4 && !mx8) || nsh < 0 ||
       nsh > 1 ||
       (nv && (!g13 || !g2)))
     return -1;
@@ -450,6 +491,13 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
     for (size_t i = 0; i < (size_t)T * HB; ++i) xs[i] = 1.0f;  /* every scale is in the codes */
     for (int t = 0; t < T; ++t)
       decode_mxfp4_row(xq + (size_t)t * xq_r, xsc + (size_t)t * (H / 32), H, xd + (size_t)t * H);
+    if (dbg_xsc) memcpy(dbg_xsc, xsc, (size_t)T * (H / 32));
+  } else if (mx8) {
+    xsc = (uint8_t*)malloc((size_t)T * (H / 32));
+    orc_quant_act_mxfp8(T, H, x, xq, xsc);
+    for (size_t i = 0; i < (size_t)T * HB; ++i) xs[i] = 1.0f;  /* every scale is in the codes */
+    for (int t = 0; t < T; ++t)
+      decode_mxfp8_row(xq + (size_t)t * xq_r, xsc + (size_t)t * (H / 32), H, xd + (size_t)t * H);
     if (dbg_xsc) memcpy(dbg_xsc, xsc, (size_t)T * (H / 32));
   } else {
     orc_quant_act(T, H, x, xq, xs);
@@ -513,7 +561,7 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
         decode_row(wsc, wr, sr, H, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           G[(size_t)i * 2 * I + r] = row_dot(H, xd + (size_t)tok[i] * H, xs + (size_t)tok[i] * HB,
-                                             wrow, wsc == ORC_WFMT_MXFP4 ? NULL : ws);
+                                             wrow, (wsc == ORC_WFMT_MXFP4 || mx8) ? NULL : ws);
       }
       free(wrow);
       free(ws);
@@ -534,6 +582,11 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
           orc_quant_row_mxfp4(I, h, hqi, hsc + (size_t)i * (I / 32));
           for (int kb = 0; kb < IB; ++kb) hs[(size_t)i * IB + kb] = 1.0f;
           decode_mxfp4_row(hqi, hsc + (size_t)i * (I / 32), I, hd + (size_t)i * I);
+          if (dbg_hsc) memcpy(dbg_hsc + (size_t)pos[i] * (I / 32), hsc + (size_t)i * (I / 32), (size_t)(I / 32));
+        } else if (mx8) {
+          orc_quant_row_mxfp8(I, h, hqi, hsc + (size_t)i * (I / 32));
+          for (int kb = 0; kb < IB; ++kb) hs[(size_t)i * IB + kb] = 1.0f;
+          decode_mxfp8_row(hqi, hsc + (size_t)i * (I / 32), I, hd + (size_t)i * I);
           if (dbg_hsc) memcpy(dbg_hsc + (size_t)pos[i] * (I / 32), hsc + (size_t)i * (I / 32), (size_t)(I / 32));
         } else {
           orc_quant_row_f32(I, h, hqi, hs + (size_t)i * IB);
@@ -567,7 +620,7 @@ int orc_forward_ex(const orc_dims* d, const uint16_t* x, const int32_t* ids,
         decode_row(wsc, wr, sr, I, e4m3_tab, wrow);
         for (int i = 0; i < n; ++i)
           Y[(size_t)cidx[pos[i]] * H + r] = row_dot(I, hd + (size_t)i * I, hs + (size_t)i * IB,
-                                                    wrow, wsc == ORC_WFMT_MXFP4 ? NULL : ws);
+                                                    wrow, (wsc == ORC_WFMT_MXFP4 || mx8) ? NULL : ws);
       }
       free(wrow);
       free(ws);

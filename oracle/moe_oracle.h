@@ -51,7 +51,7 @@
 extern "C" {
 #endif
 
-enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1, ORC_WFMT_NVFP4 = 2, ORC_WFMT_MXFP4_A4 = 3 };
+enum { ORC_WFMT_FP8 = 0, ORC_WFMT_MXFP4 = 1, ORC_WFMT_NVFP4 = 2, ORC_WFMT_MXFP4_A4 = 3, ORC_WFMT_MXFP8 = 4 };
 
 /* ---- codecs (OCP FP8 / OCP MX v1.0) ---------------------------------- */
 float   orc_e4m3_decode(uint8_t code);          /* exact value, NaN for S.1111.111 */
@@ -107,6 +107,17 @@ void orc_quant_act_nvfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* 
 void orc_quant_row_mxfp4(int K, const float* v, uint8_t* q, uint8_t* sc);
 void orc_quant_act_mxfp4(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc);
 
+/* MXFP8 form of steps 2 and 5 (OCP MX v1.0, "MX-compliant" conversion, with
+ * E4M3 elements and an E8M0 shared scale per 32 consecutive elements):
+ *   X = floor(log2(amax32)) - 8 (8 = the largest E4M3 exponent), clamped to
+ *   [-127, 127]; an all-zero block takes X = -127;
+ *   code = X + 127 (E8M0), q = e4m3(v / 2^X)  (round-to-nearest-even,
+ *   saturating at +-448).
+ * One fp32 row of K (multiple of 32) values -> q E4M3 [K] and sc E8M0 codes
+ * [K/32]. */
+void orc_quant_row_mxfp8(int K, const float* v, uint8_t* q, uint8_t* sc);
+void orc_quant_act_mxfp8(int T, int H, const uint16_t* x, uint8_t* xq, uint8_t* xsc);
+
 /* ---- steps 1-8: the whole layer -------------------------------------- */
 typedef struct {
   int T, H, I, E, k;
@@ -132,7 +143,17 @@ int orc_forward(const orc_dims* d, const uint16_t* x, const int32_t* ids,
                 float* out_f32, uint16_t* out_bf16,
                 uint8_t* dbg_xq, float* dbg_xs, uint8_t* dbg_hq, float* dbg_hs);
 
-/* All four formats.  ORC_WFMT_MXFP4_A4 takes the MXFP4 weight layout above
+/* All five formats.  ORC_WFMT_MXFP8 (E4M3 weights and activations, one E8M0
+ * scale per 32 elements along K on both operands, the OCP MXFP8 format):
+ *   w13 u8 E4M3 [NE, 2I, H], s13 u8 E8M0 [NE, 2I, H/32]
+ *   w2  u8 E4M3 [NE, H, I],  s2  u8 E8M0 [NE, H, I/32]
+ * weight value = e4m3(q) * 2^(s - 127); the activations (x and the SwiGLU
+ * output) are quantised with orc_quant_row_mxfp8; every product is then
+ * (element x 2^X) x (element x 2^X), summed per 128-wide K block in
+ * ascending k and the blocks added in ascending order with no further
+ * scale.  Its debug outputs: xq [T, H], xsc [T, H/32]; hq [P, I], hsc
+ * [P, I/32] (xs / hs unused).
+ * ORC_WFMT_MXFP4_A4 takes the MXFP4 weight layout above
  * and quantises the activations (x and the SwiGLU output) to MXFP4 with
  * orc_quant_row_mxfp4; every product is then (element x 2^X) x (element x
  * 2^X), summed per 128-wide K block in ascending k and the blocks added in

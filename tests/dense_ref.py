@@ -110,12 +110,36 @@ def quant_mxfp4(v: np.ndarray):
     return vals.reshape(a.shape), ones, q.reshape(a.shape), (X + 127).astype(np.uint8)
 
 
+def quant_mxfp8(v: np.ndarray):
+    """fp32 rows [..., K] -> (element x 2^X values float64 [..., K], unit per-128
+    scales float32 [..., K/128], E4M3 codes uint8 [..., K], E8M0 codes [..., K/32]).
+    X = floor(log2 amax32) - 8 from numpy's frexp (exact), clamped to
+    [-127, 127], -127 for an all-zero block; elements by torch's RNE cast to
+    float8_e4m3fn of v / 2^X clamped to +-448 (the cast itself does not
+    saturate)."""
+    a = np.ascontiguousarray(v, dtype=np.float32)
+    K = a.shape[-1]
+    g = a.reshape(*a.shape[:-1], K // 32, 32)
+    amax = np.abs(g).max(axis=-1)
+    _, ex = np.frexp(amax.astype(np.float64))        # amax = m * 2^ex with m in [0.5, 1)
+    X = np.where(amax == 0, -127, ex - 1 - 8)
+    X = np.clip(X, -127, 127)
+    scale = np.ldexp(1.0, X)
+    r = np.clip(g.astype(np.float64) / scale[..., None], -448.0, 448.0).astype(np.float32)
+    q = torch.from_numpy(np.ascontiguousarray(r)).to(torch.float8_e4m3fn)
+    vals = q.to(torch.float64).numpy() * scale[..., None]
+    ones = np.ones(a.shape[:-1] + (K // 128,), np.float32)
+    return vals.reshape(a.shape), ones, q.view(torch.uint8).numpy().reshape(a.shape), (X + 127).astype(np.uint8)
+
+
 def dequant_weights(w: np.ndarray, s: np.ndarray, wfmt: int, K: int) -> np.ndarray:
     """One expert's weights [R, K] as float64 code values, with the MXFP4 E8M0
     scale (NVFP4: the E4M3 block scale) folded in.  FP8 block scales and the
     NVFP4 global scale are applied separately."""
     if wfmt == 0:
         return e4m3_values(w)
+    if wfmt == 4:  # MXFP8: E4M3 elements, E8M0 scale per 32
+        return e4m3_values(w) * np.repeat(np.exp2(s.astype(np.float64) - 127.0), 32, axis=1)
     vals = _E2M1_ARR[unpack_e2m1(w, K)]
     if wfmt == 2:
         return vals * np.repeat(e4m3_values(s), 16, axis=1)
@@ -140,6 +164,12 @@ def grouped_gemm(ad: np.ndarray, as_: np.ndarray, wd: np.ndarray, ws, wfmt: int,
 
 def expert_ffn(xd, xs, w13, s13, w2, s2, wfmt, H, I, g13=None, g2=None):
     """Tokens of one expert: quantised activations -> fp64 expert output [n,H]."""
+    if wfmt == 4:  # MXFP8: every scale is folded into the values on both sides
+        G = grouped_gemm(xd, xs, dequant_weights(w13, s13, 4, H), s13, 1)
+        g, u = G[:, :I], G[:, I:]
+        h = g / (1.0 + np.exp(-g)) * u
+        hd, hs = quant_mxfp8(h.astype(np.float32))[:2]
+        return grouped_gemm(hd, hs, dequant_weights(w2, s2, 4, I), s2, 1)
     if wfmt == 3:  # MXFP4 weights: the E8M0 scales are folded in by dequant_weights
         wfmt_w = 1
         G = grouped_gemm(xd, xs, dequant_weights(w13, s13, 1, H), s13, 1)
@@ -162,7 +192,8 @@ def expert_ffn(xd, xs, w13, s13, w2, s2, wfmt, H, I, g13=None, g2=None):
 def moe_layer(x_bits, ids, topk_w, w13, s13, w2, s2, *, H, I, E, wfmt, n_shared=0, g13=None, g2=None):
     """Whole layer, token by token and slot by slot, in fp64."""
     x = (x_bits.astype(np.uint32) << 16).view(np.float32)
-    xd, xs = quant_nvfp4(x)[:2] if wfmt == 2 else quant_mxfp4(x)[:2] if wfmt == 3 else quant128(x)
+    xd, xs = (quant_nvfp4(x)[:2] if wfmt == 2 else quant_mxfp4(x)[:2] if wfmt == 3
+              else quant_mxfp8(x)[:2] if wfmt == 4 else quant128(x))
     T, k = ids.shape
     out = np.zeros((T, H), dtype=np.float64)
 

@@ -46,6 +46,11 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
     s13_bytes = sizeof(float) * NE * (2 * I / 128) * (H / 128);
     w2_bytes = (size_t)NE * H * I;
     s2_bytes = sizeof(float) * NE * (H / 128) * (I / 128);
+  } else if (wfmt == ORC_WFMT_MXFP8) {
+    w13_bytes = (size_t)NE * 2 * I * H;
+    s13_bytes = (size_t)NE * 2 * I * (H / 32);
+    w2_bytes = (size_t)NE * H * I;
+    s2_bytes = (size_t)NE * H * (I / 32);
   } else if (wfmt == ORC_WFMT_NVFP4) {
     w13_bytes = (size_t)NE * 2 * I * H / 2;
     s13_bytes = (size_t)NE * 2 * I * (H / 16);
@@ -85,13 +90,13 @@ static int run_layer(int T, int H, int I, int E, int k, int wfmt, int n_shared, 
   float* out = malloc(sizeof(float) * T * H);
   uint16_t* outb = malloc(sizeof(uint16_t) * T * H);
   uint8_t* xq = malloc((size_t)T * H);
-  uint8_t* xsc = malloc((size_t)T * (H / 16));
+  uint8_t* xsc = malloc((size_t)T * (H / 16));  /* the largest block-code count (16 per code) */
   float* xs = malloc(sizeof(float) * T * (H / 128));
   uint8_t* hq = malloc(P * I + 1);
   uint8_t* hsc = malloc(P * (I / 16) + 1);
   float* hs = malloc(sizeof(float) * (P * (I / 128) + 1));
   orc_dims d = {T, H, I, E, k, wfmt, n_shared};
-  const int dropped = (wfmt == ORC_WFMT_NVFP4 || wfmt == ORC_WFMT_MXFP4_A4)
+  const int dropped = (wfmt == ORC_WFMT_NVFP4 || wfmt == ORC_WFMT_MXFP4_A4 || wfmt == ORC_WFMT_MXFP8)
       ? orc_forward_ex(&d, x, ids, w, w13, s13, g13, w2, s2, g2, NULL, out, outb, xq, xsc, xs, hq, hsc, hs)
       : orc_forward(&d, x, ids, w, w13, s13, w2, s2, NULL, out, outb, xq, xs, hq, hs);
   int ok = dropped == (bad_ids && S > 2 ? 2 : 0) && check_finite(out, (size_t)T * H);
@@ -129,6 +134,8 @@ int main(void) {
   ok &= run_layer(5, 256, 128, 6, 2, ORC_WFMT_NVFP4, 1, 1);
   ok &= run_layer(2, 384, 256, 3, 3, ORC_WFMT_NVFP4, 0, 0);
   ok &= run_layer(4, 256, 128, 5, 2, ORC_WFMT_MXFP4_A4, 1, 1);
+  ok &= run_layer(5, 256, 128, 6, 2, ORC_WFMT_MXFP8, 1, 1);
+  ok &= run_layer(2, 384, 256, 3, 3, ORC_WFMT_MXFP8, 0, 0);
   ok &= run_router(9, 256, 16, 4);
   ok &= run_router(2, 128, 8, 8);
   uint8_t codes[256];
