@@ -57,9 +57,9 @@ def parse():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", type=int, default=1,
                     help="index into synth.CONFIGS (0-4), then synth.EXTRA_CONFIGS (5: NVFP4 T=128, 6: NVFP4 T=32, "
-                         "7: MXFP4 weights and activations T=128)")
+                         "7: MXFP4 weights and activations T=128, 8: MXFP8 prefill T=4096)")
     ap.add_argument("--shape", default=None,
-                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4|nvfp4|mxfp4a4) instead of --workload")
+                    help="custom layer T,H,E,k,I,fmt[,n_shared] (fmt fp8|mxfp4|nvfp4|mxfp4a4|mxfp8) instead of --workload")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -191,8 +191,10 @@ def gpu_uuid(dev):
 
 
 # ---------------------------------------------------------------------------
-WFMT_NAMES = ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32", "nvfp4_e2m1_e4m3_k16", "mxfp4_w4a4_e2m1_e8m0_k32"]
-DTYPES = ["fp8_e4m3", "mxfp4_e2m1 x fp8_e4m3", "nvfp4_e2m1 x nvfp4_e2m1", "mxfp4_e2m1 x mxfp4_e2m1"]
+WFMT_NAMES = ["fp8_e4m3_b128", "mxfp4_e2m1_e8m0_k32", "nvfp4_e2m1_e4m3_k16", "mxfp4_w4a4_e2m1_e8m0_k32",
+              "mxfp8_e4m3_e8m0_k32"]
+DTYPES = ["fp8_e4m3", "mxfp4_e2m1 x fp8_e4m3", "nvfp4_e2m1 x nvfp4_e2m1", "mxfp4_e2m1 x mxfp4_e2m1",
+          "mxfp8_e4m3 x mxfp8_e4m3"]
 
 
 def weight_bytes_per_expert(L) -> int:
@@ -201,6 +203,8 @@ def weight_bytes_per_expert(L) -> int:
         return 2 * I * H + (2 * I // 128) * (H // 128) * 4 + H * I + (H // 128) * (I // 128) * 4
     if L.wfmt == 2:  # E2M1 nibbles, one E4M3 code per 16, one fp32 global scale per matrix
         return 2 * I * H // 2 + 2 * I * H // 16 + 4 + H * I // 2 + H * I // 16 + 4
+    if L.wfmt == 4:  # E4M3 bytes, one E8M0 code per 32
+        return 2 * I * H + 2 * I * H // 32 + H * I + H * I // 32
     return 2 * I * H // 2 + 2 * I * H // 32 + H * I // 2 + H * I // 32
 
 
@@ -210,6 +214,8 @@ def gemm1_weight_bytes_per_expert(L) -> int:
         return 2 * I * H + (2 * I // 128) * (H // 128) * 4
     if L.wfmt == 2:
         return 2 * I * H // 2 + 2 * I * H // 16 + 4
+    if L.wfmt == 4:
+        return 2 * I * H + 2 * I * H // 32
     return 2 * I * H // 2 + 2 * I * H // 32
 
 
@@ -227,6 +233,8 @@ def workload_stats(L, ids_np):
         act = P * (L.H // 2 + L.H // 16 + (L.H // 128) * 4 + L.I // 2 + L.I // 16 + (L.I // 128) * 4)
     elif L.wfmt == 3:  # activations in and out as MXFP4: nibbles and E8M0 codes
         act = P * (L.H // 2 + L.H // 32 + L.I // 2 + L.I // 32)
+    elif L.wfmt == 4:  # activations in and out as MXFP8: bytes and E8M0 codes
+        act = P * (L.H + L.H // 32 + L.I + L.I // 32)
     else:
         act = P * L.H + P * (L.H // 128) * 4 + P * L.I + P * (L.I // 128) * 4
     g1 = n_exp * gemm1_weight_bytes_per_expert(L) + act
@@ -239,7 +247,7 @@ def build_layer(args, device):
         f = args.shape.split(",")
         T, H, E, k, I = (int(v) for v in f[:5])
         wfmt = {"fp8": synth.WFMT_FP8, "mxfp4": synth.WFMT_MXFP4, "nvfp4": synth.WFMT_NVFP4,
-                "mxfp4a4": synth.WFMT_MXFP4_A4}[f[5]]
+                "mxfp4a4": synth.WFMT_MXFP4_A4, "mxfp8": synth.WFMT_MXFP8}[f[5]]
         nsh = int(f[6]) if len(f) > 6 else 0
         cfg = dict(name=f"custom_T{T}_H{H}_E{E}_k{k}_I{I}_{f[5]}" + ("_shared" if nsh else ""), T=T, H=H, E=E,
                    k=k, I=I, wfmt=wfmt, routing="uniform", n_shared=nsh)
@@ -254,7 +262,7 @@ def gpu_operands(L):
     """The layer's weights in the form moe_forward reads (MXFP4 / NVFP4 scales
     packed once, as at weight-load time) and the NVFP4 global scales."""
     from fp4_block_scaled_route_b200 import moe, synth
-    if L.wfmt in (synth.WFMT_MXFP4, synth.WFMT_MXFP4_A4):
+    if L.wfmt in (synth.WFMT_MXFP4, synth.WFMT_MXFP4_A4, synth.WFMT_MXFP8):  # E8M0 atoms
         w = (L.w13, moe.pack_mxfp4_scales(L.s13), L.w2, moe.pack_mxfp4_scales(L.s2))
     elif L.wfmt == synth.WFMT_NVFP4:
         w = (L.w13, moe.pack_nvfp4_scales(L.s13), L.w2, moe.pack_nvfp4_scales(L.s2))
@@ -646,7 +654,7 @@ def main():
     g1_tflops = g1_flops / (g1_ms * 1e-3) / 1e12 if g1_ms > 0 else None
     ratio = 4.0 if L.wfmt in (synth.WFMT_NVFP4, synth.WFMT_MXFP4_A4) else 2.0
     fp8_peak = ratio * bf16_peak
-    req = {synth.WFMT_NVFP4: "NVFP4", synth.WFMT_MXFP4_A4: "MXFP4"}.get(L.wfmt, "FP8")
+    req = {synth.WFMT_NVFP4: "NVFP4", synth.WFMT_MXFP4_A4: "MXFP4", synth.WFMT_MXFP8: "MXFP8"}.get(L.wfmt, "FP8")
     roofline = {"kernel": f"GEMM1 (grouped GEMM1 + SwiGLU + {req} requant)", "bound": "hbm",
                 "achieved": g1_gbs, "peak": hbm_peak, "unit": "GB/s",
                 "frac": (g1_gbs / hbm_peak) if g1_gbs else None,

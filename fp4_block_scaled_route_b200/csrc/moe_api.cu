@@ -62,6 +62,11 @@ struct moe_ctx {
   // that quantise the activations first, and the per-group ready counters
   int disp_ctas;
   int32_t* ready;
+  // MXFP8: the first tile of each group, and the A-operand scale atoms of
+  // GEMM1 (xsf, [tiles][H/128][512]) and GEMM2 (hsf, [tiles][I/128][512])
+  int32_t* tile_off;
+  uint8_t *xsf, *hsf;
+  int max_tiles128;
 };
 
 
@@ -167,6 +172,7 @@ size_t packed_bytes(int fmt, int NE, int rows, int K) {
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
 int pick_tile_n(const moe_ctx* c, int T) {
+  if (c->wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32) return 128;  // token-major kernels only
   const double avg = (double)T * c->k / c->E;  // expected tokens per routed expert
   int bn = avg <= 8 ? 16 : avg <= 20 ? 32 : avg <= 48 ? 64 : 128;
   if (c->tile_n_override) bn = c->tile_n_override;
@@ -204,7 +210,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   if (H % 128 || I % 128 || H > 8192 || I > 8192 || E > 1024 || k > moe::kMaxK || n_shared > 1)
     return MOE_ERR_UNSUPPORTED;
   if (wfmt != MOE_WFMT_FP8_E4M3_B128 && wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 &&
-      wfmt != MOE_WFMT_MXFP4_W4A4)
+      wfmt != MOE_WFMT_MXFP4_W4A4 && wfmt != MOE_WFMT_MXFP8_E4M3_E8M0_K32)
     return MOE_ERR_UNSUPPORTED;
   if ((long long)max_T * (k + n_shared) > (1LL << 26)) return MOE_ERR_UNSUPPORTED;
 
@@ -216,7 +222,9 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
     return MOE_ERR_CUDA;
   if (major != 10) return MOE_ERR_UNSUPPORTED;
   if (!encode_fn()) return MOE_ERR_CUDA;
-  if (moe::gemm_setup(wfmt) != cudaSuccess) return MOE_ERR_CUDA;
+  // MXFP8 runs on the token-major block-scaled kernels only
+  if ((wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32 ? moe::gemm_tmx_setup() : moe::gemm_setup(wfmt)) != cudaSuccess)
+    return MOE_ERR_CUDA;
 
   moe_ctx* c = new (std::nothrow) moe_ctx();
   if (!c) return MOE_ERR_NO_MEMORY;
@@ -241,6 +249,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
         (v == 64 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 && wfmt != MOE_WFMT_MXFP4_W4A4) ||
         (v == 128 && wfmt == MOE_WFMT_FP8_E4M3_B128))
       c->tile_n_override = v;
+    if (wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32) c->tile_n_override = 0;  // 128-token tiles only
   }
 
   const size_t HB = H / 128, IB = I / 128;
@@ -257,6 +266,11 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_ntiles = take(sizeof(int32_t) * 4);
   const size_t o_status = take(sizeof(int32_t) * 4);
   const size_t o_ready = take(sizeof(int32_t) * c->NG);
+  const size_t o_tileoff = take(sizeof(int32_t) * (c->NG + 1));
+  const bool mx8 = wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32;
+  c->max_tiles128 = c->P_max / 128 + c->NG + 1;
+  const size_t o_xsf = mx8 ? take((size_t)c->max_tiles128 * HB * 512) : 0;
+  const size_t o_hsf = mx8 ? take((size_t)c->max_tiles128 * IB * 512) : 0;
   const size_t o_tiles = take(sizeof(int4) * c->max_tiles);
   const size_t o_xq = take((size_t)c->S_pad * H);
   const size_t o_hq = take((size_t)c->S_pad * I);
@@ -293,6 +307,9 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->num_tiles = reinterpret_cast<int32_t*>(b + o_ntiles);
   c->status = reinterpret_cast<int32_t*>(b + o_status);
   c->ready = reinterpret_cast<int32_t*>(b + o_ready);
+  c->tile_off = reinterpret_cast<int32_t*>(b + o_tileoff);
+  c->xsf = mx8 ? reinterpret_cast<uint8_t*>(b + o_xsf) : nullptr;
+  c->hsf = mx8 ? reinterpret_cast<uint8_t*>(b + o_hsf) : nullptr;
   c->tiles = reinterpret_cast<int4*>(b + o_tiles);
   c->xq = reinterpret_cast<uint8_t*>(b + o_xq);
   c->hq = reinterpret_cast<uint8_t*>(b + o_hq);
@@ -451,7 +468,8 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   cudaStream_t s_disp = green ? reinterpret_cast<cudaStream_t>(c->gs_small) : s;
   cudaStream_t s_gemm = green ? reinterpret_cast<cudaStream_t>(c->gs_large) : s;
   const int grid = green ? c->gc_gemm_sms : c->num_sms;
-  const bool fp8 = (c->wfmt == MOE_WFMT_FP8_E4M3_B128);
+  const bool mx8 = (c->wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32);
+  const bool fp8 = (c->wfmt == MOE_WFMT_FP8_E4M3_B128) || mx8;  // one byte per weight
 
   // weight maps (re-encoded only when the caller's pointers change)
   const CUtensorMapL2promotion wpromo = CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
@@ -519,6 +537,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   rp.ids = ids; rp.counts = c->counts; rp.offsets = c->offsets; rp.perm = c->perm; rp.inv = c->inv;
   rp.tiles = c->tiles; rp.num_tiles = c->num_tiles; rp.status = c->status;
   rp.ready = overlap ? c->ready : nullptr;
+  rp.tile_off = mx8 ? c->tile_off : nullptr;
   mark(MOE_STAGE_ROUTE);
   if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 
@@ -531,10 +550,12 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   qp.xs_ld = c->S_pad;
   qp.out_acc = rows ? nullptr : acc;
   qp.xsc = c->xsc;
+  qp.sf_atoms = c->xsf; qp.ids = ids; qp.offsets = c->offsets; qp.tile_off = c->tile_off; qp.E = c->E;
   mark(MOE_STAGE_QUANT);
   if (!overlap) {
     const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)
                            : a4  ? moe::launch_quant_mxfp4(qp, s_disp)
+                           : mx8 ? moe::launch_quant_mxfp8(qp, s_disp)
                                  : moe::launch_quant(qp, s_disp);
     if (qe != cudaSuccess) return MOE_ERR_CUDA;
   }
@@ -567,7 +588,13 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
     g.T = T; g.NG = c->NG;
   }
   mark(MOE_STAGE_GEMM1);
-  if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (mx8) {
+    g.act_sf = c->xsf;
+    g.hsc = c->hsf;
+    if (moe::launch_gemm1_tmx(grid, c->tm_w13, c->tm_xq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
 
   g.disp = 0;  // GEMM2 reads GEMM1's outputs after the kernel boundary
   g.zero_acc = nullptr;
@@ -577,7 +604,12 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   g.ascale = c->hs;
   mark(MOE_STAGE_GEMM2);
   g.y_rows = rows ? c->y_rows : nullptr;
-  if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, tsh, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  if (mx8) {
+    g.act_sf = c->hsf;
+    if (moe::launch_gemm2_tmx(grid, c->tm_w2, c->tm_hq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (moe::launch_gemm2(c->wfmt, BN, grid, c->tm_w2, c->tm_hq, tsh, g, s_gemm) != cudaSuccess) {
+    return MOE_ERR_CUDA;
+  }
 
   mark(MOE_STAGE_FINALIZE);
   if (partial) {
@@ -705,7 +737,8 @@ moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
 
 moe_status moe_declare_packed_scales(const void* p, long long bytes, int wfmt) {
   if (!p || bytes <= 0) return MOE_ERR_INVALID_ARG;
-  if (wfmt == MOE_WFMT_MXFP4_W4A4) wfmt = MOE_WFMT_MXFP4_E2M1_E8M0_K32;  // the same E8M0 atoms
+  if (wfmt == MOE_WFMT_MXFP4_W4A4 || wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32)
+    wfmt = MOE_WFMT_MXFP4_E2M1_E8M0_K32;  // the same E8M0 atoms
   if (wfmt != MOE_WFMT_MXFP4_E2M1_E8M0_K32 && wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16) return MOE_ERR_INVALID_ARG;
   register_packed(p, (size_t)bytes, wfmt);
   return MOE_OK;
@@ -762,8 +795,55 @@ moe_status moe_get_activations(moe_ctx* c, uint8_t* xq, float* xs, uint8_t* hq, 
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// MXFP8: the E8M0 codes of the last call's activations, gathered from the
+// per-tile scale atoms into [P][K/32] rows in routing-position order.
+static moe_status get_block_scales_mxfp8(moe_ctx* c, uint8_t* xsc, uint8_t* hsc, void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;
+  const int NG = c->NG;
+  const size_t P = (size_t)c->last_T * c->k + (size_t)c->n_shared * c->last_T;
+  if (!P) return MOE_OK;
+  int32_t* off = new (std::nothrow) int32_t[NG + 1];
+  int32_t* toff = new (std::nothrow) int32_t[NG + 1];
+  moe_status st = (off && toff) ? MOE_OK : MOE_ERR_NO_MEMORY;
+  if (st == MOE_OK && (cudaMemcpy(off, c->offsets, sizeof(int32_t) * (NG + 1), cudaMemcpyDeviceToHost) != cudaSuccess ||
+                       cudaMemcpy(toff, c->tile_off, sizeof(int32_t) * (NG + 1), cudaMemcpyDeviceToHost) != cudaSuccess))
+    st = MOE_ERR_CUDA;
+  auto gather = [&](uint8_t* dst, const uint8_t* atoms, int K) {
+    if (!dst || st != MOE_OK) return;
+    const int KB = K / 128;
+    const size_t nt = (size_t)toff[NG];
+    uint8_t* a = new (std::nothrow) uint8_t[nt * KB * 512 + 1];
+    uint8_t* out = new (std::nothrow) uint8_t[P * (K / 32)];
+    if (!a || !out) {
+      st = MOE_ERR_NO_MEMORY;
+    } else if (cudaMemcpy(a, atoms, nt * KB * 512, cudaMemcpyDeviceToHost) != cudaSuccess) {
+      st = MOE_ERR_CUDA;
+    } else {
+      memset(out, 0, P * (K / 32));
+      int g = 0;
+      for (size_t pos = 0; pos < (size_t)off[NG]; ++pos) {
+        while ((int)pos >= off[g + 1]) ++g;
+        const int within = (int)pos - off[g];
+        const int ti = toff[g] + within / 128, r = within % 128;
+        for (int kb = 0; kb < KB; ++kb)
+          for (int j = 0; j < 4; ++j)
+            out[pos * (K / 32) + kb * 4 + j] = a[((size_t)ti * KB + kb) * 512 + (r % 32) * 16 + (r / 32) * 4 + j];
+      }
+      if (cudaMemcpy(dst, out, P * (K / 32), cudaMemcpyDefault) != cudaSuccess) st = MOE_ERR_CUDA;
+    }
+    delete[] a;
+    delete[] out;
+  };
+  gather(xsc, c->xsf, c->H);
+  gather(hsc, c->hsf, c->I);
+  delete[] off;
+  delete[] toff;
+  return st;
+}
+
 moe_status moe_get_block_scales(moe_ctx* c, uint8_t* xsc, uint8_t* hsc, void* stream) {
   if (!c) return MOE_ERR_INVALID_ARG;
+  if (c->wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32) return get_block_scales_mxfp8(c, xsc, hsc, stream);
   if (c->wfmt != MOE_WFMT_NVFP4_E2M1_E4M3_K16 && c->wfmt != MOE_WFMT_MXFP4_W4A4) return MOE_ERR_UNSUPPORTED;
   const int code_step = (c->wfmt == MOE_WFMT_NVFP4_E2M1_E4M3_K16) ? 64 : 128;  // K columns per 4-code entry
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MOE_ERR_CUDA;

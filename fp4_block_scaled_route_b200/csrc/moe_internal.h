@@ -23,6 +23,7 @@ struct RouteParams {
   int32_t* num_tiles;     // [1]
   int32_t* status;        // [1]
   int32_t* ready;         // [E + n_shared] dispatch-overlap counters, zeroed here (null: not used)
+  int32_t* tile_off;      // [E + n_shared + 1] first tile of each group (null: not exported)
 };
 
 struct QuantParams {
@@ -42,6 +43,15 @@ struct QuantParams {
   //   MXFP4 (quant_mxfp4_kernel): E8M0 codes, [H/128][xs_ld][16], one entry
   //     per 128-column K block (its two MMA steps use bytes 0-1 and 2-3).
   uint8_t* xsc;
+  // MXFP8 (quant_mxfp8_kernel): E8M0 codes per 32 columns written straight
+  // into the MMA's A-operand scale atoms of the token-major kernel: per tile
+  // of 128 positions and 128-column K block one 512-byte atom, position row
+  // r's four codes at bytes (r % 32) * 16 + (r / 32) * 4 + 0..3.
+  uint8_t* sf_atoms;      // [tiles][H/128][512]
+  const int32_t* ids;     // [T*k] expert ids (group of a routed position)
+  const int32_t* offsets; // [NG + 1] first position of each group
+  const int32_t* tile_off;// [NG + 1] first tile of each group
+  int E;
 };
 
 struct GemmParams {
@@ -79,6 +89,10 @@ struct GemmParams {
   float* xs;              // [H/128, scale_ld], written by the dispatch warps (= ascale)
   float* zero_acc;        // fp32 [T, H] combine buffer the dispatch warps clear (null: none)
   int T, NG;
+  // MXFP8 token-major kernels (moe_gemm_tmx.cu): the A operand's E8M0
+  // scale atoms ([tiles][K/128][512], the layout of QuantParams::sf_atoms);
+  // GEMM1 writes GEMM2's into hsc in the same layout.
+  const uint8_t* act_sf;
 };
 
 struct CombineParams {
@@ -126,6 +140,13 @@ cudaError_t launch_gemm1_tm(int grid, const CUtensorMap& tw, const CUtensorMap& 
                             cudaStream_t s);
 cudaError_t launch_gemm2_tm(int grid, const CUtensorMap& tw, const CUtensorMap& th, const GemmParams& p,
                             cudaStream_t s);
+// MXFP8 token-major kernels (block-scaled MMA, no promotion), moe_gemm_tmx.cu.
+cudaError_t gemm_tmx_setup();
+cudaError_t launch_gemm1_tmx(int grid, const CUtensorMap& tw, const CUtensorMap& tx, const GemmParams& p,
+                             cudaStream_t s);
+cudaError_t launch_gemm2_tmx(int grid, const CUtensorMap& tw, const CUtensorMap& th, const GemmParams& p,
+                             cudaStream_t s);
+cudaError_t launch_quant_mxfp8(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_combine(const CombineParams& p, cudaStream_t s);
 cudaError_t launch_pack_e8m0(const uint8_t* src, uint8_t* dst, int rows, int kgroups, cudaStream_t s);
 

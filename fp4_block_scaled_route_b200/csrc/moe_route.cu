@@ -14,6 +14,7 @@
 #include <cuda_bf16.h>
 
 #include "moe_internal.h"
+#include "moe_mxfp8.cuh"
 #include "moe_ptx.cuh"
 
 namespace moe {
@@ -137,6 +138,8 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
 
   for (int g = tid; g < NG; g += kRouteThreads) p.counts[g] = cnt[g];
   for (int g = tid; g <= NG; g += kRouteThreads) p.offsets[g] = off[g];
+  if (p.tile_off)
+    for (int g = tid; g <= NG; g += kRouteThreads) p.tile_off[g] = toff[g];
 
   // pass B: stable scatter
   for (int b0 = beg; b0 < end; b0 += 32 * kRouteBatch) {
@@ -373,6 +376,71 @@ __global__ void __launch_bounds__(kQuantThreads) quant_mxfp4_kernel(QuantParams 
 
 cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s) {
   quant_mxfp4_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// MXFP8 form of step 2 (OCP MX v1.0 with E4M3 elements): per 32 columns
+// X = floor(log2 amax) - 8 (clamped to [-127, 127], -127 for an all-zero
+// block), E8M0 code X + 127, elements e4m3(v / 2^X) with round-to-nearest-
+// even and saturation.  Same grid as quant_kernel; a lane holds 4
+// consecutive columns, so a 32-column block is 8 neighbouring lanes.  Codes
+// go to every routed position of the token (rows in routing order); the
+// E8M0 codes go straight into the token-major kernel's A-operand scale
+// atoms: the position's tile ti = tile_off[g] + (pos - offsets[g]) / 128 and
+// row r = (pos - offsets[g]) % 128 within it.
+__global__ void __launch_bounds__(kQuantThreads) quant_mxfp8_kernel(QuantParams p) {
+  griddep_launch_dependents();  // GEMM1 may start its weight prefetch now
+  const int t = blockIdx.x;
+  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  __shared__ int rows[kMaxK + 1];
+  __shared__ int atom[kMaxK + 1];  // byte offset of the position's row in its tile's atoms
+  __shared__ int nrows;
+  if (threadIdx.x == 0) {
+    int n = 0;
+    for (int j = 0; j <= p.k; ++j) {
+      if (j == p.k && !p.n_shared) break;
+      const int r = (j < p.k) ? p.inv[t * p.k + j] : p.inv[S + t];
+      if (r < 0) continue;
+      const int g = (j < p.k) ? p.ids[t * p.k + j] : p.E;
+      const int within = r - p.offsets[g];
+      const int ti = p.tile_off[g] + within / 128, rr = within % 128;
+      rows[n] = r;
+      atom[n] = ti * HB * 512 + (rr % 32) * 16 + (rr / 32) * 4;
+      ++n;
+    }
+    nrows = n;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xr = p.x + (size_t)t * H;
+  for (int g = warp; g < HB; g += kQuantThreads / 32) {
+    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+    float f[4];
+    f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
+    f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
+    f[2] = __uint_as_float((raw.y & 0xFFFFu) << 16);
+    f[3] = __uint_as_float(raw.y & 0xFFFF0000u);
+    float amax = fmaxf(fmaxf(fabsf(f[0]), fabsf(f[1])), fmaxf(fabsf(f[2]), fabsf(f[3])));
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+    float sc;
+    const int X = mx_e4m3_exponent(amax, &sc);
+    const uint32_t packed = f32x2_to_e4m3x2(__fdiv_rn(f[0], sc), __fdiv_rn(f[1], sc)) |
+                            (f32x2_to_e4m3x2(__fdiv_rn(f[2], sc), __fdiv_rn(f[3], sc)) << 16);
+    for (int r = 0; r < nrows; ++r) {
+      *reinterpret_cast<uint32_t*>(p.xq + (size_t)rows[r] * H + g * 128 + lane * 4) = packed;
+      if ((lane & 7) == 0) p.sf_atoms[(size_t)atom[r] + (size_t)g * 512 + (lane >> 3)] = static_cast<uint8_t>(X + 127);
+    }
+  }
+  if (p.out_acc) {
+    float4* acc = reinterpret_cast<float4*>(p.out_acc + (size_t)t * H);
+    for (int i = threadIdx.x; i < H / 4; i += kQuantThreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+cudaError_t launch_quant_mxfp8(const QuantParams& p, cudaStream_t s) {
+  quant_mxfp8_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 

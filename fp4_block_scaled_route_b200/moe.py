@@ -29,6 +29,7 @@ MOE_WFMT_FP8_E4M3_B128 = 0
 MOE_WFMT_MXFP4_E2M1_E8M0_K32 = 1
 MOE_WFMT_NVFP4_E2M1_E4M3_K16 = 2
 MOE_WFMT_MXFP4_W4A4 = 3
+MOE_WFMT_MXFP8_E4M3_E8M0_K32 = 4
 
 # Every entry point declared in include/moe.h: name -> (restype, argtypes)
 _vp = ctypes.c_void_p

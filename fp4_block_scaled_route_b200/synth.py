@@ -34,7 +34,8 @@ global scale per expert matrix: g = amax / (448 * 6), block scale
 e4m3(amax16 / 6 / g), element e2m1(w / (block scale * g))).
 
 The NVFP4 decode workloads and an MXFP4-weights-and-activations workload
-(not rows of the table) use the decode shapes, in ``EXTRA_CONFIGS``.
+use the decode shapes, and an MXFP8 workload the prefill shape (not rows of
+the table), in ``EXTRA_CONFIGS``.
 """
 from __future__ import annotations
 
@@ -64,7 +65,8 @@ CONFIGS = [
 ]
 
 
-# Workloads beyond the five above: the NVFP4 weight format on the decode shapes.
+# Workloads beyond the five above: the NVFP4 weight format and MXFP4
+# activations on the decode shapes, and the prefill shape in MXFP8.
 EXTRA_CONFIGS = [
     dict(name="decode_T128_H7168_E256_k8_I2048_nvfp4", T=128, H=7168, E=256, k=8, I=2048,
          wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
@@ -72,6 +74,8 @@ EXTRA_CONFIGS = [
          wfmt=WFMT_NVFP4, routing="uniform", n_shared=0),
     dict(name="decode_T128_H7168_E256_k8_I2048_mxfp4_a4", T=128, H=7168, E=256, k=8, I=2048,
          wfmt=WFMT_MXFP4_A4, routing="uniform", n_shared=0),
+    dict(name="prefill_T4096_H7168_E256_k8_I2048_mxfp8", T=4096, H=7168, E=256, k=8, I=2048,
+         wfmt=WFMT_MXFP8, routing="uniform", n_shared=0),
 ]
 
 

@@ -90,7 +90,20 @@ enum {
    * tensor cores (kind::mxf4, UE8M0 scales on both operands) apply every
    * scale and no fp32 scale is promoted.  Used through moe_forward(); tiles
    * hold at most 32 tokens. */
-  MOE_WFMT_MXFP4_W4A4 = 3
+  MOE_WFMT_MXFP4_W4A4 = 3,
+  /* MXFP8 (OCP MX v1.0 with E4M3 elements; the power-of-two-scaled FP8
+   * layouts the DeepGEMM 26/09 news page names for Mega MoE): w13 u8 E4M3
+   * [NE, 2I, H], w2 u8 E4M3 [NE, H, I]; scales E8M0 (2^(e-127)) per 32
+   * elements along K, plain layout [NE, rows, K/32], converted once with
+   * moe_pack_mxfp4_scales() (the same E8M0 atom layout).  The activations
+   * (x, and the SwiGLU output) are quantised to MXFP8 per 32 columns: X =
+   * floor(log2 amax) - 8 clamped to [-127, 127] (-127 for an all-zero
+   * block), elements e4m3(v / 2^X) saturating at 448; the tensor cores
+   * (kind::mxf8f6f4 with E8M0 scales on both operands) apply every scale, so
+   * no fp32 scale is promoted and the accumulator of a whole K loop stays in
+   * tensor memory.  Used through moe_forward(); always in tiles of 128
+   * tokens (the token-major kernels). */
+  MOE_WFMT_MXFP8_E4M3_E8M0_K32 = 4
 };
 
 /* moe_create -- context for a layer with hidden size H, expert intermediate
@@ -200,7 +213,8 @@ moe_status moe_pack_nvfp4_scales(const uint8_t* src, uint8_t* dst, int rows, int
 
 /* moe_declare_packed_scales -- declares that the device range [p, p + bytes)
  * holds block scales already in the packed layout of format wfmt
- * (MOE_WFMT_MXFP4_E2M1_E8M0_K32 or MOE_WFMT_MXFP4_W4A4: the layout of
+ * (MOE_WFMT_MXFP4_E2M1_E8M0_K32, MOE_WFMT_MXFP4_W4A4 or
+ * MOE_WFMT_MXFP8_E4M3_E8M0_K32: the E8M0 atom layout of
  * moe_pack_mxfp4_scales(); MOE_WFMT_NVFP4_E2M1_E4M3_K16: that of
  * moe_pack_nvfp4_scales()), for scales packed earlier and loaded from
  * storage.  The forward entry points accept only scale pointers inside a
@@ -227,16 +241,18 @@ moe_status moe_get_routing(moe_ctx* ctx, int32_t* counts, int32_t* offsets, int3
  *   hq u8 E4M3 [P, I], hs fp32 [P, I/128]  (GEMM2 input)
  * (NVFP4 contexts: xq [P, H/2] and hq [P, I/2] packed E2M1, xs / hs the
  * per-128 scales S; MXFP4 x MXFP4 contexts: the same packed codes, xs / hs
- * unspecified.)  Rows of dropped positions are unspecified.  Any
- * pointer may be NULL. */
+ * unspecified; MXFP8 contexts: E4M3 codes as for FP8, xs / hs unspecified,
+ * the E8M0 codes through moe_get_block_scales.)  Rows of dropped positions
+ * are unspecified.  Any pointer may be NULL. */
 moe_status moe_get_activations(moe_ctx* ctx, uint8_t* xq, float* xs, uint8_t* hq, float* hs, void* stream);
 
 /* moe_get_block_scales -- contexts with 4-bit activations only (else
  * MOE_ERR_UNSUPPORTED): the block codes of the last call's activations,
  * after a stream synchronisation, rows in routing-position order.  NVFP4:
  * E4M3 codes xsc u8 [P, H/16], hsc u8 [P, I/16]; MXFP4 x MXFP4: E8M0 codes
- * xsc u8 [P, H/32], hsc u8 [P, I/32].  Either pointer may be NULL.  Debug /
- * test entry point. */
+ * xsc u8 [P, H/32], hsc u8 [P, I/32]; MXFP8: the E8M0 codes, xsc u8
+ * [P, H/32], hsc u8 [P, I/32].  Either pointer may be NULL.  Debug / test
+ * entry point. */
 moe_status moe_get_block_scales(moe_ctx* ctx, uint8_t* xsc, uint8_t* hsc, void* stream);
 
 /* moe_get_device_status -- synchronises `stream`, returns MOE_OK,

@@ -65,6 +65,8 @@ def swiglu64(L, tokens, groups):
         xd_all, xs_all = dense_ref.quant_nvfp4(x[tokens])[:2]
     elif wfmt == 3:
         xd_all, xs_all = dense_ref.quant_mxfp4(x[tokens])[:2]
+    elif wfmt == 4:
+        xd_all, xs_all = dense_ref.quant_mxfp8(x[tokens])[:2]
     else:
         xd_all, xs_all = dense_ref.quant128(x[tokens])
     h = np.zeros((len(tokens), I))
@@ -217,6 +219,24 @@ MIN_AGREEMENT = 0.9995
 SCALE_RTOL = 1e-5
 
 
+def check_mxfp8_requant(hq_g, hsc_g, hq_o, hsc_o, h64, bound):
+    """MXFP8 activations: X = floor(log2 amax32) - 8 (clamped to [-127, 127],
+    -127 for a zero block), E8M0 code X + 127, E4M3 elements of h / 2^X."""
+    n, I = h64.shape
+    amax32 = np.abs(h64).reshape(n, I // 32, 32).max(axis=2)
+    b32 = bound.reshape(n, I // 32, 32).max(axis=2)
+    X_g = hsc_g.astype(np.int64) - 127
+    lo = np.ldexp(1.0, X_g + 8)
+    hi = np.ldexp(1.0, X_g + 9)
+    ok_x = ((amax32 >= lo - b32) & (amax32 < hi + b32)) | ((X_g == -127) & (amax32 < hi + b32))
+    scale = np.repeat(np.ldexp(1.0, X_g), 32, axis=1)
+    v = h64 / scale
+    tol = bound / scale + 4 * 2.0 ** -24 * np.abs(v)
+    bad = _grid_check(v, hq_g, e4m3_values, lambda c: _signed_rank(c, 0x7F), e4m3_nearest, tol)
+    return CodeReport(agreement=float((hq_g == hq_o).mean()), block_agreement=float((hsc_g == hsc_o).mean()),
+                      violations=int(bad.sum()), block_violations=int((~ok_x).sum()))
+
+
 def check_requant(L, layer, ref, positions=None):
     """Runs the check of L's format on the routing positions `positions` (all
     by default) of the last forward of `layer`.  `ref` holds the oracle's
@@ -233,11 +253,13 @@ def check_requant(L, layer, ref, positions=None):
     if ref is None:
         # no oracle codes: compare the GPU with itself for the agreement fields
         ref = dict(hq=hq, hs=hs)
-        if L.wfmt in (2, 3):
+        if L.wfmt in (2, 3, 4):
             ref["hsc"] = layer.block_scales(T)[1]
     if L.wfmt in (0, 1):
         return check_fp8_requant(hq[pos], hs[pos], ref["hq"][pos], ref["hs"][pos], h64, bound)
     _, hsc = layer.block_scales(T)
+    if L.wfmt == 4:
+        return check_mxfp8_requant(hq[pos], hsc[pos], ref["hq"][pos], ref["hsc"][pos], h64, bound)
     if L.wfmt == 2:
         return check_nvfp4_requant(hq[pos], hsc[pos], hs[pos], ref["hq"][pos], ref["hsc"][pos], ref["hs"][pos],
                                    h64, bound)

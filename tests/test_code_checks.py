@@ -50,10 +50,11 @@ def _scale(hq, hs):
 
 
 CASES = [(dict(T=40, H=512, I=256, E=8, k=2, wfmt=0), 3), (dict(T=40, H=512, I=256, E=8, k=2, wfmt=1), 4),
-         (dict(T=20, H=512, I=384, E=8, k=2, wfmt=2, n_shared=1), 5), (dict(T=20, H=512, I=384, E=8, k=2, wfmt=3), 6)]
+         (dict(T=20, H=512, I=384, E=8, k=2, wfmt=2, n_shared=1), 5), (dict(T=20, H=512, I=384, E=8, k=2, wfmt=3), 6),
+         (dict(T=20, H=512, I=384, E=8, k=2, wfmt=4, n_shared=1), 7)]
 
 
-@pytest.mark.parametrize("cfg,seed", CASES, ids=["fp8", "mxfp4", "nvfp4_shared", "mxfp4_a4"])
+@pytest.mark.parametrize("cfg,seed", CASES, ids=["fp8", "mxfp4", "nvfp4_shared", "mxfp4_a4", "mxfp8_shared"])
 def test_checker_passes_the_oracle_and_fails_planted_defects(cfg, seed):
     L = synth.make_layer(dict(cfg, routing="uniform"), seed, device="cpu")
     g = dict(g13=L.g13.numpy(), g2=L.g2.numpy()) if L.wfmt == 2 else {}

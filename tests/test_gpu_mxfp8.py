@@ -1,0 +1,149 @@
+"""GPU parity of the MXFP8 path (MOE_WFMT_MXFP8_E4M3_E8M0_K32: E4M3 weights
+and activations with E8M0 scales per 32 on both operands, tcgen05
+kind::mxf8f6f4 block-scaled MMAs in the token-major kernels) against the
+oracle.
+
+- Routing bit for bit; activation quantisation: E4M3 codes and E8M0 codes
+  per routed position bit for bit (both sides take every decision in the
+  same fp32 operations).
+- SwiGLU-output codes and exponents: equal to the oracle's except where the
+  summation order moves a value across a rounding midpoint or a power of two
+  (tests/code_checks.py).
+- Layer outputs element by element with the layer's tolerance
+  |gpu - oracle| <= 2e-2 * max|oracle| + 1e-3 and cosine >= 0.9999; the
+  prefill-sized layer on the tokens holding every expert's first and last
+  position.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from fp4_block_scaled_route_b200 import moe, synth
+from tests import code_checks
+
+pytestmark = pytest.mark.gpu
+
+RTOL = 2e-2
+ATOL = 1e-3
+MIN_COS = 0.9999
+WFMT = moe.MOE_WFMT_MXFP8_E4M3_E8M0_K32
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    from fp4_block_scaled_route_b200 import build
+    build.build()
+    yield
+
+
+def assert_close(gpu, ref, what=""):
+    gpu = np.asarray(gpu, np.float64)
+    ref = np.asarray(ref, np.float64)
+    scale = np.abs(ref).max()
+    err = np.abs(gpu - ref).max()
+    assert err <= RTOL * scale + ATOL, f"{what}: max err {err:.3e} vs bound {RTOL * scale + ATOL:.3e}"
+    den = np.linalg.norm(gpu) * np.linalg.norm(ref)
+    cos = 1.0 if den == 0 else float((gpu * ref).sum() / den)
+    assert cos >= MIN_COS, f"{what}: cosine {cos:.6f}"
+
+
+def run_gpu(L):
+    layer = moe.MoeLayer(L.H, L.I, L.E, L.k, WFMT, max_T=max(L.T, 1), n_shared=L.n_shared)
+    out = layer.forward(L.x, L.ids, L.topk_w, L.w13, moe.pack_mxfp4_scales(L.s13), L.w2,
+                        moe.pack_mxfp4_scales(L.s2))
+    torch.cuda.synchronize()
+    return layer, out
+
+
+def oracle_ref(L, debug=False, tokens=None):
+    ids = L.ids.cpu().numpy()
+    if tokens is None:
+        return oracle.forward(synth.bf16_bits(L.x), ids, L.topk_w.cpu().numpy(), L.w13.cpu().numpy(),
+                              L.s13.cpu().numpy(), L.w2.cpu().numpy(), L.s2.cpu().numpy(), H=L.H, I=L.I, E=L.E,
+                              wfmt=WFMT, n_shared=L.n_shared, debug=debug)
+    tokens = np.asarray(tokens)
+    sub = ids[tokens]
+    used = np.unique(sub)
+    remap = np.full(L.E, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    sel = list(used) + ([L.E] if L.n_shared else [])
+    idx = torch.tensor(sel, device=L.w13.device, dtype=torch.long)
+    pick = lambda t: t.index_select(0, idx).cpu().numpy()
+    tsel = torch.tensor(tokens, device=L.x.device, dtype=torch.long)
+    return oracle.forward(synth.bf16_bits(L.x.index_select(0, tsel)), remap[sub].astype(np.int32),
+                          L.topk_w.index_select(0, tsel).cpu().numpy(), pick(L.w13), pick(L.s13), pick(L.w2),
+                          pick(L.s2), H=L.H, I=L.I, E=len(used), wfmt=WFMT, n_shared=L.n_shared)
+
+
+SMALL = [
+    ("tiny", dict(T=4, H=256, I=256, E=8, k=2), 81),
+    ("two_tiles_per_expert", dict(T=300, H=384, I=256, E=4, k=2), 82),   # ~150 positions: a short second tile
+    ("shared", dict(T=9, H=256, I=384, E=5, k=3, n_shared=1), 83),
+    ("odd_kblocks", dict(T=21, H=640, I=384, E=7, k=2), 84),            # GEMM2: a trailing 128-row W2 half tile
+    ("one_token_k8", dict(T=1, H=1024, I=512, E=32, k=8), 85),
+    ("full_tile", dict(T=256, H=512, I=256, E=2, k=1), 86),             # exactly 128 positions per expert
+]
+
+
+@pytest.mark.parametrize("name,cfg,seed", SMALL, ids=[s[0] for s in SMALL])
+def test_mxfp8_layer_small_all_elements(name, cfg, seed):
+    cfg = dict(cfg, wfmt=WFMT, routing="uniform")
+    L = synth.make_layer(cfg, seed, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.device_status() == moe.MOE_OK
+    assert layer.last_config()[0] == 128
+    ref = oracle_ref(L, debug=True)
+    assert_close(out.float().cpu().numpy(), ref["out_f32"], name)
+
+    counts, offsets, perm, inv = layer.routing(L.T)
+    rc, ro, rp, ri, _ = oracle.route(L.ids.cpu().numpy(), L.E, L.n_shared)
+    assert np.array_equal(counts, rc) and np.array_equal(perm, rp) and np.array_equal(inv, ri)
+    P = int(offsets[-1])
+    tok, _ = code_checks.position_map(perm, offsets, L.T, L.k)
+    xq, _, hq, _ = layer.activations(L.T)
+    xsc, hsc = layer.block_scales(L.T)
+    # step 2 (MXFP8): bit-exact per routed position
+    assert np.array_equal(xsc[:P], ref["xsc"][tok])
+    assert np.array_equal(xq[:P], ref["xq"][tok])
+    # SwiGLU-output codes and exponents
+    code_checks.assert_requant(code_checks.check_requant(L, layer, ref), name)
+
+
+def test_mxfp8_zero_input_and_repeated_calls():
+    L = synth.make_layer(dict(T=5, H=256, I=256, E=4, k=2, wfmt=WFMT, n_shared=1), 87, device="cuda")
+    layer = moe.MoeLayer(L.H, L.I, L.E, L.k, WFMT, max_T=8, n_shared=1)
+    s13, s2 = moe.pack_mxfp4_scales(L.s13), moe.pack_mxfp4_scales(L.s2)
+    out = layer.forward(torch.zeros_like(L.x), L.ids, L.topk_w, L.w13, s13, L.w2, s2)
+    torch.cuda.synchronize()
+    assert layer.device_status() == moe.MOE_OK
+    assert not out.float().abs().max().item()
+    ref = oracle_ref(L)["out_f32"]
+    for _ in range(2):  # the scale atoms are rewritten, not accumulated, by every call
+        out = layer.forward(L.x, L.ids, L.topk_w, L.w13, s13, L.w2, s2)
+        torch.cuda.synchronize()
+        assert layer.device_status() == moe.MOE_OK
+        assert_close(out.float().cpu().numpy(), ref, "repeated")
+
+
+def test_mxfp8_prefill_sized_layer():
+    """T=4096, H=7168, E=256, k=8, I=2048 in MXFP8, in the benchmark's launch
+    configuration: the tokens holding each expert's first and last routing
+    position (every expert's first tile and its last, short one) against the
+    oracle; every row finite; SwiGLU-output codes of a few experts' edges."""
+    cfg = next(c for c in synth.EXTRA_CONFIGS if c["wfmt"] == WFMT)
+    L = synth.make_layer(cfg, 3000, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.device_status() == moe.MOE_OK
+    counts, offsets, perm, inv = layer.routing(L.T)
+    tok, grp = code_checks.position_map(perm, offsets, L.T, L.k)
+    firsts = offsets[:-1][counts > 0]
+    lasts = offsets[1:][counts > 0] - 1
+    tokens = np.unique(np.concatenate([tok[firsts], tok[lasts], [L.T - 1]]))
+    ref = oracle_ref(L, tokens=tokens)["out_f32"]
+    assert_close(out.float().cpu().numpy()[tokens], ref, cfg["name"])
+    assert torch.isfinite(out.float()).all()
+    code_checks.assert_requant(code_checks.check_requant(L, layer, None, code_checks.edge_positions(layer, L, 4)),
+                               cfg["name"])
