@@ -1,5 +1,6 @@
 """A model of the barrier protocol of the decode GEMM kernel
-(fp4_block_scaled_route_b200/csrc/moe_gemm.cu), run under random
+(fp4_block_scaled_route_b200/csrc/moe_gemm.cu), and at the end of the file
+of the MXFP8 token-major kernel (moe_gemm_tmx.cu), run under random
 interleavings on the CPU.
 
 Agents, as in the kernel:
@@ -187,3 +188,107 @@ def test_fewer_stages_than_producers_breaks(STAGES, NBUF, NPROD):
     assert not rule_holds(STAGES, NBUF, NPROD=NPROD)
     found = [v for seed in range(400) for v in run(STAGES, NBUF, NPROD=NPROD, seed=seed)]
     assert any(v[0].startswith("second post") for v in found), found[:3]
+
+
+# ---- the MXFP8 token-major kernel (moe_gemm_tmx.cu) -------------------------------
+def run_tmx(STAGES, KB, units=5, NPROD=2, unit_barrier=True, seed=0):
+    """One random schedule of the MXFP8 kernel's protocol.  Producers as
+    above; one MMA warp takes every iteration in order and, at a unit's first
+    K block, waits for the epilogue to have read the one accumulator (tempty,
+    one phase per unit); each iteration's commit arrives on mdone[it % NMD]
+    (NMD = STAGES + 1), and the unit's last one also on the unit barrier
+    afull.  The epilogue waits once per unit, on afull (unit_barrier) or, as
+    a first version of the kernel did, on the ring barrier of the unit's last
+    iteration; then it releases the accumulator."""
+    rng = random.Random(seed)
+    NMD = STAGES + 1
+    iters = units * KB
+    full = [Barrier() for _ in range(STAGES)]
+    mdone = [Barrier() for _ in range(NMD)]
+    afull, tempty = Barrier(), Barrier()
+    landed, mma_done, violations = set(), set(), []
+    prod_next = list(range(NPROD))
+    mma_next, epi_unit = [0], [0]
+    in_flight_bytes, in_flight_mma = [], []
+
+    def epi_passes(j):
+        last = j * KB + KB - 1
+        if unit_barrier:
+            return afull.passes(j & 1)
+        return mdone[last % NMD].passes((last // NMD) & 1)
+
+    def step():
+        actions = []
+        for p in range(NPROD):
+            it = prod_next[p]
+            if it < iters and (it < STAGES or mdone[(it - STAGES) % NMD].passes(((it - STAGES) // NMD) & 1)):
+                actions.append(("prod", p))
+        it = mma_next[0]
+        if it < iters:
+            j, kb = divmod(it, KB)
+            if (kb != 0 or tempty.passes((j & 1) ^ 1)) and full[it % STAGES].passes((it // STAGES) & 1):
+                actions.append(("mma", 0))
+        if epi_unit[0] < units and epi_passes(epi_unit[0]):
+            actions.append(("epi", 0))
+        actions += [("land", i) for i in range(len(in_flight_bytes))]
+        if in_flight_mma:
+            actions.append(("commit", 0))
+        if not actions:
+            return False
+        kind, idx = rng.choice(actions)
+        if kind == "prod":
+            it = prod_next[idx]
+            b = full[it % STAGES]
+            if b.posted:
+                violations.append(("second post on an incomplete phase", it))
+            b.posted, b.pending = True, b.pending + 1
+            in_flight_bytes.append(it)
+            prod_next[idx] += NPROD
+        elif kind == "mma":
+            it = mma_next[0]
+            if it not in landed:
+                violations.append(("MMA passed its stage before the bytes landed", it))
+            in_flight_mma.append(it)
+            mma_next[0] += 1
+        elif kind == "epi":
+            j = epi_unit[0]
+            if j * KB + KB - 1 not in mma_done:
+                violations.append(("epilogue read the accumulator before the unit's MMAs completed", j))
+            tempty.arrive()
+            epi_unit[0] += 1
+        elif kind == "land":
+            it = in_flight_bytes.pop(idx)
+            b = full[it % STAGES]
+            landed.add(it)
+            b.pending -= 1
+            if b.posted and b.pending == 0:
+                b.posted = False
+                b.arrive()
+        else:
+            it = in_flight_mma.pop(0)  # one warp: commits complete in issue order
+            mma_done.add(it)
+            mdone[it % NMD].arrive()
+            if it % KB == KB - 1:
+                afull.arrive()
+        return True
+
+    for _ in range(200000):
+        if not step() or violations:
+            break
+    return violations
+
+
+@pytest.mark.parametrize("KB", [1, 2, 4, 5, 6, 8, 16])
+def test_mxfp8_kernel_keeps_the_protocol(KB):
+    """moe_gemm_tmx.cu as built: 4 stages, 2 producer warps, the unit barrier."""
+    for seed in range(100):
+        assert run_tmx(4, KB, seed=seed) == [], (KB, seed)
+
+
+def test_mxfp8_epilogue_on_the_ring_barrier_breaks_past_the_ring():
+    """With more K blocks per unit than ring slots, a parity wait on the ring
+    barrier of the unit's last iteration can pass on an earlier phase: the
+    failure the MXFP8 kernel first had (H >= 768 at 4 stages)."""
+    assert all(run_tmx(4, 5, unit_barrier=False, seed=s) == [] for s in range(100))  # within the ring: exact
+    found = [v for seed in range(200) for v in run_tmx(4, 6, unit_barrier=False, seed=seed)]
+    assert any(v[0].startswith("epilogue read") for v in found), found[:3]
