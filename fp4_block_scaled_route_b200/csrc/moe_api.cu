@@ -67,6 +67,7 @@ struct moe_ctx {
   int32_t* tile_off;
   uint8_t *xsf, *hsf;
   int max_tiles128;
+  int32_t* route_part;  // per-chunk expert counts of the multi-CTA route [kMaxRouteParts][E]
 };
 
 
@@ -267,6 +268,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   const size_t o_status = take(sizeof(int32_t) * 4);
   const size_t o_ready = take(sizeof(int32_t) * c->NG);
   const size_t o_tileoff = take(sizeof(int32_t) * (c->NG + 1));
+  const size_t o_rpart = take(sizeof(int32_t) * moe::kMaxRouteParts * E);
   const bool mx8 = wfmt == MOE_WFMT_MXFP8_E4M3_E8M0_K32;
   c->max_tiles128 = c->P_max / 128 + c->NG + 1;
   const size_t o_xsf = mx8 ? take((size_t)c->max_tiles128 * HB * 512) : 0;
@@ -308,6 +310,7 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
   c->status = reinterpret_cast<int32_t*>(b + o_status);
   c->ready = reinterpret_cast<int32_t*>(b + o_ready);
   c->tile_off = reinterpret_cast<int32_t*>(b + o_tileoff);
+  c->route_part = reinterpret_cast<int32_t*>(b + o_rpart);
   c->xsf = mx8 ? reinterpret_cast<uint8_t*>(b + o_xsf) : nullptr;
   c->hsf = mx8 ? reinterpret_cast<uint8_t*>(b + o_hsf) : nullptr;
   c->tiles = reinterpret_cast<int4*>(b + o_tiles);
@@ -538,6 +541,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   rp.tiles = c->tiles; rp.num_tiles = c->num_tiles; rp.status = c->status;
   rp.ready = overlap ? c->ready : nullptr;
   rp.tile_off = mx8 ? c->tile_off : nullptr;
+  rp.part = c->route_part;
   mark(MOE_STAGE_ROUTE);
   if (moe::launch_route(rp, s_disp) != cudaSuccess) return MOE_ERR_CUDA;
 

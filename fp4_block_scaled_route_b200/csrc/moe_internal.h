@@ -24,7 +24,13 @@ struct RouteParams {
   int32_t* status;        // [1]
   int32_t* ready;         // [E + n_shared] dispatch-overlap counters, zeroed here (null: not used)
   int32_t* tile_off;      // [E + n_shared + 1] first tile of each group (null: not exported)
+  // Multi-CTA routing for many slots: part [kMaxRouteParts][E] per-chunk
+  // expert counts (null: always one CTA).  nparts and chunk are set by
+  // launch_route.
+  int32_t* part;
+  int nparts, chunk;
 };
+constexpr int kMaxRouteParts = 64;
 
 struct QuantParams {
   int T, H, k, n_shared;

@@ -52,18 +52,23 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   int* off = cnt + NG;           // [NG + 1]
   int* toff = off + NG + 1;      // [NG + 1]
   int* wc = toff + NG + 1;       // [32][NG]: per-warp counts, then per-warp bases
+  int* cbase = wc + 32 * NG;     // [NG]: positions of each group in earlier CTAs' chunks
   __shared__ int s_bad;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  // This CTA's slots (all of them with one CTA; with several, chunk
+  // blockIdx.x of p.chunk slots, the later chunks after it in every group).
+  const bool lead = blockIdx.x == 0;
+  const int c0 = min(S, (int)blockIdx.x * p.chunk), c1 = min(S, c0 + p.chunk);
 
   for (int i = tid; i < 32 * NG; i += kRouteThreads) wc[i] = 0;
-  if (p.ready)  // dispatch-overlap counters of the GEMM1 launch that follows
+  if (p.ready && lead)  // dispatch-overlap counters of the GEMM1 launch that follows
     for (int g = tid; g < NG; g += kRouteThreads) p.ready[g] = 0;
   if (tid == 0) s_bad = 0;
   __syncthreads();
 
-  const int chunk = (((S + 31) / 32) + 31) & ~31;
+  const int chunk = ((((c1 - c0) + 31) / 32) + 31) & ~31;
   const int kbits = 32 - __clz(E);  // bits of the largest key, E (a dropped id)
-  const int beg = min(S, warp * chunk), end = min(S, beg + chunk);
+  const int beg = min(c1, c0 + warp * chunk), end = min(c1, beg + chunk);
 
   // The expert ids of kRouteBatch consecutive 32-slot steps, loaded before
   // any of them is used, so a warp waits for one load latency per batch
@@ -101,7 +106,9 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   if (bad) s_bad = 1;
   __syncthreads();
 
-  // per expert: total count, and counts of earlier warps (exclusive over warps)
+  // per expert: total count, and counts of earlier warps (exclusive over
+  // warps); with several CTAs the totals and this chunk's base come from the
+  // per-chunk counts of route_count_kernel
   for (int e = tid; e < E; e += kRouteThreads) {
     int run = 0;
     for (int w = 0; w < 32; ++w) {
@@ -109,9 +116,22 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
       wc[w * NG + e] = run;
       run += c;
     }
-    cnt[e] = run;
+    int total = run, base = 0;
+    if (p.nparts > 1) {
+      total = 0;
+      for (int b = 0; b < p.nparts; ++b) {
+        const int c = p.part[b * E + e];
+        if (b < (int)blockIdx.x) base += c;
+        total += c;
+      }
+    }
+    cnt[e] = total;
+    cbase[e] = base;
   }
-  if (p.n_shared && tid == 0) cnt[E] = p.T;
+  if (p.n_shared && tid == 0) {
+    cnt[E] = p.T;
+    cbase[E] = 0;
+  }
   __syncthreads();
 
   // exclusive scans: group offsets, and tile offsets (ceil(count / BN) tiles)
@@ -136,10 +156,12 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   }
   __syncthreads();
 
-  for (int g = tid; g < NG; g += kRouteThreads) p.counts[g] = cnt[g];
-  for (int g = tid; g <= NG; g += kRouteThreads) p.offsets[g] = off[g];
-  if (p.tile_off)
-    for (int g = tid; g <= NG; g += kRouteThreads) p.tile_off[g] = toff[g];
+  if (lead) {
+    for (int g = tid; g < NG; g += kRouteThreads) p.counts[g] = cnt[g];
+    for (int g = tid; g <= NG; g += kRouteThreads) p.offsets[g] = off[g];
+    if (p.tile_off)
+      for (int g = tid; g <= NG; g += kRouteThreads) p.tile_off[g] = toff[g];
+  }
 
   // pass B: stable scatter
   for (int b0 = beg; b0 < end; b0 += 32 * kRouteBatch) {
@@ -154,7 +176,7 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
       const int rank = __popc(peers & ((1u << lane) - 1u));
       if (s < end) {
         if (e >= 0) {
-          const int pos = off[e] + wc[warp * NG + e] + rank;
+          const int pos = off[e] + cbase[e] + wc[warp * NG + e] + rank;
           p.perm[pos] = s;
           p.inv[s] = pos;
         } else {
@@ -167,6 +189,10 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
     }
   }
 
+  if (!lead) {
+    if (tid == 0 && s_bad) atomicOr(p.status, DEV_BAD_ROUTING);
+    return;
+  }
   // shared expert: every token, as virtual slot S + t, after the routed groups
   if (p.n_shared) {
     for (int t = tid; t < p.T; t += kRouteThreads) {
@@ -189,9 +215,37 @@ __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) 
   }
 }
 
-size_t route_smem_bytes(int n_groups) { return sizeof(int) * (3 * (size_t)n_groups + 2 + 32 * (size_t)n_groups); }
+size_t route_smem_bytes(int n_groups) { return sizeof(int) * (4 * (size_t)n_groups + 2 + 32 * (size_t)n_groups); }
 
-cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
+// Per-chunk expert counts for the multi-CTA route: CTA b counts the valid
+// expert ids of slots [b * chunk, (b + 1) * chunk) into part[b][e].
+__global__ void __launch_bounds__(kRouteThreads) route_count_kernel(RouteParams p) {
+  extern __shared__ int hist[];  // [E]
+  const int S = p.T * p.k, E = p.E;
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) hist[e] = 0;
+  __syncthreads();
+  const int c0 = min(S, (int)blockIdx.x * p.chunk), c1 = min(S, c0 + p.chunk);
+  for (int s = c0 + threadIdx.x; s < c1; s += kRouteThreads) {
+    const int e = p.ids[s];
+    if (e >= 0 && e < E) atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += kRouteThreads) p.part[blockIdx.x * E + e] = hist[e];
+}
+
+// Slots per CTA of the multi-CTA route, and the slot count from which it is used
+constexpr int kRouteChunk = 2048;
+constexpr int kRouteMultiSlots = 4096;
+
+cudaError_t launch_route(const RouteParams& p0, cudaStream_t s) {
+  RouteParams p = p0;
+  const int S = p.T * p.k;
+  p.nparts = 1;
+  p.chunk = S;
+  if (p.part && S >= kRouteMultiSlots) {
+    p.nparts = min(kMaxRouteParts, (S + kRouteChunk - 1) / kRouteChunk);
+    p.chunk = (S + p.nparts - 1) / p.nparts;
+  }
   const size_t smem = route_smem_bytes(p.E + p.n_shared);
   static bool attr_set = false;
   if (!attr_set) {
@@ -200,7 +254,12 @@ cudaError_t launch_route(const RouteParams& p, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  route_kernel<<<1, kRouteThreads, smem, s>>>(p);
+  if (p.nparts > 1) {
+    route_count_kernel<<<p.nparts, kRouteThreads, sizeof(int) * p.E, s>>>(p);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  route_kernel<<<p.nparts, kRouteThreads, smem, s>>>(p);
   return cudaGetLastError();
 }
 
