@@ -21,13 +21,14 @@ WFMT_FP8 = 0
 WFMT_MXFP4 = 1
 WFMT_NVFP4 = 2
 WFMT_MXFP4_A4 = 3
+WFMT_MXFP8 = 4
 
 
 def shard_weights(w13, s13, w2, s2, wfmt: int, I: int, rank: int, world: int, g13=None, g2=None) -> dict:
     """The slice of rank ``rank`` (of ``world``) of one layer's expert weights.
 
-    Layouts as in include/moe.h, with the MXFP4 / NVFP4 scales in their plain
-    layouts (pack each rank's slice with pack_shard).  Returns a dict w13,
+    Layouts as in include/moe.h, with the MXFP4 / NVFP4 / MXFP8 scales in
+    their plain layouts (pack each rank's slice with pack_shard).  Returns a dict w13,
     s13, w2, s2 (contiguous) and, for NVFP4, g13, g2 (unchanged: the
     per-expert global scales apply to every slice)."""
     import torch
@@ -55,6 +56,11 @@ def shard_weights(w13, s13, w2, s2, wfmt: int, I: int, rank: int, world: int, g1
         if wfmt == WFMT_NVFP4:
             out.update(g13=g13, g2=g2)
         return out
+    if wfmt == WFMT_MXFP8:
+        return dict(w13=gate_up(w13, c0, c1, I),                # [NE, 2I, H] E4M3 bytes
+                    s13=gate_up(s13, c0, c1, I),                # [NE, 2I, H/32]
+                    w2=w2[:, :, c0:c1].contiguous(),            # [NE, H, I]
+                    s2=s2[:, :, c0 // 32:c1 // 32].contiguous())  # [NE, H, I/32]
     raise ValueError(f"unknown weight format {wfmt}")
 
 
@@ -73,7 +79,7 @@ class TPMoeLayer:
     ``forward`` runs the rank's I slice through the library
     (moe_forward_partial), all-reduces the fp32 partial over the process
     group, and rounds it to bf16 (moe_finalize_bf16).  Weights are given
-    already sharded (shard_weights) and, for MXFP4 / NVFP4, packed."""
+    already sharded (shard_weights) and, for MXFP4 / NVFP4 / MXFP8, packed."""
 
     def __init__(self, H, I, E, k, wfmt, world: int, max_T=4096, n_shared=0, group=None):
         if I % world or (I // world) % 128:
@@ -92,10 +98,10 @@ class TPMoeLayer:
 
 
 def pack_shard(shard: dict, wfmt: int, stream=None) -> dict:
-    """A rank's slice with its MXFP4 / NVFP4 scales converted to the layout the
-    library reads (FP8 scales are used as they are)."""
+    """A rank's slice with its MXFP4 / NVFP4 / MXFP8 scales converted to the
+    layout the library reads (FP8 scales are used as they are)."""
     out = dict(shard)
-    if wfmt in (WFMT_MXFP4, WFMT_MXFP4_A4):
+    if wfmt in (WFMT_MXFP4, WFMT_MXFP4_A4, WFMT_MXFP8):
         out["s13"], out["s2"] = moe.pack_mxfp4_scales(shard["s13"], stream), moe.pack_mxfp4_scales(shard["s2"], stream)
     elif wfmt == WFMT_NVFP4:
         out["s13"], out["s2"] = moe.pack_nvfp4_scales(shard["s13"], stream), moe.pack_nvfp4_scales(shard["s2"], stream)

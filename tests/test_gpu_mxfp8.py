@@ -128,6 +128,17 @@ def test_mxfp8_zero_input_and_repeated_calls():
         assert_close(out.float().cpu().numpy(), ref, "repeated")
 
 
+@pytest.mark.parametrize("mode", ["atomic", "rows"])
+def test_mxfp8_combine_paths(mode, monkeypatch):
+    """Both top-k combines with the token-major MXFP8 GEMM2: fused fp32
+    reductions, and stored per-position rows summed by the combine pass."""
+    monkeypatch.setenv("MOE_COMBINE", mode)
+    L = synth.make_layer(dict(T=150, H=256, I=256, E=8, k=4, wfmt=WFMT, n_shared=1), 88, device="cuda")
+    layer, out = run_gpu(L)
+    assert layer.device_status() == moe.MOE_OK
+    assert_close(out.float().cpu().numpy(), oracle_ref(L)["out_f32"], f"combine {mode}")
+
+
 def test_mxfp8_prefill_sized_layer():
     """T=4096, H=7168, E=256, k=8, I=2048 in MXFP8, in the benchmark's launch
     configuration: the tokens holding each expert's first and last routing

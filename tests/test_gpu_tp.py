@@ -37,7 +37,8 @@ CASES = [("fp8_shared", dict(T=24, H=512, I=512, E=8, k=2, wfmt=0, n_shared=1), 
          ("fp8_g4", dict(T=9, H=256, I=512, E=6, k=3, wfmt=0), 4),
          ("nvfp4", dict(T=16, H=512, I=512, E=8, k=2, wfmt=2), 2),
          ("mxfp4_a4", dict(T=16, H=512, I=512, E=8, k=2, wfmt=3, n_shared=1), 2),
-         ("mxfp4", dict(T=12, H=512, I=512, E=8, k=2, wfmt=1), 2)]
+         ("mxfp4", dict(T=12, H=512, I=512, E=8, k=2, wfmt=1), 2),
+         ("mxfp8_shared", dict(T=20, H=512, I=512, E=8, k=2, wfmt=4, n_shared=1), 2)]
 
 
 @pytest.mark.parametrize("name,cfg,G", CASES, ids=[c[0] for c in CASES])

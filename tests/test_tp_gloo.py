@@ -12,7 +12,8 @@ import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
-CASES = [dict(wfmt=0, n_shared=1), dict(wfmt=2, n_shared=0), dict(wfmt=3, n_shared=1), dict(wfmt=1, n_shared=0)]
+CASES = [dict(wfmt=0, n_shared=1), dict(wfmt=2, n_shared=0), dict(wfmt=3, n_shared=1), dict(wfmt=1, n_shared=0),
+         dict(wfmt=4, n_shared=1)]
 
 
 def _free_port():
@@ -66,7 +67,7 @@ def test_two_ranks_sum_to_the_whole_layer():
         assert np.array_equal(out[(0, ci)], out[(1, ci)])  # every rank holds the same sum
 
 
-@pytest.mark.parametrize("wfmt", [0, 1, 2, 3])
+@pytest.mark.parametrize("wfmt", [0, 1, 2, 3, 4])
 def test_shards_reassemble_the_weights(wfmt):
     from fp4_block_scaled_route_b200 import tp
     L = _layer(dict(wfmt=wfmt, n_shared=0))
