@@ -1,8 +1,7 @@
 // moe_noalloc.cu -- moe_forward_noalloc(): the MoE layer without any device
 // allocation, for callers that cannot call cudaMalloc (for example code that
-// runs inside a host framework which owns every device allocation, or that
-// must not allocate while a stream is being captured or while a memory pool
-// is locked).  The layer's scratch (routing arrays, tile list, quantised
+// runs inside a host framework which owns every device allocation, or while
+// a memory pool is locked).  The layer's scratch (routing arrays, tile list, quantised
 // activations, fp32 combine buffer, status word) lives in one file-scope
 // device array of fixed size instead of a context's workspace.
 #include <cuda.h>

@@ -375,19 +375,18 @@ moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
 
 /* moe_forward_noalloc -- the same layer as moe_forward(), for callers that
  * cannot allocate device memory: code running under a host framework that
- * owns every device allocation (its allocator may not be bypassed), code that
- * must not allocate while a stream is being captured, or a memory-pool-locked
- * process.  No context is needed and nothing is allocated: no cudaMalloc,
- * cudaFree or allocating library routine.  The scratch (routing arrays, tile
- * list, quantised activations, fp32 combine buffer) is one file-scope device
- * array of MOE_NOALLOC_SCRATCH_BYTES that every GPU which loads the library
- * keeps until the process exits.  The method's sources describe no
- * counterpart of this entry point; it exists only for such callers.
+ * owns every device allocation (its allocator may not be bypassed), or a
+ * memory-pool-locked process.  No context is needed and nothing is
+ * allocated: no cudaMalloc, cudaFree or allocating library routine.  The
+ * scratch (routing arrays, tile list, quantised activations, fp32 combine
+ * buffer) is one file-scope device array of MOE_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads the library keeps until the process exits.  The
+ * method's sources describe no counterpart of this entry point; it exists
+ * only for such callers.
  *   H, I, E, k, n_shared   the layer, as in moe_create_ex()
  *   wfmt       MOE_WFMT_FP8_E4M3_B128 or MOE_WFMT_MXFP4_E2M1_E8M0_K32 (scales
- *              packed with moe_pack_mxfp4_scales()); the two formats with
- *              4-bit activations (NVFP4, MXFP4_W4A4) return
- *              MOE_ERR_UNSUPPORTED
+ *              packed with moe_pack_mxfp4_scales()); the other formats
+ *              (NVFP4, MXFP4_W4A4, MXFP8) return MOE_ERR_UNSUPPORTED
  *   T, x, topk_ids, topk_w, w13, s13, w2, s2, out   as in moe_forward()
  *   d_status   optional device int32 (caller memory): cleared, then receives
  *              the device status bits of this call (1 = expert id out of
@@ -398,14 +397,13 @@ moe_status moe_profile_read(moe_ctx* ctx, float* avg_ms, int* calls);
  * 15 MB); a shape that needs more than MOE_NOALLOC_SCRATCH_BYTES returns
  * MOE_ERR_UNSUPPORTED before any device work.
  * The first call on a device performs a one-time set-up on the current
- * device (looks up the array's device address, sets kernel attributes);
- * make that first call before any stream capture.  That set-up is
- * thread-safe: host threads making their first calls at the same time
- * wait for one another.  A device index of 64 or more returns
- * MOE_ERR_UNSUPPORTED.  Every call, on every
- * stream, shares the one array and leaves its contents behind: calls whose
- * execution overlaps on the GPU race and corrupt each other's results, so
- * order them (one stream, or events). */
+ * device (looks up the array's device address, sets kernel attributes).
+ * That set-up is thread-safe: host threads making their first calls at the
+ * same time wait for one another.  A device index of 64 or more returns
+ * MOE_ERR_UNSUPPORTED.  Every call, on every stream, shares the one array
+ * and leaves its contents behind: calls whose execution overlaps on the GPU
+ * race and corrupt each other's results, so order them (one stream, or
+ * events). */
 moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, int n_shared, int T, const void* x,
                                const int32_t* topk_ids, const float* topk_w, const void* w13, const void* s13,
                                const void* w2, const void* s2, void* out, int32_t* d_status, void* stream);

@@ -1,7 +1,7 @@
 """moe_forward_noalloc: the layer for callers that cannot allocate device memory.
 
 Such callers (code under a host framework that owns all device allocations,
-code that must not allocate during stream capture) get one entry point that
+or a memory-pool-locked process) get one entry point that
 keeps its scratch in a fixed file-scope device array instead of a context's
 workspace.  These tests call it through the C ABI and compare its output with
 moe_forward's (the entry point that allocates a workspace), within the
@@ -38,8 +38,8 @@ def test_noalloc_rejects_shapes_beyond_the_scratch():
     rc = moe.moe_forward_noalloc(100, 2048, 256, 8, 0, 0, 4, None, None, None, None, None, None, None,
                                  None, None, None)
     assert rc == moe.MOE_ERR_UNSUPPORTED
-    # the formats with 4-bit activations are not offered here
-    for wfmt in (moe.MOE_WFMT_NVFP4_E2M1_E4M3_K16, moe.MOE_WFMT_MXFP4_W4A4):
+    # the formats with 4-bit activations, and MXFP8, are not offered here
+    for wfmt in (moe.MOE_WFMT_NVFP4_E2M1_E4M3_K16, moe.MOE_WFMT_MXFP4_W4A4, moe.MOE_WFMT_MXFP8_E4M3_E8M0_K32):
         rc = moe.moe_forward_noalloc(512, 256, 8, 2, wfmt, 0, 4, None, None, None, None, None, None, None,
                                      None, None, None)
         assert rc == moe.MOE_ERR_UNSUPPORTED
