@@ -154,6 +154,14 @@ struct GemmCfg {
   static_assert(!P4 || BN <= 32, "4-bit activation tiles hold at most 32 tokens");
 };
 
+// Moves entries CH..N-1 of a register array to 0..N-CH-1 (the last CH are
+// left for the caller); with static indices the array stays in registers.
+template <int N, int CH>
+__device__ __forceinline__ void rotl(float* a) {
+#pragma unroll
+  for (int i = 0; i + CH < N; ++i) a[i] = a[i + CH];
+}
+
 // Bounded wait that ignores the abort word (used to drain in-flight copies
 // and MMAs before the CTA releases its shared memory and TMEM).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -507,6 +515,46 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     uint32_t tphase = 0;
     bool ok = true;
     int eit = 0;  // pipeline iteration
+    auto unit_rt = [&](int uu) { return C::TILE_MAJOR ? uu % NRT : uu / num_tiles; };
+    auto unit_ti = [&](int uu) { return C::TILE_MAJOR ? uu / NRT : uu % num_tiles; };
+    // Inputs of unit u that do not come from the previous kernel: the weight
+    // block scales (NVFP4: the expert's global scale) and, in GEMM2, the
+    // combine target of every column (route outputs and the top-k weights).
+    auto load_static = [&](int u, const int4& tile) {
+      const int e = tile.x, p0 = tile.y, nv = tile.z, rt = unit_rt(u);
+      (void)e; (void)p0; (void)nv; (void)rt;
+      if constexpr (WFMT == 0) {
+        for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
+          const int a = i / KB, kb = i % KB;
+          wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + tile_rb(rt, a)) * KB + kb];
+        }
+      }
+      if constexpr (NV) {
+        if (etid == 0) wsc[0] = p.wglobal[e];
+      }
+      if constexpr (KIND == 2) {
+        for (int j = etid; j < BN; j += C::EPI_THREADS) {
+          int tok = 0;
+          float w = 0.0f;
+          if (j < nv) {
+            const int slot = p.perm[p0 + j];
+            tok = (slot < S) ? slot / p.k : slot - S;
+            w = (slot < S) ? p.topk_w[slot] : 1.0f;
+          }
+          slot_tok[j] = tok;
+          slot_w[j] = w;
+        }
+      }
+    };
+    // The first unit's are read before waiting for the previous kernel (the
+    // memory system is still quiet then), so that after the wait only its
+    // activation scales remain to be read.
+    const int u0 = blockIdx.x;
+    int4 tile0 = make_int4(0, 0, 0, 0);
+    if (u0 < total) {
+      tile0 = p.tiles[unit_ti(u0)];
+      load_static(u0, tile0);
+    }
     griddep_wait();  // activation scales / combine buffer come from earlier kernels
     if constexpr (DISP) {
       // dispatch overlap: the last p.disp CTAs' epilogue warps quantise first
@@ -522,8 +570,6 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
     // routing slot and combine weight included, made it slower.)
     constexpr bool PREF = BN <= 32 && KIND == 1 && !DISP;  // (dispatch overlap: scales read after the ready wait)
     constexpr int NPA = PREF ? (BN * KB_MAX + C::EPI_THREADS - 1) / C::EPI_THREADS : 1;
-    auto unit_rt = [&](int uu) { return C::TILE_MAJOR ? uu % NRT : uu / num_tiles; };
-    auto unit_ti = [&](int uu) { return C::TILE_MAJOR ? uu / NRT : uu % num_tiles; };
     int4 tile_n = make_int4(0, 0, 0, 0);
     float pa[NPA];
     float pw = 0.0f;
@@ -554,9 +600,23 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
       }
     };
     bool from_regs = false;
+    if constexpr (PREF) {
+      // the first unit's activation scales, all loads in flight together
+      if (u0 < total) {
+        tile_n = tile0;
+        if constexpr (!MXA) {
+#pragma unroll
+          for (int r = 0; r < NPA; ++r) {
+            const int i = etid + r * C::EPI_THREADS;
+            pa[r] = (i < BN * KB) ? p.ascale[(size_t)(i / BN) * p.scale_ld + tile0.y + (i % BN)] : 0.0f;
+          }
+        }
+        from_regs = true;
+      }
+    }
     for (int u = blockIdx.x; u < total; u += gridDim.x) {
       const int rt = unit_rt(u), ti = unit_ti(u);
-      const int4 tile = from_regs ? tile_n : p.tiles[ti];
+      const int4 tile = from_regs ? tile_n : p.tiles[ti];  // (the first unit's: a cache hit)
       const int e = tile.x, p0 = tile.y, nv = tile.z;
       if constexpr (DISP) {
         if (ok) ok = dispatch_ready(p, e, abort);
@@ -569,41 +629,32 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
             if (i < BN * KB) asc[i] = pa[r];
           }
         }
-        if constexpr (WFMT == 0) {
-          if (etid < NA * KB) wsc[(etid / KB) * KB_MAX + etid % KB] = pw;
-        }
-        if constexpr (NV) {
-          if (etid == 0) wsc[0] = pw;
+        if (u != u0) {  // the first unit's came from load_static
+          if constexpr (WFMT == 0) {
+            if (etid < NA * KB) wsc[(etid / KB) * KB_MAX + etid % KB] = pw;
+          }
+          if constexpr (NV) {
+            if (etid == 0) wsc[0] = pw;
+          }
         }
       } else {
         if constexpr (!MXA) {
-          for (int i = etid; i < BN * KB; i += C::EPI_THREADS) {
-            const int kb = i / BN, j = i % BN;
-            asc[i] = p.ascale[(size_t)kb * p.scale_ld + p0 + j];
-          }
-        }
-        if constexpr (WFMT == 0) {
-          for (int i = etid; i < NA * KB; i += C::EPI_THREADS) {
-            const int a = i / KB, kb = i % KB;
-            wsc[a * KB_MAX + kb] = p.wscale[((size_t)e * RB + tile_rb(rt, a)) * KB + kb];
-          }
-        }
-        if constexpr (NV) {
-          if (etid == 0) wsc[0] = p.wglobal[e];
-        }
-        if constexpr (KIND == 2) {
-          for (int j = etid; j < BN; j += C::EPI_THREADS) {
-            int tok = 0;
-            float w = 0.0f;
-            if (j < nv) {
-              const int slot = p.perm[p0 + j];
-              tok = (slot < S) ? slot / p.k : slot - S;
-              w = (slot < S) ? p.topk_w[slot] : 1.0f;
+          // four loads in flight per thread and round
+          for (int i0 = etid; i0 < BN * KB; i0 += 4 * C::EPI_THREADS) {
+            float v[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int i = i0 + r * C::EPI_THREADS;
+              v[r] = (i < BN * KB) ? p.ascale[(size_t)(i / BN) * p.scale_ld + p0 + (i % BN)] : 0.0f;
             }
-            slot_tok[j] = tok;
-            slot_w[j] = w;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int i = i0 + r * C::EPI_THREADS;
+              if (i < BN * KB) asc[i] = v[r];
+            }
           }
         }
+        if (u != u0) load_static(u, tile);
       }
       named_sync(1, C::EPI_THREADS);
       const int un = u + gridDim.x;
@@ -698,96 +749,125 @@ __global__ void __launch_bounds__(GemmCfg<KIND, BN, WFMT, NT>::THREADS, 1)
       if constexpr (KIND == 1) {
         // Per gate/up pair (gate rows 0..I-1 of W13, up rows I..2I-1: same
         // channels): SwiGLU, then requantisation per token over the output
-        // tile's 128 channels -- NVFP4 (the rule of quant_nvfp4_kernel: lanes
-        // 16i .. 16i+15 of a warp hold one 16-channel block, the four warps
-        // one 128 group) or FP8.  h overwrites the gate accumulator in place.
+        // tile's 128 channels -- FP8, NVFP4 (the rule of quant_nvfp4_kernel:
+        // lanes 16i .. 16i+15 of a warp hold one 16-channel block, the four
+        // warps one 128 group) or MXFP4 (the rule of quant_mxfp4_kernel: a
+        // 32-channel block is one warp).  h overwrites the gate accumulator.
+        //
+        // The columns are taken CH at a time in rolled loops, and the
+        // register arrays rotate left by CH per step (static indices keep
+        // them in registers).  Fully unrolled, this tail is tens of KB of
+        // code per kernel, and the first unit of every launch then waits on
+        // instruction fetches from a memory system that the weight stream
+        // keeps saturated.
+        // (CH chosen per shape to keep the tail free of register spills:
+        // NVFP4 at 32 columns stays unrolled)
+        constexpr int CH = CPT <= 8 ? CPT : CPT >= 64 ? 8 : CPT < 32 ? 2 : NV ? CPT : WFMT == 1 ? 8 : 4;
 #pragma unroll
         for (int pr = 0; pr < NA / 2; ++pr) {
           float* h = acc[2 * pr];
-          const float* up = acc[2 * pr + 1];
+          float* up = acc[2 * pr + 1];
           const int ct = rt * CT + pr;  // output channel tile
           const int ch = ct * 128 + row;
           if constexpr (MXA) {
-            // MXFP4 requantisation (the rule of quant_mxfp4_kernel): a 32-
-            // channel block is one warp, so its amax is a warp reduction and
-            // lane 0 writes the block's E8M0 code (byte q of the tile's entry)
+            // one pass: SwiGLU, the block's amax (a warp reduction), lane 0
+            // writes the block's E8M0 code (byte q of the tile's entry)
+#pragma unroll 1
+            for (int c0 = 0; c0 < CPT; c0 += CH) {
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-              const float g = h[c];
-              const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
-              h[c] = g * sig * up[c];
-            }
-            if (ok) {
-#pragma unroll
-              for (int c = 0; c < CPT; ++c) {
-                const int j = cg * CPT + c;
-                float m = fabsf(h[c]);
+              for (int i = 0; i < CH; ++i) {
+                const int j = cg * CPT + c0 + i;
+                const float g = h[i];
+                const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+                const float hv = g * sig * up[i];
+                float m = fabsf(hv);
 #pragma unroll
                 for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
                 float sc;
                 const int X = mx_e2m1_exponent(m, &sc);
-                const uint32_t nib = f32_to_e2m1(__fdiv_rn(h[c], sc));
+                const uint32_t nib = f32_to_e2m1(__fdiv_rn(hv, sc));
                 uint32_t word = nib << (4 * (lane & 7));
                 word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
                 word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
                 word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-                if (j < nv) {
+                if (ok && j < nv) {
                   if ((lane & 7) == 0)
                     *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
                   if (lane == 0)
                     p.hsc[((size_t)ct * p.scale_ld + p0 + j) * 16 + q] = static_cast<uint8_t>(X + 127);
                 }
               }
+              rotl<CPT, CH>(h);
+              rotl<CPT, CH>(up);
             }
-            continue;
-          }
-          float a16[NV ? CPT : 1];
+          } else {
+            // pass 1: SwiGLU and the per-quarter amax of each column; h takes
+            // the SwiGLU outputs and (NVFP4) up the 16-channel block amaxes
+#pragma unroll 1
+            for (int c0 = 0; c0 < CPT; c0 += CH) {
+              float hv[CH], bv[CH];
 #pragma unroll
-          for (int c = 0; c < CPT; ++c) {
-            const float g = h[c];
-            const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
-            h[c] = g * sig * up[c];
-            float m = fabsf(h[c]);
+              for (int i = 0; i < CH; ++i) {
+                const float g = h[i];
+                const float sig = __fdiv_rn(1.0f, 1.0f + expf(-g));
+                hv[i] = g * sig * up[i];
+                float m = fabsf(hv[i]);
 #pragma unroll
-            for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-            if constexpr (NV) a16[c] = m;
-            m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
-            if (lane == 0) red[q * BN + cg * CPT + c] = m;
-          }
-          named_sync(1, C::EPI_THREADS);
-          if (ok) {
+                for (int o = 8; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+                bv[i] = m;
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 16));
+                if (lane == 0) red[q * BN + cg * CPT + c0 + i] = m;
+              }
+              rotl<CPT, CH>(h);
+              rotl<CPT, CH>(up);
 #pragma unroll
-            for (int c = 0; c < CPT; ++c) {
-              const int j = cg * CPT + c;
-              const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
-              if constexpr (NV) {
-                const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
-                const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16[c], 6.0f), sg));
-                const float d = __fmul_rn(e4m3_code_value(code), sg);
-                const uint32_t nib = code ? f32_to_e2m1(__fdiv_rn(h[c], d)) : 0u;
-                // eight neighbouring channels -> one 32-bit word of packed codes
-                uint32_t word = nib << (4 * (lane & 7));
-                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
-                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
-                word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
-                if (j < nv) {
-                  if ((lane & 7) == 0)
-                    *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
-                  if ((lane & 15) == 0)
-                    p.hsc[((size_t)(ch / 64) * p.scale_ld + p0 + j) * 16 + (ch / 16) % 4] =
-                        static_cast<uint8_t>(code);
-                  if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sg;
-                }
-              } else {
-                const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
-                if (j < nv) {
-                  p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[c], sc)));
-                  if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sc;
-                }
+              for (int i = 0; i < CH; ++i) {
+                h[CPT - CH + i] = hv[i];
+                up[CPT - CH + i] = bv[i];
               }
             }
+            const float* a16 = up;
+            named_sync(1, C::EPI_THREADS);
+            // pass 2: the per-token scale of the 128 channels, the codes
+            if (ok) {
+#pragma unroll 1
+              for (int c0 = 0; c0 < CPT; c0 += CH) {
+#pragma unroll
+                for (int i = 0; i < CH; ++i) {
+                  const int j = cg * CPT + c0 + i;
+                  const float amax = fmaxf(fmaxf(red[j], red[BN + j]), fmaxf(red[2 * BN + j], red[3 * BN + j]));
+                  if constexpr (NV) {
+                    const float sg = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 2688.0f);
+                    const uint32_t code = f32_to_e4m3(__fdiv_rn(__fdiv_rn(a16[i], 6.0f), sg));
+                    const float d = __fmul_rn(e4m3_code_value(code), sg);
+                    const uint32_t nib = code ? f32_to_e2m1(__fdiv_rn(h[i], d)) : 0u;
+                    // eight neighbouring channels -> one 32-bit word of packed codes
+                    uint32_t word = nib << (4 * (lane & 7));
+                    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 1);
+                    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+                    word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+                    if (j < nv) {
+                      if ((lane & 7) == 0)
+                        *reinterpret_cast<uint32_t*>(p.hq + (size_t)(p0 + j) * (p.I / 2) + ch / 2) = word;
+                      if ((lane & 15) == 0)
+                        p.hsc[((size_t)(ch / 64) * p.scale_ld + p0 + j) * 16 + (ch / 16) % 4] =
+                            static_cast<uint8_t>(code);
+                      if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sg;
+                    }
+                  } else {
+                    const float sc = (amax == 0.0f) ? 1.0f : __fdiv_rn(amax, 448.0f);
+                    if (j < nv) {
+                      p.hq[(size_t)(p0 + j) * p.I + ch] = static_cast<uint8_t>(f32_to_e4m3(__fdiv_rn(h[i], sc)));
+                      if (row == 0) p.hs[(size_t)ct * p.scale_ld + p0 + j] = sc;
+                    }
+                  }
+                }
+                rotl<CPT, CH>(h);
+                if constexpr (NV) rotl<CPT, CH>(up);
+              }
+            }
+            if (pr + 1 < NA / 2) named_sync(1, C::EPI_THREADS);  // red is reused by the next pair
           }
-          if (pr + 1 < NA / 2) named_sync(1, C::EPI_THREADS);  // red is reused by the next pair
         }
       } else {
         if (ok) {

@@ -267,27 +267,59 @@ cudaError_t launch_route(const RouteParams& p0, cudaStream_t s) {
 // One CTA per token, 8 warps; warp w quantises column groups w, w+8, ...
 // Each lane holds 4 consecutive bf16 values of the 128-column group.
 constexpr int kQuantThreads = 256;
+constexpr int kQuantGroups = 64 / (kQuantThreads / 32);  // H <= 8192: at most 8 groups per warp
+
+// The token's 128-column groups of this warp (g = warp, warp + 8, ...), all
+// loads issued at once and before the routing rows are known: x does not
+// depend on the route kernel, and a warp then waits for one load latency
+// instead of one per group.
+__device__ __forceinline__ void load_token_groups(const QuantParams& p, int t, uint2 (&raw)[kQuantGroups]) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint16_t* xr = p.x + (size_t)t * p.H;
+#pragma unroll
+  for (int i = 0; i < kQuantGroups; ++i) {
+    const int g = warp + i * (kQuantThreads / 32);
+    raw[i] = (g < p.H / 128) ? *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4) : make_uint2(0u, 0u);
+  }
+}
+
+// Drops raw[0] and moves the rest down (static indices: registers).
+__device__ __forceinline__ void next_group(uint2 (&raw)[kQuantGroups]) {
+#pragma unroll
+  for (int i = 0; i + 1 < kQuantGroups; ++i) raw[i] = raw[i + 1];
+}
+
+// The token's routed positions in routing order (slot j of the token in
+// lane j, the shared expert's position last), gathered by warp 0 in one
+// round of loads: rows[0 .. *nrows).
+__device__ __forceinline__ void gather_rows(const QuantParams& p, int t, int* rows, int* nrows) {
+  const int lane = threadIdx.x & 31;
+  const int S = p.T * p.k;
+  const int r = (lane < p.k) ? p.inv[t * p.k + lane] : -1;
+  const int rs = (lane == 0 && p.n_shared) ? p.inv[S + t] : -1;
+  const unsigned valid = __ballot_sync(0xFFFFFFFFu, r >= 0);
+  if (r >= 0) rows[__popc(valid & ((1u << lane) - 1u))] = r;
+  if (lane == 0) {
+    int n = __popc(valid);
+    if (p.n_shared) rows[n++] = rs;
+    *nrows = n;
+  }
+}
 
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
   griddep_launch_dependents();  // GEMM1 may start its weight prefetch now
   const int t = blockIdx.x;
-  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j < p.k; ++j) {
-      const int r = p.inv[t * p.k + j];
-      if (r >= 0) rows[n++] = r;
-    }
-    if (p.n_shared) rows[n++] = p.inv[S + t];
-    nrows = n;
-  }
+  uint2 raws[kQuantGroups];
+  load_token_groups(p, t, raws);
+  if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint16_t* xr = p.x + (size_t)t * H;
-  for (int g = warp; g < HB; g += kQuantThreads / 32) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+#pragma unroll 1
+  for (int g = warp; g < HB; g += kQuantThreads / 32, next_group(raws)) {
+    const uint2 raw = raws[0];
     float sc;
     const uint32_t packed = quant_group_e4m3(raw, &sc);
     for (int r = 0; r < nrows; ++r) {
@@ -321,23 +353,17 @@ cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
 __global__ void __launch_bounds__(kQuantThreads) quant_nvfp4_kernel(QuantParams p) {
   griddep_launch_dependents();
   const int t = blockIdx.x;
-  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j < p.k; ++j) {
-      const int r = p.inv[t * p.k + j];
-      if (r >= 0) rows[n++] = r;
-    }
-    if (p.n_shared) rows[n++] = p.inv[S + t];
-    nrows = n;
-  }
+  uint2 raws[kQuantGroups];
+  load_token_groups(p, t, raws);
+  if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint16_t* xr = p.x + (size_t)t * H;
-  for (int g = warp; g < HB; g += kQuantThreads / 32) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+#pragma unroll 1
+  for (int g = warp; g < HB; g += kQuantThreads / 32, next_group(raws)) {
+    const uint2 raw = raws[0];
     float f[4];
     f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
     f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
@@ -388,23 +414,17 @@ cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s) {
 __global__ void __launch_bounds__(kQuantThreads) quant_mxfp4_kernel(QuantParams p) {
   griddep_launch_dependents();
   const int t = blockIdx.x;
-  const int H = p.H, HB = p.H / 128, S = p.T * p.k;
+  const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j < p.k; ++j) {
-      const int r = p.inv[t * p.k + j];
-      if (r >= 0) rows[n++] = r;
-    }
-    if (p.n_shared) rows[n++] = p.inv[S + t];
-    nrows = n;
-  }
+  uint2 raws[kQuantGroups];
+  load_token_groups(p, t, raws);
+  if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint16_t* xr = p.x + (size_t)t * H;
-  for (int g = warp; g < HB; g += kQuantThreads / 32) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+#pragma unroll 1
+  for (int g = warp; g < HB; g += kQuantThreads / 32, next_group(raws)) {
+    const uint2 raw = raws[0];
     float f[4];
     f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
     f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
@@ -455,26 +475,39 @@ __global__ void __launch_bounds__(kQuantThreads) quant_mxfp8_kernel(QuantParams 
   __shared__ int rows[kMaxK + 1];
   __shared__ int atom[kMaxK + 1];  // byte offset of the position's row in its tile's atoms
   __shared__ int nrows;
-  if (threadIdx.x == 0) {
-    int n = 0;
-    for (int j = 0; j <= p.k; ++j) {
-      if (j == p.k && !p.n_shared) break;
-      const int r = (j < p.k) ? p.inv[t * p.k + j] : p.inv[S + t];
-      if (r < 0) continue;
-      const int g = (j < p.k) ? p.ids[t * p.k + j] : p.E;
+  uint2 raws[kQuantGroups];
+  load_token_groups(p, t, raws);
+  if (threadIdx.x < 32) {
+    // slot j of the token in lane j, the shared expert's position in lane 0
+    const int lane = threadIdx.x;
+    auto atom_of = [&](int r, int g) {
       const int within = r - p.offsets[g];
       const int ti = p.tile_off[g] + within / 128, rr = within % 128;
-      rows[n] = r;
-      atom[n] = ti * HB * 512 + (rr % 32) * 16 + (rr / 32) * 4;
-      ++n;
+      return ti * HB * 512 + (rr % 32) * 16 + (rr / 32) * 4;
+    };
+    const int r = (lane < p.k) ? p.inv[t * p.k + lane] : -1;
+    const int rs = (lane == 0 && p.n_shared) ? p.inv[S + t] : -1;
+    const unsigned valid = __ballot_sync(0xFFFFFFFFu, r >= 0);
+    if (r >= 0) {
+      const int i = __popc(valid & ((1u << lane) - 1u));
+      rows[i] = r;
+      atom[i] = atom_of(r, p.ids[t * p.k + lane]);
     }
-    nrows = n;
+    if (lane == 0) {
+      int n = __popc(valid);
+      if (p.n_shared) {
+        rows[n] = rs;
+        atom[n] = atom_of(rs, p.E);
+        ++n;
+      }
+      nrows = n;
+    }
   }
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const uint16_t* xr = p.x + (size_t)t * H;
-  for (int g = warp; g < HB; g += kQuantThreads / 32) {
-    const uint2 raw = *reinterpret_cast<const uint2*>(xr + g * 128 + lane * 4);
+#pragma unroll 1
+  for (int g = warp; g < HB; g += kQuantThreads / 32, next_group(raws)) {
+    const uint2 raw = raws[0];
     float f[4];
     f[0] = __uint_as_float((raw.x & 0xFFFFu) << 16);
     f[1] = __uint_as_float(raw.x & 0xFFFF0000u);
