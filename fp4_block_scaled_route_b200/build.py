@@ -21,8 +21,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmoe.so")
 BUILD_DIR = os.path.join(PKG, "_build")
 
-SOURCES = ["moe_api.cu", "moe_route.cu", "moe_gemm.cu", "moe_gemm_tm.cu", "moe_gemm_tmx.cu", "moe_router.cu",
-           "moe_noalloc.cu"]
+SOURCES = ["moe_api.cu", "moe_route.cu", "moe_gemm.cu", "moe_gemm_tm.cu", "moe_gemm_tmx.cu", "moe_gemm_pair.cu",
+           "moe_router.cu", "moe_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

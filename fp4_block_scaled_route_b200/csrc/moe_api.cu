@@ -39,6 +39,11 @@ struct moe_ctx {
   const void* c_w2;
   int c_bn;
   CUtensorMap tm_w13, tm_w2, tm_xq, tm_hq;
+  // MOE_PAIR_MMA=1 (MXFP4 weights, FP8 activations): GEMM1 of 16-token
+  // tiles on CTA pairs; its activation map (8-row boxes) and scale map
+  int pair_mma;
+  CUtensorMap tm_xq8, tm_s13;
+  const void* c_s13;
   // last call
   int last_T, last_bn, last_grid;
   // profiling: events[call][stage boundary]
@@ -242,6 +247,8 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
     if (!strcmp(env, "rows")) c->combine_mode = 2;
   }
   if (const char* env = getenv("MOE_GREEN_CTX")) c->gc_sms = atoi(env);  // applied below, once created
+  if (const char* env = getenv("MOE_PAIR_MMA"))
+    c->pair_mma = (wfmt == MOE_WFMT_MXFP4_E2M1_E8M0_K32 && !strcmp(env, "1") && moe::gemm_pair_setup() == cudaSuccess);
   int want_disp = 0;
   if (const char* env = getenv("MOE_DISPATCH_CTAS")) want_disp = atoi(env);  // applied below, once created
   if (const char* env = getenv("MOE_TILE_N")) {
@@ -331,6 +338,9 @@ moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_
     delete c;
     return MOE_ERR_CUDA;
   }
+  if (c->pair_mma && !make_map(&c->tm_xq8, CU_TENSOR_MAP_DATA_TYPE_UINT8, c->xq, H, c->S_pad, H, 8,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    c->pair_mma = 0;
   c->y_rows = want_rows ? reinterpret_cast<float*>(b + o_rows) : nullptr;
   c->rt_logits = want_router ? reinterpret_cast<float*>(b + o_rt_logits) : nullptr;
   if (want_router && moe::router_setup(E) != cudaSuccess) {
@@ -592,10 +602,23 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
     g.T = T; g.NG = c->NG;
   }
   mark(MOE_STAGE_GEMM1);
+  const bool pair = c->pair_mma && BN == 16 && !overlap && !green;
+  if (pair && s13 != c->c_s13) {
+    // the packed scales as rows of 256 bytes: atom (row / 128, K block) = rows 2a, 2a + 1
+    const uint64_t atoms = (uint64_t)(c->E + c->n_shared) * (2 * I / 128) * (H / 128);
+    if (!make_map(&c->tm_s13, CU_TENSOR_MAP_DATA_TYPE_UINT8, s13, 256, 2 * atoms, 256, 2,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, 256, CU_TENSOR_MAP_SWIZZLE_NONE)) {
+      c->c_s13 = nullptr;
+      return MOE_ERR_CUDA;
+    }
+    c->c_s13 = s13;
+  }
   if (mx8) {
     g.act_sf = c->xsf;
     g.hsc = c->hsf;
     if (moe::launch_gemm1_tmx(grid, c->tm_w13, c->tm_xq, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (pair) {
+    if (moe::launch_gemm1_pair(c->tm_w13, c->tm_xq8, c->tm_s13, g, s_gemm) != cudaSuccess) return MOE_ERR_CUDA;
   } else if (moe::launch_gemm1(c->wfmt, BN, grid, c->tm_w13, c->tm_xq, tsx, g, s_gemm) != cudaSuccess) {
     return MOE_ERR_CUDA;
   }

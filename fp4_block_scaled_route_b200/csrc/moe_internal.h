@@ -133,6 +133,14 @@ cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_finalize(const float* acc, uint16_t* out, long long n, cudaStream_t s);
 cudaError_t gemm_setup(int wfmt);  // raise shared-memory limits once per process
+// GEMM1 for MXFP4 weights with FP8 activations and 16-token tiles on CTA
+// pairs (moe_gemm_pair.cu): set-up, the number of pairs it launches, launch
+// (tx8: the activations with 8-row boxes; tsf: the packed weight scales as
+// [atoms * 2][256] bytes).
+cudaError_t gemm_pair_setup();
+int gemm_pair_clusters();
+cudaError_t launch_gemm1_pair(const CUtensorMap& tw, const CUtensorMap& tx8, const CUtensorMap& tsf,
+                              const GemmParams& p, cudaStream_t s);
 // tw: weight tiles; tx / th: token tiles.
 // tsf: NVFP4 token block-scale codes, map over [K/64 * S_pad rows, 16 bytes]
 // with boxes of 32 rows; unused otherwise.

@@ -129,7 +129,10 @@ moe_status moe_create(int H, int I, int E, int k, int wfmt, moe_ctx** out);
  * as fp32 reductions (default), or from stored per-position fp32 expert
  * outputs in a separate, deterministic pass that sums each token's experts
  * in ascending j (the context then holds an extra [positions, H] fp32
- * buffer). */
+ * buffer).  MOE_PAIR_MMA=1 (MXFP4 weights with FP8 activations only) runs
+ * GEMM1 of 16-token tiles on pairs of CTAs (tcgen05 MMAs with M = 256 over
+ * two SMs, gate rows on one, up rows on the other); same results within the
+ * layer tolerance, measured slower than the default on B200. */
 moe_status moe_create_ex(int H, int I, int E, int k, int wfmt, int max_T, int n_shared, moe_ctx** out);
 
 /* moe_destroy -- frees the context and its workspace (synchronises the
