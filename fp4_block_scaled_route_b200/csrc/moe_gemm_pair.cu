@@ -7,12 +7,12 @@
 // pipe's issue rate, not HBM, bounds it.  Here one MMA with M = 256 covers
 // the gate rows (in the even CTA of a cluster of two) and the up rows of the
 // same 128 channels (in the odd CTA): per 16 KB of weights the even CTA
-// issues 4 MMAs, one scale copy and one commit for both SMs.
+// issues 4 MMAs, one scale copy and a commit to each CTA for both SMs.
 //
 // Measured, it is slower than the single-CTA kernel (decode T = 128: 1.42-
 // 1.52 ms against 1.12-1.18 ms per layer): an SM takes one tcgen05
 // instruction per ~90 cycles whoever issues it, and only the even CTA of a
-// pair issues, so 6 instructions per 16 KB on one SM of two lose to 11 per
+// pair issues, so 7 instructions per 16 KB on one SM of two lose to 11 per
 // 16 KB on each SM.  The kernel stays as an option (MOE_PAIR_MMA=1).
 //
 // Sources: GC-MoE abstract (operand-swapped tcgen05 block-scaled MMA on FP4
@@ -93,13 +93,11 @@ __device__ __forceinline__ void mma_pair_mxf8f6f4(uint32_t d, uint64_t a, uint64
 __device__ __forceinline__ void tmem_cp_pair_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
-// arrive on `bar` (same offset) in both CTAs once the pair MMAs issued so far completed
-__device__ __forceinline__ void mma_commit_pair(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
-          smem_u32(bar)),
-      "h"((uint16_t)3)
-      : "memory");
+// arrive on the barrier at a cluster address once the pair MMAs issued so
+// far by this thread completed (one commit per CTA whose barrier is signalled)
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar_cluster) {
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar_cluster)
+               : "memory");
 }
 // arrive on a barrier of either CTA: release at cluster scope (data written
 // to the partner's shared memory before it), or default semantics (only an
@@ -194,7 +192,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
   float* xbuf = red + 4 * BN;                                             // [2][128][BH] received half
   uint64_t* bars = reinterpret_cast<uint64_t*>(xbuf + 2 * 128 * BH);
   uint64_t* full = bars;                // [STAGES] (used in the even CTA)
-  uint64_t* mdone = full + STAGES;      // [NMD] (both CTAs, by the multicast commit)
+  uint64_t* mdone = full + STAGES;      // [NMD] (both CTAs, a commit to each)
   uint64_t* tempty = mdone + NMD;       // [NBUF] (even CTA: 4 local + 4 remote warp arrivals)
   uint64_t* xfull = tempty + NBUF;      // [2] partner's half landed (4 remote warp arrivals)
   uint64_t* xempty = xfull + 2;         // [2] partner consumed our half (4 remote warp arrivals)
@@ -330,6 +328,7 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
     // ---------------- pair MMA issuers (even CTA) ----------------
     if (lead) {
       const int mw = warp - C::MMA_WARP;
+      const uint32_t mdone1 = mapa_rank(mdone, 1);  // the odd CTA's stage-done barriers
       bool ok = true;
       int mit = 0;
       for (int u = pair; u < total; u += npairs) {
@@ -356,7 +355,8 @@ __global__ void __launch_bounds__(PairCfg::THREADS, 1)
             for (int kk = 0; kk < 4; ++kk)
               mma_pair_mxf8f6f4(tmem + buf * BN, ad + 2 * kk, bd + 2 * kk, idesc_mxf8f6f4(256, BN, 5, 0, kk, 0), sfa,
                                 tmem + C::SFB_COL, kk > 0);
-            mma_commit_pair(&mdone[mit % NMD]);
+            mma_commit_pair(smem_u32(&mdone[mit % NMD]));
+            mma_commit_pair(mdone1 + 8u * (mit % NMD));
           }
           __syncwarp();
         }
