@@ -565,6 +565,7 @@ static moe_status forward_impl(moe_ctx* c, int T, const void* x, const int32_t* 
   qp.out_acc = rows ? nullptr : acc;
   qp.xsc = c->xsc;
   qp.sf_atoms = c->xsf; qp.ids = ids; qp.offsets = c->offsets; qp.tile_off = c->tile_off; qp.E = c->E;
+  qp.pdl = moe::quant_pdl(T, c->k, c->E, c->n_shared, H, I);
   mark(MOE_STAGE_QUANT);
   if (!overlap) {
     const cudaError_t qe = nvfp4 ? moe::launch_quant_nvfp4(qp, s_disp)

@@ -40,6 +40,7 @@ struct QuantParams {
   float* xs;              // [H/128, xs_ld]    K-block major: one row of position scales per K block
   int xs_ld;              // = S_pad
   float* out_acc;         // [T, H] zeroed here (null: not needed)
+  int pdl;                // launched as a programmatic dependent of the route kernel (see quant_pdl)
   // 4-bit activations: xq holds packed E2M1 [S_pad, H/2] and xsc the block
   // codes in 16-byte entries, four codes in bytes 0..3 (bytes 4..15 stay
   // zero), so that 32 consecutive positions form a block-scale atom of the
@@ -128,6 +129,16 @@ cudaError_t launch_router(const CUtensorMap& tx, const CUtensorMap& tw, const Ro
 
 size_t route_smem_bytes(int n_groups);
 cudaError_t launch_route(const RouteParams& p, cudaStream_t s);
+// Whether the quantisation kernel overlaps the route kernel (a programmatic
+// dependent of it, QuantParams::pdl): only when the layer's weight stream is
+// short.  GEMM1 may then be scheduled only once the routing is complete, so
+// its first ring of weight loads no longer runs during the routing; for a
+// long weight stream that costs more than the hidden launch gap saves.
+// Bound: min(E, T*k) routed experts plus the shared one, 3*H*I bytes each.
+inline bool quant_pdl(int T, int k, int E, int n_shared, int H, int I) {
+  const long long routed = (long long)T * k < E ? (long long)T * k : E;
+  return (routed + n_shared) * 3LL * H * I <= (32LL << 20);
+}
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s);
 cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s);

@@ -198,6 +198,7 @@ extern "C" moe_status moe_forward_noalloc(int H, int I, int E, int k, int wfmt, 
   qp.T = T; qp.H = H; qp.k = k; qp.n_shared = n_shared;
   qp.x = static_cast<const uint16_t*>(x); qp.inv = rp.inv; qp.xq = xq; qp.xs = xs; qp.out_acc = acc;
   qp.xs_ld = (int)S_pad;
+  qp.pdl = moe::quant_pdl(T, k, E, n_shared, H, I);
   if (moe::launch_quant(qp, s) != cudaSuccess) return MOE_ERR_CUDA;
 
   moe::GemmParams g{};

@@ -41,9 +41,9 @@ __device__ __forceinline__ unsigned ballot_match(int key, int nbits) {
 }
 
 __global__ void __launch_bounds__(kRouteThreads, 1) route_kernel(RouteParams p) {
-  // a GEMM1 launched with dispatch overlap may be scheduled now; it waits
-  // for this grid's completion before it reads the routing (no effect on a
-  // following kernel launched without programmatic dependence)
+  // The next kernel (a quantisation kernel, or GEMM1 with dispatch overlap,
+  // when launched as a programmatic dependent) may be scheduled now; it waits
+  // for this grid's completion before it reads the routing.
   griddep_launch_dependents();
   extern __shared__ int sm[];
   const int E = p.E, NG = p.E + p.n_shared;
@@ -283,6 +283,35 @@ __device__ __forceinline__ void load_token_groups(const QuantParams& p, int t, u
   }
 }
 
+// Launched as a programmatic dependent of the route kernel (QuantParams::pdl),
+// a quantisation kernel loads its token while the routing is computed and
+// then waits for it; otherwise the wait returns at once.  GEMM1 may be
+// scheduled only after that point: it reads the tile list before its own
+// wait, and its weight prefetch then starts as the quantisation begins.
+__device__ __forceinline__ void after_route() {
+  griddep_wait();
+  griddep_launch_dependents();
+}
+
+// One CTA per token; a programmatic dependent of the route kernel when p.pdl.
+template <typename K>
+static cudaError_t launch_quant_kernel(K kernel, const QuantParams& p, cudaStream_t s) {
+  if (!p.pdl) {
+    kernel<<<p.T, kQuantThreads, 0, s>>>(p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.T);
+  cfg.blockDim = dim3(kQuantThreads);
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
 // Drops raw[0] and moves the rest down (static indices: registers).
 __device__ __forceinline__ void next_group(uint2 (&raw)[kQuantGroups]) {
 #pragma unroll
@@ -307,13 +336,13 @@ __device__ __forceinline__ void gather_rows(const QuantParams& p, int t, int* ro
 }
 
 __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
-  griddep_launch_dependents();  // GEMM1 may start its weight prefetch now
   const int t = blockIdx.x;
   const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
   uint2 raws[kQuantGroups];
   load_token_groups(p, t, raws);
+  after_route();
   if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -334,8 +363,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_kernel(QuantParams p) {
 }
 
 cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
-  quant_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_quant_kernel(quant_kernel, p, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -351,13 +379,13 @@ cudaError_t launch_quant(const QuantParams& p, cudaStream_t s) {
 // byte c), the four block codes of each step as one 32-bit word (layout of
 // QuantParams::xsc), S.
 __global__ void __launch_bounds__(kQuantThreads) quant_nvfp4_kernel(QuantParams p) {
-  griddep_launch_dependents();
   const int t = blockIdx.x;
   const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
   uint2 raws[kQuantGroups];
   load_token_groups(p, t, raws);
+  after_route();
   if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -399,8 +427,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_nvfp4_kernel(QuantParams 
 }
 
 cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s) {
-  quant_nvfp4_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_quant_kernel(quant_nvfp4_kernel, p, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -412,13 +439,13 @@ cudaError_t launch_quant_nvfp4(const QuantParams& p, cudaStream_t s) {
 // K block is the warp.  Outputs per routed position: packed codes and the
 // K block's four E8M0 codes as one 32-bit word (layout of QuantParams::xsc).
 __global__ void __launch_bounds__(kQuantThreads) quant_mxfp4_kernel(QuantParams p) {
-  griddep_launch_dependents();
   const int t = blockIdx.x;
   const int H = p.H, HB = p.H / 128;
   __shared__ int rows[kMaxK + 1];
   __shared__ int nrows;
   uint2 raws[kQuantGroups];
   load_token_groups(p, t, raws);
+  after_route();
   if (threadIdx.x < 32) gather_rows(p, t, rows, &nrows);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -454,8 +481,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_mxfp4_kernel(QuantParams 
 }
 
 cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s) {
-  quant_mxfp4_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_quant_kernel(quant_mxfp4_kernel, p, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -469,7 +495,6 @@ cudaError_t launch_quant_mxfp4(const QuantParams& p, cudaStream_t s) {
 // atoms: the position's tile ti = tile_off[g] + (pos - offsets[g]) / 128 and
 // row r = (pos - offsets[g]) % 128 within it.
 __global__ void __launch_bounds__(kQuantThreads) quant_mxfp8_kernel(QuantParams p) {
-  griddep_launch_dependents();  // GEMM1 may start its weight prefetch now
   const int t = blockIdx.x;
   const int H = p.H, HB = p.H / 128, S = p.T * p.k;
   __shared__ int rows[kMaxK + 1];
@@ -477,6 +502,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_mxfp8_kernel(QuantParams 
   __shared__ int nrows;
   uint2 raws[kQuantGroups];
   load_token_groups(p, t, raws);
+  after_route();
   if (threadIdx.x < 32) {
     // slot j of the token in lane j, the shared expert's position in lane 0
     const int lane = threadIdx.x;
@@ -532,8 +558,7 @@ __global__ void __launch_bounds__(kQuantThreads) quant_mxfp8_kernel(QuantParams 
 }
 
 cudaError_t launch_quant_mxfp8(const QuantParams& p, cudaStream_t s) {
-  quant_mxfp8_kernel<<<p.T, kQuantThreads, 0, s>>>(p);
-  return cudaGetLastError();
+  return launch_quant_kernel(quant_mxfp8_kernel, p, s);
 }
 
 // ---------------------------------------------------------------------------
