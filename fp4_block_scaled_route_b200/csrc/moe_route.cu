@@ -237,6 +237,141 @@ __global__ void __launch_bounds__(kRouteThreads) route_count_kernel(RouteParams 
 constexpr int kRouteChunk = 2048;
 constexpr int kRouteMultiSlots = 4096;
 
+// ---------------------------------------------------------------------------
+// Routing for a few slots (S <= kRouteSmallSlots): one CTA of 256 threads.
+// The same counting sort and the same outputs as route_kernel, in fewer
+// steps: the ids go to shared memory once, a shared-memory histogram gives
+// the counts, one block scan the group and tile offsets, and warp 0 walks
+// the slots in 32-slot steps in order, a slot's position being its group's
+// offset plus the slots of the group already placed plus its rank among the
+// lanes with the same id (a warp-ballot match), which is the stable
+// counting-sort position.  Decode layers route 8 to a few hundred slots,
+// where the 32-warp kernel spends its time in block barriers and in
+// fetching its larger code.
+constexpr int kRouteSmallSlots = 1024;
+constexpr int kRouteSmallThreads = 256;
+
+__global__ void __launch_bounds__(kRouteSmallThreads, 1) route_small_kernel(RouteParams p) {
+  griddep_launch_dependents();  // see route_kernel
+  __shared__ int ids_s[kRouteSmallSlots];
+  __shared__ int cnt[kMaxGroups], run[kMaxGroups];
+  __shared__ int off[kMaxGroups + 1], toff[kMaxGroups + 1];
+  __shared__ int wtot[2][kRouteSmallThreads / 32];
+  __shared__ int s_bad;
+  const int E = p.E, NG = p.E + p.n_shared;
+  const int S = p.T * p.k, P = S + p.n_shared * p.T;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  for (int g = tid; g < NG; g += kRouteSmallThreads) {
+    cnt[g] = (g == E) ? p.T : 0;  // the shared expert takes every token
+    if (p.ready) p.ready[g] = 0;  // dispatch-overlap counters of the GEMM1 launch that follows
+  }
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int s = tid; s < S; s += kRouteSmallThreads) {
+    int e = p.ids[s];
+    if (e < 0 || e >= E) {
+      e = -1;
+      s_bad = 1;
+    } else {
+      atomicAdd(&cnt[e], 1);
+    }
+    ids_s[s] = e;
+  }
+  __syncthreads();
+
+  // exclusive scans of the counts and of the tiles per group (ceil(count / BN));
+  // thread tid owns groups [tid * per, tid * per + per)
+  {
+    const int per = (NG + kRouteSmallThreads - 1) / kRouteSmallThreads;
+    const int b = min(NG, tid * per), en = min(NG, b + per);
+    int lc = 0, lt = 0;
+    for (int g = b; g < en; ++g) {
+      lc += cnt[g];
+      lt += (cnt[g] + p.BN - 1) / p.BN;
+    }
+    int ic = lc, it = lt;  // inclusive within the warp
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int vc = __shfl_up_sync(0xFFFFFFFFu, ic, o), vt = __shfl_up_sync(0xFFFFFFFFu, it, o);
+      if (lane >= o) {
+        ic += vc;
+        it += vt;
+      }
+    }
+    if (lane == 31) {
+      wtot[0][warp] = ic;
+      wtot[1][warp] = it;
+    }
+    __syncthreads();
+    int bc = 0, bt = 0;  // totals of the earlier warps
+    for (int w = 0; w < warp; ++w) {
+      bc += wtot[0][w];
+      bt += wtot[1][w];
+    }
+    int rc = bc + ic - lc, rt = bt + it - lt;
+    for (int g = b; g < en; ++g) {
+      off[g] = rc;
+      toff[g] = rt;
+      run[g] = rc;
+      rc += cnt[g];
+      rt += (cnt[g] + p.BN - 1) / p.BN;
+    }
+    if (tid == kRouteSmallThreads - 1) {
+      off[NG] = rc;
+      toff[NG] = rt;
+    }
+  }
+  __syncthreads();
+
+  for (int g = tid; g < NG; g += kRouteSmallThreads) p.counts[g] = cnt[g];
+  for (int g = tid; g <= NG; g += kRouteSmallThreads) {
+    p.offsets[g] = off[g];
+    if (p.tile_off) p.tile_off[g] = toff[g];
+  }
+  if (warp == 0) {
+    // stable scatter of the routed slots, in order
+    const int kbits = 32 - __clz(E);  // bits of the largest key, E (a dropped id)
+    for (int b0 = 0; b0 < S; b0 += 32) {
+      const int s = b0 + lane;
+      const int e = (s < S) ? ids_s[s] : -1;
+      const unsigned peers = ballot_match(e >= 0 ? e : E, kbits);
+      if (s < S) {
+        if (e >= 0) {
+          const int pos = run[e] + __popc(peers & ((1u << lane) - 1u));
+          p.perm[pos] = s;
+          p.inv[s] = pos;
+        } else {
+          p.inv[s] = -1;
+        }
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(peers) - 1) run[e] += __popc(peers);
+      __syncwarp();
+    }
+  } else {
+    // shared expert: every token, as virtual slot S + t, after the routed groups
+    const int t0 = tid - 32, nt = kRouteSmallThreads - 32;
+    if (p.n_shared)
+      for (int t = t0; t < p.T; t += nt) {
+        const int pos = off[E] + t;
+        p.perm[pos] = S + t;
+        p.inv[S + t] = pos;
+      }
+    for (int i = off[NG] + t0; i < P; i += nt) p.perm[i] = -1;  // tail left by dropped slots
+    // tile list: tiles[toff[g] + j] covers positions off[g] + j*BN ..
+    for (int g = t0; g < NG; g += nt) {
+      const int n = cnt[g];
+      for (int j = 0; j * p.BN < n; ++j)
+        p.tiles[toff[g] + j] = make_int4(g, off[g] + j * p.BN, min(p.BN, n - j * p.BN), 0);
+    }
+    if (t0 == 0) {
+      *p.num_tiles = toff[NG];
+      if (s_bad) atomicOr(p.status, DEV_BAD_ROUTING);
+    }
+  }
+}
+
 cudaError_t launch_route(const RouteParams& p0, cudaStream_t s) {
   RouteParams p = p0;
   const int S = p.T * p.k;
@@ -253,6 +388,10 @@ cudaError_t launch_route(const RouteParams& p0, cudaStream_t s) {
                                          (int)route_smem_bytes(kMaxGroups));
     if (e != cudaSuccess) return e;
     attr_set = true;
+  }
+  if (S <= kRouteSmallSlots) {
+    route_small_kernel<<<1, kRouteSmallThreads, 0, s>>>(p);
+    return cudaGetLastError();
   }
   if (p.nparts > 1) {
     route_count_kernel<<<p.nparts, kRouteThreads, sizeof(int) * p.E, s>>>(p);
