@@ -77,21 +77,23 @@ def oracle_ref(L, ids=None, debug=False, tokens=None):
 
 
 SMALL = [
-    ("tiny", dict(T=4, H=256, I=256, E=8, k=2), 51),
-    ("ragged_bn16", dict(T=37, H=512, I=384, E=16, k=4), 52),
-    ("ragged_bn32", dict(T=70, H=384, I=256, E=6, k=2), 53),
-    ("shared", dict(T=9, H=256, I=384, E=5, k=3, n_shared=1), 54),
-    ("odd_kblocks", dict(T=21, H=640, I=384, E=7, k=2), 55),      # H/128 = 5: last token-code box half past the row
-    ("one_token_k8", dict(T=1, H=1024, I=512, E=32, k=8), 56),
+    # name, cfg, seed, token-tile width the layer picks (from T*k/E, at most 32)
+    ("tiny", dict(T=4, H=256, I=256, E=8, k=2), 51, 16),
+    ("ragged_k4_bn32", dict(T=37, H=512, I=384, E=16, k=4), 52, 32),
+    ("ragged_bn32", dict(T=70, H=384, I=256, E=6, k=2), 53, 32),
+    ("shared", dict(T=9, H=256, I=384, E=5, k=3, n_shared=1), 54, 16),
+    ("odd_kblocks", dict(T=21, H=640, I=384, E=7, k=2), 55, 16),      # H/128 = 5: last token-code box half past the row
+    ("one_token_k8", dict(T=1, H=1024, I=512, E=32, k=8), 56, 16),
 ]
 
 
-@pytest.mark.parametrize("name,cfg,seed", SMALL, ids=[s[0] for s in SMALL])
-def test_nvfp4_layer_small_all_elements(name, cfg, seed):
+@pytest.mark.parametrize("name,cfg,seed,bn", SMALL, ids=[s[0] for s in SMALL])
+def test_nvfp4_layer_small_all_elements(name, cfg, seed, bn):
     cfg = dict(cfg, wfmt=synth.WFMT_NVFP4, routing="uniform")
     L = synth.make_layer(cfg, seed, device="cuda")
     layer, out = run_gpu(L)
     assert layer.device_status() == moe.MOE_OK
+    assert layer.last_config()[0] == bn
     ref = oracle_ref(L, debug=True)
     assert_close(out.float().cpu().numpy(), ref["out_f32"], name)
 

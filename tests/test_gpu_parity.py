@@ -159,24 +159,26 @@ def test_activation_codes_bit_exact(T, H, E, k, nsh):
 
 # ---- the whole layer, small shapes, every output element ------------------------
 SMALL = [
-    # name, cfg, seed
-    ("config0_tiny", synth.CONFIGS[0], synth.config_seed(0)),
-    ("ragged_bn32", dict(T=64, H=512, I=256, E=8, k=2, wfmt=0), 21),
-    ("ragged_bn64", dict(T=100, H=384, I=384, E=6, k=3, wfmt=0), 22),
-    ("ragged_bn128", dict(T=300, H=256, I=256, E=16, k=4, wfmt=0), 23),
-    ("one_token", dict(T=1, H=1024, I=512, E=32, k=8, wfmt=0), 24),
-    ("shared_fp8", dict(T=10, H=256, I=256, E=6, k=2, wfmt=0, n_shared=1), 25),
-    ("mxfp4_small", dict(T=20, H=512, I=256, E=8, k=2, wfmt=1), 26),
-    ("mxfp4_ragged_bn64", dict(T=90, H=256, I=384, E=6, k=3, wfmt=1), 27),
-    ("mxfp4_shared", dict(T=7, H=384, I=256, E=5, k=2, wfmt=1, n_shared=1), 28),
+    # name, cfg, seed, token-tile width the layer picks (from T*k/E)
+    ("config0_tiny", synth.CONFIGS[0], synth.config_seed(0), 16),
+    ("ragged_bn32", dict(T=64, H=512, I=256, E=8, k=2, wfmt=0), 21, 32),
+    ("ragged_bn64", dict(T=90, H=384, I=384, E=6, k=3, wfmt=0), 29, 64),
+    ("ragged_k3_bn128", dict(T=100, H=384, I=384, E=6, k=3, wfmt=0), 22, 128),
+    ("ragged_bn128", dict(T=300, H=256, I=256, E=16, k=4, wfmt=0), 23, 128),
+    ("one_token", dict(T=1, H=1024, I=512, E=32, k=8, wfmt=0), 24, 16),
+    ("shared_fp8", dict(T=10, H=256, I=256, E=6, k=2, wfmt=0, n_shared=1), 25, 16),
+    ("mxfp4_small", dict(T=20, H=512, I=256, E=8, k=2, wfmt=1), 26, 16),
+    ("mxfp4_ragged_bn64", dict(T=90, H=256, I=384, E=6, k=3, wfmt=1), 27, 64),
+    ("mxfp4_shared", dict(T=7, H=384, I=256, E=5, k=2, wfmt=1, n_shared=1), 28, 16),
 ]
 
 
-@pytest.mark.parametrize("name,cfg,seed", SMALL, ids=[s[0] for s in SMALL])
-def test_layer_small_all_elements(name, cfg, seed):
+@pytest.mark.parametrize("name,cfg,seed,bn", SMALL, ids=[s[0] for s in SMALL])
+def test_layer_small_all_elements(name, cfg, seed, bn):
     L = synth.make_layer(cfg, seed, device="cuda")
     layer, out = run_gpu(L)
     assert layer.device_status() == moe.MOE_OK
+    assert layer.last_config()[0] == bn
     ref = oracle_full(L, debug=True)
     assert_close(bf16_to_f32(out), ref["out_f32"], name)
     # SwiGLU-output codes and scales: equal to the oracle's except where the
