@@ -333,7 +333,7 @@ def workload_record(idx: int, args, dev, stream, sampler):
     t1 = time.time()
     moe.moe_profile_enable(layer.ctx, 1)
     time_steps(step, steps, stream, flush_buf)
-    stage_ms, ncalls = moe.moe_profile_read(layer.ctx)
+    stage_ms, _ = moe.moe_profile_read(layer.ctx)
     moe.moe_profile_enable(layer.ctx, 0)
     if layer.device_status() != moe.MOE_OK:
         raise RuntimeError(f"device status not OK after workload {cfg['name']}")

@@ -107,7 +107,6 @@ ROUTE_CASES += [(1, 256, 8, "uniform", 0, 1), (1, 1, 1, "uniform", 1, 2), (257, 
 @pytest.mark.parametrize("T,E,k,kind,nsh,seed", ROUTE_CASES)
 def test_routing_bit_exact(T, E, k, kind, nsh, seed):
     ids, w = synth.make_routing(T, E, k, kind, seed)
-    cfg = dict(T=T, H=128, I=128, E=E, k=k, wfmt=0, n_shared=nsh)
     dev = "cuda"
     w13 = torch.zeros(E + nsh, 256, 128, dtype=torch.uint8, device=dev)
     s13 = torch.ones(E + nsh, 2, 1, dtype=torch.float32, device=dev)

@@ -4,7 +4,6 @@ max over ranks of the device time, sum over ranks of the bytes streamed."""
 import os
 import socket
 
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 

@@ -8,8 +8,6 @@ moe_forward's (the entry point that allocates a workspace), within the
 layer's tolerance, on two calls in a row, so that scratch left behind by one
 call cannot leak into the next.  The file is named to be collected last.
 """
-import ctypes
-
 import numpy as np
 import pytest
 import torch
