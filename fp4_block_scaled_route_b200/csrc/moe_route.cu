@@ -238,7 +238,7 @@ constexpr int kRouteChunk = 2048;
 constexpr int kRouteMultiSlots = 4096;
 
 // ---------------------------------------------------------------------------
-// Routing for a few slots (S <= kRouteSmallSlots): one CTA of 256 threads.
+// Routing for a few slots (S <= kRouteSmallUpTo): one CTA of 256 threads.
 // The same counting sort and the same outputs as route_kernel, in fewer
 // steps: the ids go to shared memory once, a shared-memory histogram gives
 // the counts, one block scan the group and tile offsets, and warp 0 walks
@@ -247,8 +247,12 @@ constexpr int kRouteMultiSlots = 4096;
 // lanes with the same id (a warp-ballot match), which is the stable
 // counting-sort position.  Decode layers route 8 to a few hundred slots,
 // where the 32-warp kernel spends its time in block barriers and in
-// fetching its larger code.
-constexpr int kRouteSmallSlots = 1024;
+// fetching its larger code.  Its scatter is one warp walking all S slots
+// in order: at 1024 slots the kernel measured slower than the 32-warp one,
+// whose warps scatter their slot ranges side by side (19.5-21.4 us against
+// 12.6-14.4 us), at 256 and fewer faster, so it is used up to 256 slots.
+constexpr int kRouteSmallSlots = 1024;  // capacity of its shared id array
+constexpr int kRouteSmallUpTo = 256;    // slot count up to which launch_route picks it
 constexpr int kRouteSmallThreads = 256;
 
 __global__ void __launch_bounds__(kRouteSmallThreads, 1) route_small_kernel(RouteParams p) {
@@ -389,7 +393,8 @@ cudaError_t launch_route(const RouteParams& p0, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  if (S <= kRouteSmallSlots) {
+  static_assert(kRouteSmallUpTo <= kRouteSmallSlots, "the small route kernel holds every id in shared memory");
+  if (S <= kRouteSmallUpTo) {
     route_small_kernel<<<1, kRouteSmallThreads, 0, s>>>(p);
     return cudaGetLastError();
   }

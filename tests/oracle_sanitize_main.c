@@ -2,7 +2,7 @@
  * (built by tests/test_oracle_sanitizers.py with -fsanitize=address,undefined
  * -fno-sanitize-recover=all, single-threaded).  Every entry point runs on
  * small seeded inputs that include ragged shapes, the shared expert, dropped
- * ids, all four weight formats and the router; any out-of-bounds access, leak or
+ * ids, all five weight formats and the router; any out-of-bounds access, leak or
  * undefined operation aborts with a non-zero exit status. */
 #include <math.h>
 #include <stdint.h>

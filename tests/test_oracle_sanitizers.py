@@ -1,8 +1,8 @@
 """The CPU oracle under AddressSanitizer and UndefinedBehaviorSanitizer.
 
 tests/oracle_sanitize_main.c drives every oracle entry point (routing with
-dropped ids, activation quantisation, the layer in both weight formats with
-and without the shared expert, the router) on small seeded inputs; it is
+dropped ids, activation quantisation, the layer in all five weight formats
+with and without the shared expert, the router) on small seeded inputs; it is
 compiled together with oracle/moe_oracle.c with -fsanitize=address,undefined
 and -fno-sanitize-recover=all, so any out-of-bounds access, leak or undefined
 operation fails the run.  CPU only.
