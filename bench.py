@@ -258,6 +258,15 @@ def build_layer(args, device):
     return cfg, L
 
 
+def launches_per_call(L, dispatch_overlap: bool = False) -> int:
+    """Kernels one moe_forward call launches: the route (from 4096 routed
+    slots on two kernels, per-chunk expert counts and then the scatter), the
+    quantisation (none with dispatch overlap, where GEMM1 quantises), GEMM1,
+    GEMM2 and the bf16 output pass."""
+    route = 2 if L.T * L.k >= 4096 else 1
+    return route + (0 if dispatch_overlap else 1) + 3
+
+
 def gpu_operands(L):
     """The layer's weights in the form moe_forward reads (MXFP4 / NVFP4 scales
     packed once, as at weight-load time) and the NVFP4 global scales."""
@@ -363,7 +372,7 @@ def workload_record(idx: int, args, dev, stream, sampler):
                   "source": f"{src} hbm_gbs; {src} bf16_tflops x {ratio:g} ({'FP4' if ratio == 4 else 'FP8'}/bf16 "
                             f"nominal ratio)"},
         "l2": l2_label(st["weight_bytes"], flush), "steps": steps, "warmup": max(args.warmup, 3),
-        "gpu_launches": moe.MOE_NUM_STAGES * steps, "clocks": sampler.summary(t0, t1),
+        "gpu_launches": launches_per_call(L) * steps, "clocks": sampler.summary(t0, t1),
     }
     layer.close()
     del L, out, flush_buf, w13, s13, w2, s2, gsc
@@ -724,7 +733,7 @@ def main():
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": moe.MOE_NUM_STAGES * args.steps,  # per timed region
+        "gpu_launches": launches_per_call(L, bool(disp)) * args.steps,  # per timed region
         "clocks": clocks,
     }
     if workloads:
