@@ -75,3 +75,21 @@ def test_decode_fp8_gemm1_bytes_closed_form():
     assert st["gemm1_bytes"] == n * (2 * I * H + (2 * I // 128) * (H // 128) * 4) + P * (H + I + (H // 128 + I // 128) * 4)
     # the figures the bench line reports for this layer (165 experts touched)
     assert (n, st["gemm1_bytes"], st["weight_bytes"]) == (165, 4_848_036_864, 7_268_405_760)
+
+
+def test_small_layers_are_timed_l2_cold():
+    """The bench flushes the L2 between timed calls of a layer whose weight
+    stream is under 8 x the 126 MB L2: the tiny and Zipf decode layers
+    (their weights fit, wholly or mostly, in the L2); the others stream
+    gigabytes per call and are not flushed."""
+    flushed = {}
+    for i, cfg in enumerate(synth.CONFIGS + synth.EXTRA_CONFIGS):
+        ids, _ = synth.make_routing(cfg["T"], cfg["E"], cfg["k"], cfg.get("routing", "uniform"), synth.config_seed(i))
+
+        class Shape:
+            T, H, E, k, I, wfmt = cfg["T"], cfg["H"], cfg["E"], cfg["k"], cfg["I"], cfg["wfmt"]
+            n_shared = cfg.get("n_shared", 0)
+
+        flushed[cfg["name"]] = bench.workload_stats(Shape, ids)["weight_bytes"] < bench.FLUSH_BELOW_BYTES
+    assert {n for n, f in flushed.items() if f} == {synth.CONFIGS[0]["name"], synth.CONFIGS[3]["name"]}
+    assert bench.FLUSH_BELOW_BYTES == 8 * bench.L2_BYTES and bench.L2_BYTES >= 126 * 10**6
