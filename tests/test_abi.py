@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from fp4_block_scaled_route_b200 import build as moe_build
 from fp4_block_scaled_route_b200 import moe
@@ -63,6 +64,13 @@ def test_host_argument_checks_without_gpu(libmoe):
     assert libmoe.moe_forward(None, 1, None, None, None, None, None, None, None, None, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_pack_mxfp4_scales(None, None, 128, 128, None) == moe.MOE_ERR_INVALID_ARG
     assert libmoe.moe_set_fault_injection(None, 1) == moe.MOE_ERR_INVALID_ARG
+    if not torch.cuda.is_available():
+        # valid arguments on a machine with no GPU: a CUDA error, no context, no crash
+        ctx = ctypes.c_void_p(1)
+        assert libmoe.moe_create(256, 128, 8, 2, 0, ctypes.byref(ctx)) == moe.MOE_ERR_CUDA and ctx.value is None
+        ctx = ctypes.c_void_p(1)
+        assert libmoe.moe_create_ex(256, 128, 8, 2, 1, 16, 1, ctypes.byref(ctx)) == moe.MOE_ERR_CUDA
+        assert ctx.value is None
 
 
 def test_product_path_does_not_use_the_oracle():
